@@ -1,0 +1,210 @@
+/*
+ * mk.h -- C ABI of the persistent decode megakernel for B200 (sm_100a).
+ *
+ * One decode step of a Llama-style dense decoder (RMSNorm + QKV + RoPE, GQA
+ * attention over a paged bf16 KV cache, O-projection + residual, RMSNorm +
+ * SwiGLU gate/up, down-projection + residual, final norm + LM head + greedy
+ * argmax) runs as ONE persistent kernel launch: every SM walks its own
+ * precomputed instruction tape, instructions wait on global-memory counters
+ * instead of kernel boundaries, and shared memory is a ring of pages into which
+ * the next instructions' weights are streamed while the current one computes.
+ *
+ * Sources of the method: the Hazy Research megakernel article "Stanford team's
+ * new work lets Llama-1B reach millisecond inference" (m.youleyou.com/wenzhang/
+ * 2897217), section "Megakernel: a deep-fusion design from scratch": one kernel
+ * for the whole forward; an on-GPU instruction interpreter; a per-SM execution
+ * plan of fused instructions (RMSNorm+QKV+RoPE, attention, MLP); dependencies
+ * resolved before the run; paged shared memory so the next stage preloads its
+ * weights; completion counters in global memory (atomic +1, waiters spin until
+ * a preset value) instead of global barriers.  The interface below is this
+ * library's own; the pages define none.
+ *
+ * Conventions
+ *  - All weights are caller-owned DEVICE pointers to bf16, row-major [out, in],
+ *    and must stay valid (and unmodified) for the life of the handle.
+ *  - Output buffers are caller-owned; the library owns the KV cache, the
+ *    scratch activations, the counters and the tapes.
+ *  - Calls return an mk_status and never abort the process.  Kernel launches
+ *    are asynchronous on the given stream; device-side failures (a bounded wait
+ *    that ran out, an out-of-range token) are recorded in a device error word
+ *    and reported by mk_sync / mk_get_error.  After such a failure every later
+ *    step returns at once until mk_clear_error is called.
+ *  - One step at a time per handle: steps of one handle must be ordered on one
+ *    stream (or otherwise serialised); two handles may run concurrently.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ */
+#ifndef MK_H
+#define MK_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct mk_ctx* mk_handle;
+
+typedef enum {
+  MK_OK = 0,
+  MK_ERR_INVALID_ARG = 1,   /* a NULL pointer, a size or index out of range */
+  MK_ERR_UNSUPPORTED = 2,   /* a shape this build does not handle (see mk_create) */
+  MK_ERR_OOM = 3,           /* device allocation failed */
+  MK_ERR_CUDA = 4,          /* a CUDA runtime call failed (no device, launch error) */
+  MK_ERR_TIMEOUT = 5,       /* a bounded wait inside the kernel ran out */
+  MK_ERR_DEVICE_FAULT = 6,  /* the kernel reported bad input (e.g. token >= vocab) */
+  MK_ERR_ABORTED = 7        /* an earlier device error is pending; see mk_clear_error */
+} mk_status;
+
+/* Model shape and capacity.  Requirements checked by mk_create:
+ *   head_dim in {64, 128}; n_heads % n_kv_heads == 0 with n_heads/n_kv_heads
+ *   in {1, 2, 4, 8}; hidden, ffn multiples of 8; hidden <= 4096 and
+ *   n_heads*head_dim <= 8192 (two rows of Wq/Wgate, one row of Wo, fit a
+ *   16 KiB page);
+ *   1 <= max_batch <= 8; B * max(hidden, n_heads*head_dim) <= 16384 where B is
+ *   max_batch rounded up to 1, 2, 4 or 8.
+ * RoPE rotates half-split pairs (i, i + head_dim/2) by pos * inv_freq[i],
+ * inv_freq[i] = rope_theta^(-2i/head_dim); with rope_scaling != 0 the Llama-3
+ * rule (rope_factor, rope_low_freq, rope_high_freq, rope_orig_max) rescales
+ * long wavelengths. */
+typedef struct {
+  int32_t n_layers;
+  int32_t hidden;
+  int32_t n_heads;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t ffn;
+  int32_t vocab;
+  int32_t tied;            /* 1: LM head is the embedding matrix */
+  float rms_eps;
+  float rope_theta;
+  int32_t rope_scaling;    /* 0: none, 1: Llama-3 frequency scaling */
+  float rope_factor;
+  float rope_low_freq;
+  float rope_high_freq;
+  int32_t rope_orig_max;
+  int32_t max_batch;       /* sequence slots 0..max_batch-1 */
+  int32_t max_seq;         /* positions 0..max_seq-1 per slot */
+} mk_config;
+
+/* Device pointers (bf16).  The per-layer members are HOST arrays of n_layers
+ * device pointers; mk_create copies them. */
+typedef struct {
+  const void* embed;        /* [vocab, hidden] */
+  const void* lm_head;      /* [vocab, hidden]; NULL iff tied */
+  const void* final_norm;   /* [hidden] */
+  const void* const* attn_norm;  /* [hidden] each */
+  const void* const* wq;         /* [n_heads*head_dim, hidden] */
+  const void* const* wk;         /* [n_kv_heads*head_dim, hidden] */
+  const void* const* wv;         /* [n_kv_heads*head_dim, hidden] */
+  const void* const* wo;         /* [hidden, n_heads*head_dim] */
+  const void* const* mlp_norm;   /* [hidden] */
+  const void* const* w_gate;     /* [ffn, hidden] */
+  const void* const* w_up;       /* [ffn, hidden] */
+  const void* const* w_down;     /* [hidden, ffn] */
+} mk_weights;
+
+/* Optional knobs (pass NULL for defaults). */
+typedef struct {
+  int32_t device;            /* CUDA device ordinal (default 0) */
+  int32_t wait_limit_ms;     /* bound of every in-kernel wait (default 1000) */
+  int32_t n_sm;              /* SMs to use (0 = all) */
+  int32_t ring_pages;        /* shared-memory pages in the weight ring (0 = as many as fit) */
+  int32_t debug_fault;       /* test hook, 0 in normal use.  1: raise the wait target of
+                                one instruction by one, so that wait can never be met and
+                                runs out after wait_limit_ms (the step then reports
+                                MK_ERR_TIMEOUT and the context stays usable) */
+  int32_t profile;           /* 1: every step records per-instruction timestamps
+                                (see mk_profile_read); costs a few stores per instruction */
+} mk_options;
+
+/* Create a handle: validates the config, lowers it into per-SM instruction
+ * tapes (one set per active batch size 1..max_batch), allocates the KV cache
+ * (bf16, pages of 16 KiB per layer and kv head) and scratch, zeroes them.
+ * Returns MK_ERR_INVALID_ARG / MK_ERR_UNSUPPORTED before touching the GPU when
+ * the config or pointers are bad. */
+mk_status mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt,
+                    mk_handle* out);
+
+/* Run one decode step for lanes b = 0..nb-1, lane b using sequence slot b.
+ *   tokens_dev    device int32[nb]: the input token of each lane (may be the
+ *                 previous step's ids_dev, so steps chain without a host sync)
+ *   positions     HOST int32[nb]: absolute position of that token; slot b's
+ *                 cache must hold positions 0..pos-1
+ *   logits_dev    device float[nb, vocab] or NULL (not written)
+ *   ids_dev       device int32[nb]: greedy argmax, lowest index on ties
+ * Writes K/V of each lane's position into its slot.  Asynchronous. */
+mk_status mk_decode_step(mk_handle h, int32_t nb, const int32_t* tokens_dev,
+                         const int32_t* positions, float* logits_dev, int32_t* ids_dev,
+                         void* stream);
+
+/* The same step with HOST buffers: copies tokens in, runs the step, copies ids
+ * (and logits when logits_host != NULL, float[nb, vocab]) back, and waits for
+ * the stream.  Returns the step's device status. */
+mk_status mk_decode_step_host(mk_handle h, int32_t nb, const int32_t* tokens_host,
+                              const int32_t* positions, float* logits_host,
+                              int32_t* ids_host, void* stream);
+
+/* Prefill sequence slot `seq` with n HOST tokens at positions start_pos ..
+ * start_pos+n-1, one decode step per token.  logits_last_dev (device
+ * float[vocab], nullable) and id_last_host (host int32*, nullable) receive the
+ * last position's logits and greedy id; when id_last_host is non-NULL the call
+ * waits for the stream.  The prompt is copied before the call returns. */
+mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_host, int32_t n,
+                     int32_t start_pos, float* logits_last_dev, int32_t* id_last_host,
+                     void* stream);
+
+/* Wait for `stream` and return the device status of the steps run so far. */
+mk_status mk_sync(mk_handle h, void* stream);
+
+/* Decode the device error word into `buf` (always NUL-terminated); returns the
+ * status it maps to.  Synchronises the device. */
+mk_status mk_get_error(mk_handle h, char* buf, int32_t len);
+
+/* Clear a recorded device error, the abort flag and all counters. */
+mk_status mk_clear_error(mk_handle h);
+
+/* Profile records of the last step (handle created with mk_options.profile = 1).
+ * Layout: int64 out[n_sm][stride][8]; record i of SM s describes the i-th
+ * instruction of that SM's tape: [0] op | layer << 8 | n_units << 24,
+ * [1] consumer start, [2] dependency met, [3] units done, [4] counter signalled,
+ * [5] producer issued the first unit's page, [6] producer issued the last
+ * unit's page, [7] unused -- all %globaltimer nanoseconds, 0 where not reached.
+ * `cap` is the capacity of `out` in int64 elements; *n_sm and *stride are set
+ * even when out is NULL, so a first call can size the buffer.  Synchronises
+ * the device. */
+mk_status mk_profile_read(mk_handle h, int64_t* out, int64_t cap, int32_t* n_sm, int32_t* stride);
+
+/* Free everything the library owns (never the caller's weights or outputs). */
+mk_status mk_destroy(mk_handle h);
+
+/* ---- host-only introspection (no GPU needed) ---- */
+
+typedef struct {
+  int32_t n_instr_total;     /* instructions over all SMs */
+  int32_t n_counters;        /* counters per set */
+  int32_t max_instr_per_sm;
+  int64_t bytes_min_sm;      /* weight + estimated KV bytes streamed per SM */
+  int64_t bytes_max_sm;
+  int32_t deadlock_free;     /* 1 if the tape simulator ran every instruction */
+  int32_t coverage_ok;       /* 1 if every output tile is produced exactly once */
+  int32_t targets_ok;        /* 1 if every wait target equals its counter's signal count */
+  int32_t attn_slices;       /* attention slices per (lane, kv head) */
+  int32_t ring_pages;        /* pages the kernel would use for this shape */
+  int32_t smem_bytes;        /* dynamic shared memory per CTA */
+} mk_plan_report;
+
+/* Lower `cfg` for `n_sm` SMs and `nb` active lanes, run the CPU tape simulator
+ * over the result and fill `rep`.  `fault` != 0 plants a fault in the tape
+ * first (1: one signal dropped, 2: one wait target raised by one) so tests can
+ * see the simulator report it. */
+mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
+                        mk_plan_report* rep);
+
+/* Library version string (static storage). */
+const char* mk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MK_H */

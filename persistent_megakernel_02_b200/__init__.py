@@ -1,0 +1,262 @@
+"""Persistent decode megakernel for B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI in ``include/mk.h``.  It only marshals
+arguments -- every step of the decode path runs in the CUDA library
+``libmk.so`` built from ``csrc/`` (``python -m persistent_megakernel_02_b200.build``).
+There is no fallback: if the library is missing or a call fails, an
+:class:`MkError` is raised.
+
+PyTorch is used by callers for device memory and streams; this module only
+reads ``tensor.data_ptr()`` and stream handles.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+from .build import LIB
+
+__all__ = ["Megakernel", "MkError", "plan_check", "version", "lib", "STATUS"]
+
+STATUS = {
+    0: "MK_OK",
+    1: "MK_ERR_INVALID_ARG",
+    2: "MK_ERR_UNSUPPORTED",
+    3: "MK_ERR_OOM",
+    4: "MK_ERR_CUDA",
+    5: "MK_ERR_TIMEOUT",
+    6: "MK_ERR_DEVICE_FAULT",
+    7: "MK_ERR_ABORTED",
+}
+
+
+class MkError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+
+
+class MkConfig(ctypes.Structure):
+    _fields_ = [
+        ("n_layers", ctypes.c_int32), ("hidden", ctypes.c_int32), ("n_heads", ctypes.c_int32),
+        ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("ffn", ctypes.c_int32),
+        ("vocab", ctypes.c_int32), ("tied", ctypes.c_int32), ("rms_eps", ctypes.c_float),
+        ("rope_theta", ctypes.c_float), ("rope_scaling", ctypes.c_int32),
+        ("rope_factor", ctypes.c_float), ("rope_low_freq", ctypes.c_float),
+        ("rope_high_freq", ctypes.c_float), ("rope_orig_max", ctypes.c_int32),
+        ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32),
+    ]
+
+
+_PP = ctypes.POINTER(ctypes.c_void_p)
+
+
+class MkWeights(ctypes.Structure):
+    _fields_ = [
+        ("embed", ctypes.c_void_p), ("lm_head", ctypes.c_void_p), ("final_norm", ctypes.c_void_p),
+        ("attn_norm", _PP), ("wq", _PP), ("wk", _PP), ("wv", _PP), ("wo", _PP),
+        ("mlp_norm", _PP), ("w_gate", _PP), ("w_up", _PP), ("w_down", _PP),
+    ]
+
+
+class MkOptions(ctypes.Structure):
+    _fields_ = [
+        ("device", ctypes.c_int32), ("wait_limit_ms", ctypes.c_int32), ("n_sm", ctypes.c_int32),
+        ("ring_pages", ctypes.c_int32), ("debug_fault", ctypes.c_int32),
+        ("profile", ctypes.c_int32),
+    ]
+
+
+class MkPlanReport(ctypes.Structure):
+    _fields_ = [
+        ("n_instr_total", ctypes.c_int32), ("n_counters", ctypes.c_int32),
+        ("max_instr_per_sm", ctypes.c_int32), ("bytes_min_sm", ctypes.c_int64),
+        ("bytes_max_sm", ctypes.c_int64), ("deadlock_free", ctypes.c_int32),
+        ("coverage_ok", ctypes.c_int32), ("targets_ok", ctypes.c_int32),
+        ("attn_slices", ctypes.c_int32), ("ring_pages", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int32),
+    ]
+
+
+# exported entry points and their signatures (kept in step with include/mk.h)
+_SIGS = {
+    "mk_create": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.POINTER(MkWeights),
+                                 ctypes.POINTER(MkOptions), ctypes.POINTER(ctypes.c_void_p)]),
+    "mk_decode_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                      ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p,
+                                      ctypes.c_void_p, ctypes.c_void_p]),
+    "mk_decode_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32,
+                                           ctypes.POINTER(ctypes.c_int32),
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p,
+                                           ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
+    "mk_prefill": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                  ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p]),
+    "mk_sync": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "mk_get_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int32]),
+    "mk_clear_error": (ctypes.c_int, [ctypes.c_void_p]),
+    "mk_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "mk_plan_check": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.c_int32, ctypes.POINTER(MkPlanReport)]),
+    "mk_profile_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_int32),
+                                       ctypes.POINTER(ctypes.c_int32)]),
+    "mk_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmk.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise MkError(4, f"{LIB} is missing; build it with "
+                             "`python -m persistent_megakernel_02_b200.build`")
+        handle = ctypes.CDLL(LIB)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def version() -> str:
+    return lib().mk_version().decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise MkError(status, what)
+
+
+_CFG_FIELDS = [f for f, _ in MkConfig._fields_]
+
+
+def config_struct(cfg: dict) -> MkConfig:
+    return MkConfig(**{k: cfg[k] for k in _CFG_FIELDS})
+
+
+def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0) -> dict:
+    """Lower ``cfg`` on the host and run the tape simulator (no GPU needed)."""
+    rep = MkPlanReport()
+    c = config_struct(cfg)
+    _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, ctypes.byref(rep)), "mk_plan_check")
+    return {f: getattr(rep, f) for f, _ in MkPlanReport._fields_}
+
+
+def _i32_array(values):
+    vals = [int(v) for v in values]
+    return (ctypes.c_int32 * max(1, len(vals)))(*vals)
+
+
+def _stream_handle(stream):
+    if stream is None:
+        return None
+    return ctypes.c_void_p(getattr(stream, "cuda_stream", stream))
+
+
+class Megakernel:
+    """One decoder handle over caller-owned bf16 CUDA weights.
+
+    ``weights`` is the dict of :func:`synth.make_weights` layout: 'embed',
+    'lm_head' (None when tied), 'final_norm' and per-layer lists 'attn_norm',
+    'wq', 'wk', 'wv', 'wo', 'mlp_norm', 'w_gate', 'w_up', 'w_down' -- contiguous
+    bf16 CUDA tensors.  The handle keeps references to them.
+    """
+
+    _LAYER = ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")
+
+    def __init__(self, cfg: dict, weights: dict, device: int = 0, wait_limit_ms: int = 1000,
+                 n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0):
+        self.cfg = dict(cfg)
+        self._weights = weights
+        self._arrays = {}
+        for name in self._LAYER:
+            ptrs = [t.data_ptr() for t in weights[name]]
+            self._arrays[name] = (ctypes.c_void_p * len(ptrs))(*ptrs)
+        w = MkWeights(
+            embed=weights["embed"].data_ptr(),
+            lm_head=None if weights.get("lm_head") is None else weights["lm_head"].data_ptr(),
+            final_norm=weights["final_norm"].data_ptr(),
+            **{n: ctypes.cast(self._arrays[n], _PP) for n in self._LAYER},
+        )
+        opt = MkOptions(device=device, wait_limit_ms=wait_limit_ms, n_sm=n_sm,
+                        ring_pages=ring_pages, debug_fault=debug_fault, profile=profile)
+        self._cfg_struct = config_struct(cfg)
+        h = ctypes.c_void_p()
+        _check(lib().mk_create(ctypes.byref(self._cfg_struct), ctypes.byref(w), ctypes.byref(opt),
+                               ctypes.byref(h)), "mk_create")
+        self._h = h
+
+    # -- steps ------------------------------------------------------------
+    def decode_step(self, tokens, positions, ids, logits=None, stream=None):
+        """Asynchronous step over device tensors (tokens/ids int32 [nb], logits f32 [nb, V])."""
+        nb = len(positions)
+        _check(lib().mk_decode_step(self._h, nb, tokens.data_ptr(), _i32_array(positions),
+                                    None if logits is None else logits.data_ptr(), ids.data_ptr(),
+                                    _stream_handle(stream)), "mk_decode_step")
+
+    def decode_step_host(self, tokens, positions, want_logits=False, stream=None):
+        """Step over host buffers; returns (ids list, logits numpy [nb, V] or None)."""
+        import numpy as np
+
+        nb = len(positions)
+        ids = (ctypes.c_int32 * nb)()
+        lg = np.empty((nb, self.cfg["vocab"]), dtype=np.float32) if want_logits else None
+        _check(lib().mk_decode_step_host(
+            self._h, nb, _i32_array(tokens), _i32_array(positions),
+            None if lg is None else lg.ctypes.data_as(ctypes.c_void_p), ids,
+            _stream_handle(stream)), "mk_decode_step_host")
+        return list(ids), lg
+
+    def prefill(self, seq, tokens, start_pos=0, logits_last=None, want_id=True, stream=None):
+        """Run the prompt of slot ``seq`` token by token; returns the last greedy id."""
+        toks = _i32_array(tokens)
+        out = ctypes.c_int32(-1)
+        _check(lib().mk_prefill(self._h, seq, toks, len(tokens), start_pos,
+                                None if logits_last is None else logits_last.data_ptr(),
+                                ctypes.byref(out) if want_id else None, _stream_handle(stream)),
+               "mk_prefill")
+        return out.value if want_id else None
+
+    def profile_records(self):
+        """Per-instruction timestamps of the last step: int64 array [n_sm, stride, 8]."""
+        import numpy as np
+
+        n_sm, stride = ctypes.c_int32(), ctypes.c_int32()
+        lib().mk_profile_read(self._h, None, 0, ctypes.byref(n_sm), ctypes.byref(stride))
+        out = np.zeros((n_sm.value, stride.value, 8), dtype=np.int64)
+        _check(lib().mk_profile_read(self._h, out.ctypes.data_as(ctypes.c_void_p), out.size,
+                                     ctypes.byref(n_sm), ctypes.byref(stride)), "mk_profile_read")
+        return out
+
+    def sync(self, stream=None):
+        _check(lib().mk_sync(self._h, _stream_handle(stream)), "mk_sync")
+
+    def status(self, stream=None) -> int:
+        """mk_sync's status without raising."""
+        return lib().mk_sync(self._h, _stream_handle(stream))
+
+    def error_string(self) -> str:
+        buf = ctypes.create_string_buffer(256)
+        lib().mk_get_error(self._h, buf, 256)
+        return buf.value.decode()
+
+    def clear_error(self):
+        _check(lib().mk_clear_error(self._h), "mk_clear_error")
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().mk_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,506 @@
+// mk_api.cu -- the C ABI (include/mk.h): handle creation, tapes upload, one
+// cooperative launch of the persistent kernel per decode step, prefill as a
+// sequence of steps, error reporting, and the host-only tape checker.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/mk.h"
+#include "mk_kernel.cuh"
+#include "mk_plan.h"
+
+using namespace mk;
+
+struct mk_ctx {
+  mk_config cfg{};
+  Dims D{};
+  int dev = 0, n_sm = 0, nbt = 1;
+  unsigned long long wait_limit_ns = 1000000000ull;
+  SmemLayout sm{};
+  std::vector<Tape> tapes;  // index nb - 1
+  struct DevTape {
+    Instr* instrs = nullptr;
+    uint32_t* sm_off = nullptr;
+    uint32_t* units = nullptr;
+  };
+  std::vector<DevTape> dtapes;
+  LayerW* d_layers = nullptr;
+  const uint16_t *embed = nullptr, *lm = nullptr, *final_norm = nullptr;
+  float *x = nullptr, *q = nullptr, *o = nullptr, *a = nullptr, *part = nullptr;
+  int2* lm_part = nullptr;
+  uint16_t *kcache = nullptr, *vcache = nullptr;
+  int* page_table = nullptr;
+  uint32_t* counters = nullptr;
+  int n_counters = 0;
+  ErrWord* err = nullptr;
+  float2* rope = nullptr;
+  int* tok_stage = nullptr;
+  int tok_stage_cap = 0;
+  int* ids_scratch = nullptr;
+  float* logits_scratch = nullptr;
+  unsigned long long step = 0;
+  long long* prof = nullptr;
+  int prof_stride = 0;
+  std::vector<void*> allocs;
+};
+
+static const char* kVersion = "mk 0.1 (sm_100a persistent decode megakernel)";
+
+extern "C" const char* mk_version(void) { return kVersion; }
+
+namespace {
+
+mk_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return MK_OK;
+  if (e == cudaErrorMemoryAllocation) return MK_ERR_OOM;
+  return MK_ERR_CUDA;
+}
+
+#define MK_TRY(expr)                               \
+  do {                                             \
+    mk_status _s = (expr);                         \
+    if (_s != MK_OK) return _s;                    \
+  } while (0)
+
+template <class T>
+mk_status dalloc(mk_ctx* h, T** p, size_t count) {
+  void* v = nullptr;
+  size_t bytes = count * sizeof(T);
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(&v, bytes);
+  if (e != cudaSuccess) return from_cuda(e);
+  h->allocs.push_back(v);
+  cudaError_t z = cudaMemset(v, 0, bytes);
+  if (z != cudaSuccess) return from_cuda(z);
+  *p = static_cast<T*>(v);
+  return MK_OK;
+}
+
+std::string dims_from_config(const mk_config* c, int n_sm, Dims* D) {
+  if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return "rms_eps must be finite and >= 0";
+  if (!(c->rope_theta > 0.f)) return "rope_theta must be positive";
+  if (c->rope_scaling) {
+    if (!(c->rope_factor > 0.f) || !(c->rope_low_freq > 0.f) || !(c->rope_high_freq > c->rope_low_freq) ||
+        c->rope_orig_max <= 0)
+      return "invalid Llama-3 rope scaling parameters";
+  }
+  return derive_dims(c->n_layers, c->hidden, c->n_heads, c->n_kv_heads, c->head_dim, c->ffn, c->vocab,
+                     c->tied, c->rms_eps, c->max_batch, c->max_seq, n_sm, D);
+}
+
+// inverse frequencies theta^(-2i/d) with the optional Llama-3 rescaling of long wavelengths
+std::vector<double> inv_freq(const mk_config* c) {
+  const int half = c->head_dim / 2;
+  std::vector<double> f(half);
+  const double pi = 3.14159265358979323846;
+  for (int i = 0; i < half; ++i) {
+    double base = std::pow((double)c->rope_theta, -2.0 * i / c->head_dim);
+    if (c->rope_scaling) {
+      const double lo = c->rope_low_freq, hi = c->rope_high_freq, orig = c->rope_orig_max;
+      const double wl = 2.0 * pi / base;
+      if (wl > orig / lo) {
+        base = base / c->rope_factor;
+      } else if (wl >= orig / hi) {
+        const double t = (orig / wl - lo) / (hi - lo);
+        base = (1.0 - t) * base / c->rope_factor + t * base;
+      }
+    }
+    f[i] = base;
+  }
+  return f;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+mk_status check_weights(const mk_config* c, const mk_weights* w) {
+  if (!w->embed || !w->final_norm) return MK_ERR_INVALID_ARG;
+  if (c->tied ? (w->lm_head != nullptr) : (w->lm_head == nullptr)) return MK_ERR_INVALID_ARG;
+  if (!aligned16(w->embed) || !aligned16(w->final_norm) || (w->lm_head && !aligned16(w->lm_head)))
+    return MK_ERR_INVALID_ARG;
+  const void* const* arrs[] = {w->attn_norm, w->wq, w->wk, w->wv, w->wo,
+                               w->mlp_norm, w->w_gate, w->w_up, w->w_down};
+  for (auto a : arrs) {
+    if (!a) return MK_ERR_INVALID_ARG;
+    for (int l = 0; l < c->n_layers; ++l)
+      if (!a[l] || !aligned16(a[l])) return MK_ERR_INVALID_ARG;
+  }
+  return MK_OK;
+}
+
+mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
+  const Dims& D = h->D;
+  // tapes, one per active batch size
+  for (int nb = 1; nb <= D.max_batch; ++nb) {
+    h->tapes.push_back(lower(D, h->n_sm, nb));
+    const Tape& t = h->tapes.back();
+    mk_ctx::DevTape dt;
+    MK_TRY(dalloc(h, &dt.instrs, t.instrs.size()));
+    MK_TRY(dalloc(h, &dt.sm_off, t.sm_off.size()));
+    MK_TRY(dalloc(h, &dt.units, t.units.size()));
+    MK_TRY(from_cuda(cudaMemcpy(dt.instrs, t.instrs.data(), t.instrs.size() * sizeof(Instr), cudaMemcpyHostToDevice)));
+    MK_TRY(from_cuda(cudaMemcpy(dt.sm_off, t.sm_off.data(), t.sm_off.size() * 4, cudaMemcpyHostToDevice)));
+    if (!t.units.empty())
+      MK_TRY(from_cuda(cudaMemcpy(dt.units, t.units.data(), t.units.size() * 4, cudaMemcpyHostToDevice)));
+    h->dtapes.push_back(dt);
+  }
+  // weights
+  std::vector<LayerW> lw(D.L);
+  for (int l = 0; l < D.L; ++l) {
+    lw[l].attn_norm = (const uint16_t*)w->attn_norm[l];
+    lw[l].wq = (const uint16_t*)w->wq[l];
+    lw[l].wk = (const uint16_t*)w->wk[l];
+    lw[l].wv = (const uint16_t*)w->wv[l];
+    lw[l].wo = (const uint16_t*)w->wo[l];
+    lw[l].mlp_norm = (const uint16_t*)w->mlp_norm[l];
+    lw[l].w_gate = (const uint16_t*)w->w_gate[l];
+    lw[l].w_up = (const uint16_t*)w->w_up[l];
+    lw[l].w_down = (const uint16_t*)w->w_down[l];
+  }
+  MK_TRY(dalloc(h, &h->d_layers, D.L));
+  MK_TRY(from_cuda(cudaMemcpy(h->d_layers, lw.data(), D.L * sizeof(LayerW), cudaMemcpyHostToDevice)));
+  h->embed = (const uint16_t*)w->embed;
+  h->lm = D.tied ? h->embed : (const uint16_t*)w->lm_head;
+  h->final_norm = (const uint16_t*)w->final_norm;
+  // scratch and state
+  const int S1 = h->tapes[0].S;  // nb = 1 has the most slices
+  MK_TRY(dalloc(h, &h->x, (size_t)kMaxNB * D.H));
+  MK_TRY(dalloc(h, &h->q, (size_t)kMaxNB * D.qdim));
+  MK_TRY(dalloc(h, &h->o, (size_t)kMaxNB * D.qdim));
+  MK_TRY(dalloc(h, &h->a, (size_t)kMaxNB * D.F));
+  MK_TRY(dalloc(h, &h->part, (size_t)kMaxNB * D.Hkv * S1 * D.rep * (D.d + 2)));
+  MK_TRY(dalloc(h, &h->lm_part, (size_t)h->n_sm * kMaxNB));
+  const size_t kv = (size_t)D.L * D.n_phys_pages * D.Hkv * D.PL * D.d;
+  MK_TRY(dalloc(h, &h->kcache, kv));
+  MK_TRY(dalloc(h, &h->vcache, kv));
+  std::vector<int> pt((size_t)D.max_batch * D.pages_per_seq);
+  for (size_t i = 0; i < pt.size(); ++i) pt[i] = (int)i;  // slot s owns pages s*pps .. s*pps+pps-1
+  MK_TRY(dalloc(h, &h->page_table, pt.size()));
+  MK_TRY(from_cuda(cudaMemcpy(h->page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice)));
+  h->n_counters = n_counters(D);
+  MK_TRY(dalloc(h, &h->counters, (size_t)2 * h->n_counters));
+  MK_TRY(dalloc(h, &h->err, 1));
+  // RoPE table: cos/sin of pos * inv_freq[i], computed in double
+  const int half = D.d / 2;
+  std::vector<double> f = inv_freq(&h->cfg);
+  std::vector<float2> tab((size_t)D.max_seq * half);
+  for (int p = 0; p < D.max_seq; ++p)
+    for (int i = 0; i < half; ++i) {
+      const double ang = (double)p * f[i];
+      tab[(size_t)p * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+  MK_TRY(dalloc(h, &h->rope, tab.size()));
+  MK_TRY(from_cuda(cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice)));
+  MK_TRY(dalloc(h, &h->ids_scratch, kMaxNB));
+  // shared memory and kernel attributes
+  int max_dyn = 0;
+  MK_TRY(from_cuda(cudaDeviceGetAttribute(&max_dyn, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev)));
+  h->sm = smem_layout(D, h->nbt, max_dyn, want_pages);
+  if (h->sm.ring_pages < 2) return MK_ERR_UNSUPPORTED;
+  if (h->sm.ring_pages > 64) return MK_ERR_UNSUPPORTED;
+  const void* kfn[4] = {(const void*)mk_decode_kernel<1>, (const void*)mk_decode_kernel<2>,
+                        (const void*)mk_decode_kernel<4>, (const void*)mk_decode_kernel<8>};
+  for (auto k : kfn)
+    MK_TRY(from_cuda(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, h->sm.total)));
+  int blocks = 0;
+  MK_TRY(from_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, mk_decode_kernel<8>, kThreads,
+                                                                  h->sm.total)));
+  if (blocks < 1) return MK_ERR_UNSUPPORTED;
+  return from_cuda(cudaDeviceSynchronize());
+}
+
+const void* kernel_for(int nbt) {
+  switch (nbt) {
+    case 1: return (const void*)mk_decode_kernel<1>;
+    case 2: return (const void*)mk_decode_kernel<2>;
+    case 4: return (const void*)mk_decode_kernel<4>;
+    default: return (const void*)mk_decode_kernel<8>;
+  }
+}
+
+mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, const int* slot,
+                      float* logits, int* ids, cudaStream_t st) {
+  const Dims& D = h->D;
+  const Tape& t = h->tapes[nb - 1];
+  const mk_ctx::DevTape& dt = h->dtapes[nb - 1];
+  KParams p{};
+  p.instrs = dt.instrs;
+  p.sm_off = dt.sm_off;
+  p.units = dt.units;
+  p.S = t.S;
+  p.layers = h->d_layers;
+  p.embed = h->embed;
+  p.lm_head = h->lm;
+  p.final_norm = h->final_norm;
+  p.x = h->x; p.q = h->q; p.o = h->o; p.a = h->a; p.part = h->part; p.lm_part = h->lm_part;
+  p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
+  const int par = (int)(h->step & 1);
+  p.ctr = h->counters + (size_t)par * h->n_counters;
+  p.ctr_next = h->counters + (size_t)(1 - par) * h->n_counters;
+  p.n_counters = h->n_counters;
+  p.err = h->err;
+  p.rope = h->rope;
+  p.nb = nb;
+  p.tokens = tokens_dev;
+  for (int b = 0; b < kMaxNB; ++b) {
+    p.pos[b] = b < nb ? pos[b] : 0;
+    p.slot[b] = b < nb ? slot[b] : 0;
+  }
+  p.logits = logits;
+  p.ids = ids;
+  p.wait_limit_ns = h->wait_limit_ns;
+  p.prof = h->prof;
+  p.prof_stride = h->prof_stride;
+  p.ring_pages = h->sm.ring_pages;
+  p.act_off = h->sm.ring_pages * kPageBytes;
+  p.bar_off = h->sm.bar_off;
+  p.misc_off = h->sm.misc_off;
+  p.D = D;
+  void* args[] = {&p};
+  const int nbt = lanes_template(nb);
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(nbt), dim3(h->n_sm), dim3(kThreads), args,
+                                              (size_t)h->sm.total, st);
+  h->step++;
+  return from_cuda(e);
+}
+
+mk_status read_error(mk_ctx* h, ErrWord* out) {
+  return from_cuda(cudaMemcpy(out, h->err, sizeof(ErrWord), cudaMemcpyDeviceToHost));
+}
+
+mk_status status_of(const ErrWord& e) {
+  switch (e.code) {
+    case 0: return e.abort ? MK_ERR_ABORTED : MK_OK;
+    case E_BAD_TOKEN: return MK_ERR_DEVICE_FAULT;
+    default: return MK_ERR_TIMEOUT;
+  }
+}
+
+}  // namespace
+
+extern "C" mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
+                                   mk_plan_report* rep) {
+  if (!cfg || !rep || n_sm < 1) return MK_ERR_INVALID_ARG;
+  memset(rep, 0, sizeof(*rep));
+  Dims D;
+  std::string why = dims_from_config(cfg, n_sm, &D);
+  if (!why.empty()) return MK_ERR_UNSUPPORTED;
+  if (nb < 1 || nb > D.max_batch) return MK_ERR_INVALID_ARG;
+  Tape t = lower(D, n_sm, nb);
+  if (fault == 1) {  // drop one signal: the first QKV instruction of the last layer
+    for (auto& I : t.instrs)
+      if (I.op == OP_QKV && I.layer == D.L - 1) { I.sig = kNoCounter; break; }
+  } else if (fault == 2) {  // raise one wait target
+    for (auto& I : t.instrs)
+      if (I.dep != kNoCounter) { I.dep_target += 1; break; }
+  }
+  SimReport r = simulate(D, n_sm, t);
+  rep->n_instr_total = r.n_instr_total;
+  rep->n_counters = t.n_counters;
+  rep->max_instr_per_sm = r.max_instr_per_sm;
+  rep->bytes_min_sm = r.bytes_min;
+  rep->bytes_max_sm = r.bytes_max;
+  rep->deadlock_free = r.deadlock_free;
+  rep->coverage_ok = r.coverage_ok;
+  rep->targets_ok = r.targets_ok;
+  rep->attn_slices = t.S;
+  SmemLayout s = smem_layout(D, lanes_template(D.max_batch), 232448, 0);
+  rep->ring_pages = s.ring_pages;
+  rep->smem_bytes = s.total;
+  return MK_OK;
+}
+
+extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt,
+                               mk_handle* out) {
+  if (!cfg || !w || !out) return MK_ERR_INVALID_ARG;
+  *out = nullptr;
+  mk_options o{};
+  if (opt) o = *opt;
+  if (o.wait_limit_ms < 0 || o.n_sm < 0 || o.ring_pages < 0 || o.device < 0) return MK_ERR_INVALID_ARG;
+  Dims D;
+  std::string why = dims_from_config(cfg, 148, &D);  // validation only; rederived below
+  if (!why.empty()) return MK_ERR_UNSUPPORTED;
+  MK_TRY(check_weights(cfg, w));
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) return MK_ERR_CUDA;
+  if (o.device >= ndev) return MK_ERR_INVALID_ARG;
+  MK_TRY(from_cuda(cudaSetDevice(o.device)));
+  int sms = 0, major = 0, coop = 0;
+  MK_TRY(from_cuda(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, o.device)));
+  MK_TRY(from_cuda(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, o.device)));
+  MK_TRY(from_cuda(cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, o.device)));
+  if (major != 10 || !coop) return MK_ERR_UNSUPPORTED;
+  mk_ctx* h = new mk_ctx();
+  h->cfg = *cfg;
+  h->dev = o.device;
+  h->n_sm = o.n_sm > 0 ? std::min(o.n_sm, sms) : sms;
+  h->wait_limit_ns = (unsigned long long)(o.wait_limit_ms > 0 ? o.wait_limit_ms : 1000) * 1000000ull;
+  why = dims_from_config(cfg, h->n_sm, &h->D);
+  h->nbt = lanes_template(cfg->max_batch);
+  mk_status s = why.empty() ? build(h, w, o.ring_pages) : MK_ERR_UNSUPPORTED;
+  if (s == MK_OK && o.profile) {
+    int stride = 1;
+    for (const Tape& t : h->tapes)
+      for (int sm = 0; sm < h->n_sm; ++sm) stride = std::max(stride, (int)(t.sm_off[sm + 1] - t.sm_off[sm]));
+    h->prof_stride = stride;
+    s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * 8);
+  }
+  if (s == MK_OK && o.debug_fault == 1) {
+    // test hook: one wait (the first layer-0 O projection of SM 0's tape for every
+    // batch size) gets a target one above what its counter can reach
+    for (size_t k = 0; k < h->tapes.size(); ++k) {
+      Tape& t = h->tapes[k];
+      for (uint32_t i = t.sm_off[0]; i < t.sm_off[1]; ++i)
+        if (t.instrs[i].dep != kNoCounter) {
+          t.instrs[i].dep_target += 1;
+          s = from_cuda(cudaMemcpy(h->dtapes[k].instrs + i, &t.instrs[i], sizeof(Instr), cudaMemcpyHostToDevice));
+          break;
+        }
+    }
+  }
+  if (s != MK_OK) {
+    mk_destroy(h);
+    return s;
+  }
+  *out = h;
+  return MK_OK;
+}
+
+extern "C" mk_status mk_destroy(mk_handle h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaSetDevice(h->dev);
+  cudaDeviceSynchronize();
+  for (void* p : h->allocs) cudaFree(p);
+  if (h->tok_stage) cudaFree(h->tok_stage);
+  if (h->logits_scratch) cudaFree(h->logits_scratch);
+  delete h;
+  return MK_OK;
+}
+
+extern "C" mk_status mk_decode_step(mk_handle h, int32_t nb, const int32_t* tokens_dev,
+                                    const int32_t* positions, float* logits_dev, int32_t* ids_dev,
+                                    void* stream) {
+  if (!h || !tokens_dev || !positions || !ids_dev) return MK_ERR_INVALID_ARG;
+  if (nb < 1 || nb > h->D.max_batch) return MK_ERR_INVALID_ARG;
+  int slot[kMaxNB];
+  for (int b = 0; b < nb; ++b) {
+    if (positions[b] < 0 || positions[b] >= h->D.max_seq) return MK_ERR_INVALID_ARG;
+    slot[b] = b;
+  }
+  cudaSetDevice(h->dev);
+  return launch_step(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream);
+}
+
+extern "C" mk_status mk_sync(mk_handle h, void* stream) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaSetDevice(h->dev);
+  MK_TRY(from_cuda(cudaStreamSynchronize((cudaStream_t)stream)));
+  ErrWord e;
+  MK_TRY(read_error(h, &e));
+  return status_of(e);
+}
+
+extern "C" mk_status mk_decode_step_host(mk_handle h, int32_t nb, const int32_t* tokens_host,
+                                         const int32_t* positions, float* logits_host,
+                                         int32_t* ids_host, void* stream) {
+  if (!h || !tokens_host || !positions || !ids_host) return MK_ERR_INVALID_ARG;
+  if (nb < 1 || nb > h->D.max_batch) return MK_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaSetDevice(h->dev);
+  if (h->tok_stage_cap < kMaxNB) {
+    if (h->tok_stage) cudaFree(h->tok_stage);
+    h->tok_stage = nullptr;
+    MK_TRY(from_cuda(cudaMalloc(&h->tok_stage, sizeof(int) * kMaxNB)));
+    h->tok_stage_cap = kMaxNB;
+  }
+  if (logits_host && !h->logits_scratch)
+    MK_TRY(from_cuda(cudaMalloc(&h->logits_scratch, sizeof(float) * (size_t)kMaxNB * h->D.V)));
+  MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_stage, tokens_host, sizeof(int) * nb, cudaMemcpyHostToDevice, st)));
+  MK_TRY(mk_decode_step(h, nb, h->tok_stage, positions, logits_host ? h->logits_scratch : nullptr,
+                        h->ids_scratch, stream));
+  MK_TRY(from_cuda(cudaMemcpyAsync(ids_host, h->ids_scratch, sizeof(int) * nb, cudaMemcpyDeviceToHost, st)));
+  if (logits_host)
+    MK_TRY(from_cuda(cudaMemcpyAsync(logits_host, h->logits_scratch, sizeof(float) * (size_t)nb * h->D.V,
+                                     cudaMemcpyDeviceToHost, st)));
+  return mk_sync(h, stream);
+}
+
+extern "C" mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_host, int32_t n,
+                                int32_t start_pos, float* logits_last_dev, int32_t* id_last_host,
+                                void* stream) {
+  if (!h || !tokens_host || n < 1) return MK_ERR_INVALID_ARG;
+  if (seq < 0 || seq >= h->D.max_batch || start_pos < 0 || (long long)start_pos + n > h->D.max_seq)
+    return MK_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (tokens_host[i] < 0 || tokens_host[i] >= h->D.V) return MK_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  cudaSetDevice(h->dev);
+  if (h->tok_stage_cap < n) {
+    MK_TRY(from_cuda(cudaStreamSynchronize(st)));
+    if (h->tok_stage) cudaFree(h->tok_stage);
+    h->tok_stage = nullptr;
+    h->tok_stage_cap = 0;
+    MK_TRY(from_cuda(cudaMalloc(&h->tok_stage, sizeof(int) * (size_t)std::max(n, kMaxNB))));
+    h->tok_stage_cap = std::max(n, kMaxNB);
+  }
+  // pageable source: the copy completes before the call returns
+  MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_stage, tokens_host, sizeof(int) * n, cudaMemcpyHostToDevice, st)));
+  MK_TRY(from_cuda(cudaStreamSynchronize(st)));
+  for (int i = 0; i < n; ++i) {
+    int pos = start_pos + i, slot = seq;
+    MK_TRY(launch_step(h, 1, h->tok_stage + i, &pos, &slot, i == n - 1 ? logits_last_dev : nullptr,
+                       h->ids_scratch, st));
+  }
+  if (id_last_host) {
+    MK_TRY(from_cuda(cudaMemcpyAsync(id_last_host, h->ids_scratch, sizeof(int), cudaMemcpyDeviceToHost, st)));
+    return mk_sync(h, stream);
+  }
+  return MK_OK;
+}
+
+extern "C" mk_status mk_profile_read(mk_handle h, int64_t* out, int64_t cap, int32_t* n_sm,
+                                     int32_t* stride) {
+  if (!h || !n_sm || !stride) return MK_ERR_INVALID_ARG;
+  *n_sm = h->n_sm;
+  *stride = h->prof_stride;
+  if (!h->prof) return MK_ERR_INVALID_ARG;
+  const int64_t need = (int64_t)h->n_sm * h->prof_stride * 8;
+  if (!out || cap < need) return MK_ERR_INVALID_ARG;
+  cudaSetDevice(h->dev);
+  MK_TRY(from_cuda(cudaDeviceSynchronize()));
+  return from_cuda(cudaMemcpy(out, h->prof, need * sizeof(int64_t), cudaMemcpyDeviceToHost));
+}
+
+extern "C" mk_status mk_get_error(mk_handle h, char* buf, int32_t len) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaSetDevice(h->dev);
+  MK_TRY(from_cuda(cudaDeviceSynchronize()));
+  ErrWord e;
+  MK_TRY(read_error(h, &e));
+  if (buf && len > 0) {
+    const char* what = "none";
+    switch (e.code) {
+      case E_WAIT_COUNTER: what = "counter wait timed out"; break;
+      case E_WAIT_FULL: what = "ring page arrival wait timed out"; break;
+      case E_WAIT_EMPTY: what = "ring page release wait timed out"; break;
+      case E_BAD_TOKEN: what = "token out of range"; break;
+      case E_DRAIN: what = "in-flight copy drain timed out"; break;
+      default: break;
+    }
+    snprintf(buf, (size_t)len, "%s (code %u, sm %u, instr %u, info %u, abort %u)", what, e.code, e.sm,
+             e.instr, e.info, e.abort);
+  }
+  return status_of(e);
+}
+
+extern "C" mk_status mk_clear_error(mk_handle h) {
+  if (!h) return MK_ERR_INVALID_ARG;
+  cudaSetDevice(h->dev);
+  MK_TRY(from_cuda(cudaDeviceSynchronize()));
+  MK_TRY(from_cuda(cudaMemset(h->err, 0, sizeof(ErrWord))));
+  MK_TRY(from_cuda(cudaMemset(h->counters, 0, sizeof(uint32_t) * 2 * h->n_counters)));
+  return from_cuda(cudaDeviceSynchronize());
+}

@@ -1,0 +1,892 @@
+// mk_kernel.cuh -- the persistent decode megakernel (sm_100a).
+//
+// One launch = one decode step of the whole model.  Grid = one CTA per SM
+// (cooperative launch, so all CTAs are co-resident), 288 threads:
+//   warp 0, lane 0   producer: walks this SM's tape and streams every unit's
+//                    weights (or KV pages) into a ring of 16 KiB shared-memory
+//                    pages with bulk copies, running ahead of the consumers and
+//                    across instruction boundaries -- weights do not depend on
+//                    activations, so they are fetched while the consumers are
+//                    still waiting on a counter (the "paged shared memory" of
+//                    the Hazy megakernel article, section "Megakernel: a
+//                    deep-fusion design from scratch");
+//   warps 1..8       consumers: for each instruction wait on its counter, stage
+//                    the activation vector (with RMSNorm where the op fuses
+//                    it), then each warp takes whole pages (units), computes
+//                    the bf16 x fp32 matvec on CUDA cores and runs the op's
+//                    epilogue; at the end one thread bumps the op's counter
+//                    (release), the completion counters of the same article.
+// Every wait is bounded (globaltimer); on timeout the CTA records an error word,
+// raises a global abort flag that every other waiter polls, drains its in-flight
+// copies and returns, so a bad tape cannot hang the GPU.
+#pragma once
+
+#include <math_constants.h>
+
+#include "mk_device.cuh"
+#include "mk_plan.h"
+
+namespace mk {
+
+struct LayerW {
+  const uint16_t* attn_norm;
+  const uint16_t* wq;
+  const uint16_t* wk;
+  const uint16_t* wv;
+  const uint16_t* wo;
+  const uint16_t* mlp_norm;
+  const uint16_t* w_gate;
+  const uint16_t* w_up;
+  const uint16_t* w_down;
+};
+
+struct ErrWord {
+  uint32_t code, sm, instr, info;
+  uint32_t abort;
+  uint32_t pad[3];
+};
+
+enum DevErr : uint32_t {
+  E_WAIT_COUNTER = 1,  // a counter did not reach its target in time
+  E_WAIT_FULL = 2,     // a ring page did not arrive in time
+  E_WAIT_EMPTY = 3,    // a ring page was not released in time
+  E_BAD_TOKEN = 4,     // a lane's token was outside [0, vocab) (treated as 0)
+  E_DRAIN = 5,         // in-flight copies did not land before exit
+};
+
+struct KParams {
+  // tape of this step's batch size
+  const Instr* instrs;
+  const uint32_t* sm_off;
+  const uint32_t* units;
+  int S;  // attention slices per (lane, kv head)
+  // weights
+  const LayerW* layers;
+  const uint16_t* embed;
+  const uint16_t* lm_head;  // == embed when tied
+  const uint16_t* final_norm;
+  // state
+  float* x;     // [8][H] residual stream
+  float* q;     // [8][qdim] rotated queries
+  float* o;     // [8][qdim] attention output
+  float* a;     // [8][F] silu(gate) * up
+  float* part;  // attention partials [8][Hkv][S][rep][d + 2]
+  int2* lm_part;  // [n_sm][8] best (value bits, index) per SM
+  uint16_t* kcache;
+  uint16_t* vcache;
+  const int* page_table;  // [max_batch][pages_per_seq]
+  uint32_t* ctr;          // counters of this step
+  uint32_t* ctr_next;     // counters of the next step (zeroed here)
+  int n_counters;
+  ErrWord* err;
+  const float2* rope;  // [max_seq][d/2] (cos, sin)
+  // step
+  int nb;
+  const int* tokens;  // device [nb]
+  int pos[kMaxNB];
+  int slot[kMaxNB];
+  float* logits;  // device [nb][V] or null
+  int* ids;       // device [nb]
+  unsigned long long wait_limit_ns;
+  long long* prof;   // profile records [n_sm][prof_stride][8] or null
+  int prof_stride;
+  // shared memory layout
+  int ring_pages, act_off, bar_off, misc_off;
+  Dims D;
+};
+
+struct Misc {
+  float red[kConsumerWarps][kMaxNB];
+  float lmv[kConsumerWarps][kMaxNB];
+  int lmi[kConsumerWarps][kMaxNB];
+  int tok[kMaxNB];
+  volatile int stop;
+  volatile int last;
+  uint32_t issued;
+  int entry_abort;
+};
+
+// ---------------------------------------------------------------- errors & waits
+
+__device__ __forceinline__ bool aborted(const KParams& p) { return ld_relaxed_u32(&p.err->abort) != 0; }
+
+__device__ __noinline__ void raise_error(const KParams& p, uint32_t code, uint32_t instr, uint32_t info,
+                                         bool abort) {
+  if (atomicCAS(&p.err->code, 0u, code) == 0u) {
+    p.err->sm = blockIdx.x;
+    p.err->instr = instr;
+    p.err->info = info;
+  }
+  __threadfence();
+  if (abort) atomicExch(&p.err->abort, 1u);
+}
+
+// Spin until *c >= target (acquire), the abort flag rises, or the time limit passes.
+__device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, uint32_t target,
+                                          uint32_t instr) {
+  if (ld_acquire_u32(c) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_u32(c) >= target) return true;
+    if ((it & 15) == 0) {
+      if (aborted(p)) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_COUNTER, instr, target, true);
+        return false;
+      }
+    }
+    if (it > 512) __nanosleep(32);
+  }
+}
+
+// Wait for an mbarrier phase.  honor_abort = false is used by the exit drain,
+// which must wait for copies in flight even after an abort.
+__device__ __forceinline__ bool wait_mbar(const KParams& p, uint64_t* bar, uint32_t parity,
+                                          uint32_t code, uint32_t instr, bool honor_abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 7) == 0) {
+      if (honor_abort && aborted(p)) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, code, instr, parity, true);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ size_t kv_offset(const KParams& p, int layer, int b, int page, int g) {
+  const Dims& D = p.D;
+  const int phys = p.page_table[p.slot[b] * D.pages_per_seq + page];
+  return (((size_t)layer * D.n_phys_pages + phys) * D.Hkv + g) * (size_t)(D.PL * D.d);
+}
+
+// ---------------------------------------------------------------- producer
+
+__device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr& I, uint32_t u,
+                                                  uint8_t* dst, uint64_t* bar, uint64_t pol) {
+  const Dims& D = p.D;
+  switch (I.op) {
+    case OP_QKV: {
+      const LayerW& W = p.layers[I.layer];
+      const int half = D.d / 2;
+      const int P0 = (int)u * D.RP, hg = P0 / half, i0 = P0 % half;
+      const uint16_t* w;
+      int hh;
+      if (hg < D.Hq) { w = W.wq; hh = hg; }
+      else if (hg < D.Hq + D.Hkv) { w = W.wk; hh = hg - D.Hq; }
+      else { w = W.wv; hh = hg - D.Hq - D.Hkv; }
+      const size_t r0 = (size_t)hh * D.d + i0;
+      const uint32_t bytes = (uint32_t)D.RP * D.H * 2;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      bulk_g2s(dst, w + r0 * D.H, bytes, bar, pol);
+      bulk_g2s(dst + bytes, w + (r0 + half) * D.H, bytes, bar, pol);
+      break;
+    }
+    case OP_O: {
+      const int r0 = (int)u * D.Ro, nr = min(D.Ro, D.H - r0);
+      const uint32_t bytes = (uint32_t)nr * D.qdim * 2;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, p.layers[I.layer].wo + (size_t)r0 * D.qdim, bytes, bar, pol);
+      break;
+    }
+    case OP_GU: {
+      const LayerW& W = p.layers[I.layer];
+      const int r0 = (int)u * D.Rgu, nr = min(D.Rgu, D.F - r0);
+      const uint32_t bytes = (uint32_t)nr * D.H * 2;
+      mbar_arrive_expect_tx(bar, 2 * bytes);
+      bulk_g2s(dst, W.w_gate + (size_t)r0 * D.H, bytes, bar, pol);
+      bulk_g2s(dst + (size_t)D.Rgu * D.H * 2, W.w_up + (size_t)r0 * D.H, bytes, bar, pol);
+      break;
+    }
+    case OP_DOWN: {
+      const int r0 = (int)u * D.Rdn, nr = min(D.Rdn, D.H - r0);
+      const uint32_t rb = (uint32_t)D.KS * 2;
+      const uint16_t* w = p.layers[I.layer].w_down + (size_t)I.arg * D.KS;
+      mbar_arrive_expect_tx(bar, nr * rb);
+      for (int r = 0; r < nr; ++r) bulk_g2s(dst + r * rb, w + (size_t)(r0 + r) * D.F, rb, bar, pol);
+      break;
+    }
+    case OP_LM: {
+      const int r0 = (int)u * D.Rlm, nr = min(D.Rlm, D.V - r0);
+      const uint32_t bytes = (uint32_t)nr * D.H * 2;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, p.lm_head + (size_t)r0 * D.H, bytes, bar, pol);
+      break;
+    }
+  }
+}
+
+__device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
+                                      Misc* misc) {
+  const Dims& D = p.D;
+  const uint32_t NP = (uint32_t)p.ring_pages;
+  const uint64_t pol = l2_evict_first_policy();
+  const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
+  uint32_t pidx = 0;
+  bool ok = true;
+  for (uint32_t ii = i0; ii < i1 && ok; ++ii) {
+    const Instr I = p.instrs[ii];
+    long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 8 : nullptr;
+    for (uint32_t k = 0; k < I.n_units && ok; ++k) {
+      const uint32_t u = p.units[I.unit_off + k];
+      if (rec && k == 0) rec[5] = (long long)globaltimer_ns();
+      if (rec && k + 1 == I.n_units) rec[6] = (long long)globaltimer_ns();
+      if (I.op == OP_ATTN) {
+        const int b = u >> 24, g = (u >> 16) & 0xFF, s = u & 0xFFFF;
+        const int pos = p.pos[b], npg = pos / D.PL + 1;
+        const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
+        for (int j = pb; j < pe; ++j) {
+          const uint32_t slot = pidx % NP;
+          if (!(ok = wait_mbar(p, &empty[slot], ((pidx / NP) & 1) ^ 1, E_WAIT_EMPTY, ii, true))) break;
+          // only positions written by earlier steps; the current one is patched in by the consumer
+          const int n_old = min(D.PL, pos - j * D.PL);
+          if (n_old > 0) {
+            const size_t base = kv_offset(p, I.layer, b, j, g);
+            const uint32_t bytes = (uint32_t)n_old * D.d * 2;
+            uint8_t* dst = ring + (size_t)slot * kPageBytes;
+            mbar_arrive_expect_tx(&full[slot], 2 * bytes);
+            bulk_g2s(dst, p.kcache + base, bytes, &full[slot], pol);
+            bulk_g2s(dst + (size_t)D.PL * D.d * 2, p.vcache + base, bytes, &full[slot], pol);
+          } else {
+            mbar_arrive(&full[slot]);
+          }
+          ++pidx;
+        }
+      } else {
+        const uint32_t slot = pidx % NP;
+        if (!(ok = wait_mbar(p, &empty[slot], ((pidx / NP) & 1) ^ 1, E_WAIT_EMPTY, ii, true))) break;
+        issue_matvec_page(p, I, u, ring + (size_t)slot * kPageBytes, &full[slot], pol);
+        ++pidx;
+      }
+    }
+  }
+  misc->issued = pidx;
+  // every copy issued must land before the CTA exits (also after an abort)
+  const uint32_t first = pidx > NP ? pidx - NP : 0;
+  for (uint32_t q = first; q < pidx; ++q)
+    if (!wait_mbar(p, &full[q % NP], (q / NP) & 1, E_DRAIN, q, false)) break;
+}
+
+// ---------------------------------------------------------------- consumers: staging
+
+// Stage NBT activation rows of length K into shared memory in the split layout
+// used by the matvec (chunk c of lane b: elements 8c..8c+3 at lo[b*nch + c],
+// 8c+4..8c+7 at hi[b*nch + c]).  Source: fp32 rows (L2, written by other SMs in
+// this step) or, for layer 0, the bf16 embedding rows of the lanes' tokens, which
+// are also written to the residual rows [xlo, xhi).  NORM applies RMSNorm with
+// the bf16 gain.  Lanes >= nb are zero.
+template <int NBT, bool EMB, bool NORM>
+__device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, const float* src,
+                                      int ld, int K, const uint16_t* gain, int xlo, int xhi) {
+  const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
+  const int nch = K >> 3;
+  float4* lo = reinterpret_cast<float4*>(act);
+  float4* hi = lo + NBT * nch;
+  float ss[NBT];
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) ss[b] = 0.f;
+  for (int c = ct; c < nch; c += 256) {
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) {
+      float v[8];
+      if (b < p.nb) {
+        if (EMB) {
+          const uint4 w = ldnc16(p.embed + (size_t)misc->tok[b] * p.D.H + c * 8);
+          v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
+          v[4] = bf_lo(w.z); v[5] = bf_hi(w.z); v[6] = bf_lo(w.w); v[7] = bf_hi(w.w);
+          const int k0 = c * 8;
+          if (k0 + 8 > xlo && k0 < xhi) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (k0 + e >= xlo && k0 + e < xhi) p.x[(size_t)b * p.D.H + k0 + e] = v[e];
+          }
+        } else {
+          const float4 a0 = ldcg4(src + (size_t)b * ld + c * 8), a1 = ldcg4(src + (size_t)b * ld + c * 8 + 4);
+          v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
+          v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      if (NORM) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss[b] = fmaf(v[e], v[e], ss[b]);
+      }
+      lo[b * nch + c] = make_float4(v[0], v[1], v[2], v[3]);
+      hi[b * nch + c] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+  if (NORM) {
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) {
+      float s = ss[b];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+      if (lane == 0) misc->red[cw][b] = s;
+    }
+    cbar();
+    float rinv[NBT];
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) {
+      float t = 0.f;
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) t += misc->red[w][b];
+      rinv[b] = 1.0f / sqrtf(t / (float)K + p.D.eps);
+    }
+    for (int c = ct; c < nch; c += 256) {
+      const uint4 gw = ldnc16(gain + c * 8);
+      const float g0 = bf_lo(gw.x), g1 = bf_hi(gw.x), g2 = bf_lo(gw.y), g3 = bf_hi(gw.y);
+      const float g4 = bf_lo(gw.z), g5 = bf_hi(gw.z), g6 = bf_lo(gw.w), g7 = bf_hi(gw.w);
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {
+        float4 l4 = lo[b * nch + c], h4 = hi[b * nch + c];
+        const float r = rinv[b];
+        l4.x = l4.x * r * g0; l4.y = l4.y * r * g1; l4.z = l4.z * r * g2; l4.w = l4.w * r * g3;
+        h4.x = h4.x * r * g4; h4.y = h4.y * r * g5; h4.z = h4.z * r * g6; h4.w = h4.w * r * g7;
+        lo[b * nch + c] = l4;
+        hi[b * nch + c] = h4;
+      }
+    }
+  }
+  cbar();
+}
+
+// ---------------------------------------------------------------- consumers: matvec
+
+// acc[r][b] += sum_k W[r][k] * act[b][k] over this lane's 8-element chunks.
+template <int RT, int NBT>
+__device__ __forceinline__ void mv_core(uint32_t tile, int nch, const float4* alo, const float4* ahi,
+                                        int lane, float (&acc)[RT][NBT]) {
+#pragma unroll 2
+  for (int c = lane; c < nch; c += 32) {
+    float4 xl[NBT], xh[NBT];
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) {
+      xl[b] = alo[b * nch + c];
+      xh[b] = ahi[b * nch + c];
+    }
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const uint4 w = lds128(tile + (uint32_t)(r * nch + c) * 16u);
+      const float f0 = bf_lo(w.x), f1 = bf_hi(w.x), f2 = bf_lo(w.y), f3 = bf_hi(w.y);
+      const float f4 = bf_lo(w.z), f5 = bf_hi(w.z), f6 = bf_lo(w.w), f7 = bf_hi(w.w);
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {
+        float s = acc[r][b];
+        s = fmaf(f0, xl[b].x, s); s = fmaf(f1, xl[b].y, s);
+        s = fmaf(f2, xl[b].z, s); s = fmaf(f3, xl[b].w, s);
+        s = fmaf(f4, xh[b].x, s); s = fmaf(f5, xh[b].y, s);
+        s = fmaf(f6, xh[b].z, s); s = fmaf(f7, xh[b].w, s);
+        acc[r][b] = s;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ bool lm_better(float v, int i, float bv, int bi) {
+  return v > bv || (v == bv && i < bi);
+}
+
+// Warp-per-page matvec over this instruction's units, then the op's epilogue.
+template <int OPK, int RT, int NBT>
+__device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t page_base,
+                                      uint8_t* ring, const float* act, int K, uint64_t* full,
+                                      uint64_t* empty, Misc* misc, uint32_t ii) {
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
+  const uint32_t NP = (uint32_t)p.ring_pages;
+  const int nch = K >> 3;
+  const float4* alo = reinterpret_cast<const float4*>(act);
+  const float4* ahi = alo + NBT * nch;
+  float bestv[NBT];
+  int besti[NBT];
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) { bestv[b] = -CUDART_INF_F; besti[b] = 0x7FFFFFFF; }
+
+  for (uint32_t k = cw; k < I.n_units; k += kConsumerWarps) {
+    const uint32_t pidx = page_base + k, slot = pidx % NP;
+    bool ok = wait_mbar(p, &full[slot], (pidx / NP) & 1, E_WAIT_FULL, ii, true);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) misc->stop = 1;
+      break;
+    }
+    float acc[RT][NBT];
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) acc[r][b] = 0.f;
+    mv_core<RT, NBT>(smem_u32(ring + (size_t)slot * kPageBytes), nch, alo, ahi, lane, acc);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {
+        float s = acc[r][b];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        acc[r][b] = s;
+      }
+    const uint32_t u = p.units[I.unit_off + k];
+
+    if constexpr (OPK == OP_QKV) {
+      constexpr int RP = RT / 2;
+      const int half = D.d / 2;
+      const int P0 = (int)u * RP, hg = P0 / half, i0 = P0 % half;
+      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
+      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+#pragma unroll
+      for (int j = 0; j < RP; ++j)
+#pragma unroll
+        for (int b = 0; b < NBT; ++b) {
+          if (lane != ((j * NBT + b) & 31) || b >= p.nb) continue;
+          const float v1 = acc[j][b], v2 = acc[RP + j][b];
+          const int i = i0 + j, pos = p.pos[b];
+          float r1 = v1, r2 = v2;
+          if (sec < 2) {
+            const float2 cs = p.rope[(size_t)pos * half + i];
+            r1 = v1 * cs.x - v2 * cs.y;
+            r2 = v2 * cs.x + v1 * cs.y;
+          }
+          if (sec == 0) {
+            float* qq = p.q + (size_t)b * D.qdim + hh * D.d;
+            qq[i] = r1;
+            qq[i + half] = r2;
+          } else {
+            const size_t idx = kv_offset(p, I.layer, b, pos / D.PL, hh) + (size_t)(pos % D.PL) * D.d + i;
+            uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
+            cache[idx] = f2bf(r1);
+            cache[idx + half] = f2bf(r2);
+          }
+        }
+    } else if constexpr (OPK == OP_O || OPK == OP_DOWN) {
+      const int R = OPK == OP_O ? D.Ro : D.Rdn;
+      const int r0 = (int)u * R, nr = min(R, D.H - r0);
+#pragma unroll
+      for (int r = 0; r < RT; ++r)
+#pragma unroll
+        for (int b = 0; b < NBT; ++b)
+          if (lane == ((r * NBT + b) & 31) && r < nr && b < p.nb)
+            red_add_f32(p.x + (size_t)b * D.H + r0 + r, acc[r][b]);
+    } else if constexpr (OPK == OP_GU) {
+      constexpr int R = RT / 2;
+      const int r0 = (int)u * R, nr = min(R, D.F - r0);
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+#pragma unroll
+        for (int b = 0; b < NBT; ++b)
+          if (lane == ((r * NBT + b) & 31) && r < nr && b < p.nb) {
+            const float g = acc[r][b], up = acc[R + r][b];
+            p.a[(size_t)b * D.F + r0 + r] = g / (1.0f + __expf(-g)) * up;
+          }
+    } else if constexpr (OPK == OP_LM) {
+      const int r0 = (int)u * RT, nr = min(RT, D.V - r0);
+#pragma unroll
+      for (int r = 0; r < RT; ++r) {
+        if (r >= nr) break;
+#pragma unroll
+        for (int b = 0; b < NBT; ++b) {
+          if (b >= p.nb) continue;
+          const float v = acc[r][b];
+          if (lm_better(v, r0 + r, bestv[b], besti[b])) { bestv[b] = v; besti[b] = r0 + r; }
+          if (p.logits && lane == ((r * NBT + b) & 31)) p.logits[(size_t)b * D.V + r0 + r] = v;
+        }
+      }
+    }
+  }
+
+  if constexpr (OPK == OP_LM) {
+    // combine the warps' running argmax, publish this SM's, the last SM reduces
+    if (lane == 0)
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) { misc->lmv[cw][b] = bestv[b]; misc->lmi[cw][b] = besti[b]; }
+    cbar();
+    if (ct < NBT) {
+      float bv = -CUDART_INF_F;
+      int bi = 0x7FFFFFFF;
+      for (int w = 0; w < kConsumerWarps; ++w)
+        if (lm_better(misc->lmv[w][ct], misc->lmi[w][ct], bv, bi)) { bv = misc->lmv[w][ct]; bi = misc->lmi[w][ct]; }
+      p.lm_part[blockIdx.x * kMaxNB + ct] = make_int2(__float_as_int(bv), bi);
+    }
+    __threadfence();
+    cbar();
+    if (ct == 0) {
+      const uint32_t old = atom_acq_rel_add(p.ctr + ctr_lm(D), 1u);
+      misc->last = (old == gridDim.x - 1) && !misc->stop;
+    }
+    cbar();
+    if (misc->last && ct < p.nb) {
+      float bv = -CUDART_INF_F;
+      int bi = 0x7FFFFFFF;
+      for (int s = 0; s < (int)gridDim.x; ++s) {
+        const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
+        const float v = __int_as_float(e.x);
+        if (lm_better(v, e.y, bv, bi)) { bv = v; bi = e.y; }
+      }
+      p.ids[ct] = (bi >= 0 && bi < D.V) ? bi : 0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------- consumers: attention
+
+// Split-KV GQA decode attention for the slices of this instruction.  A slice
+// covers a contiguous range of KV pages of one (lane, kv head); the 8 warps take
+// its pages round-robin, each keeping an online-softmax partial (running max m,
+// sum l, unnormalised output o) for the REP query heads of the group; the CTA
+// combines them into one slice partial, and the last slice to finish (atomic
+// counter) merges all slices of the (lane, kv head) into o.
+template <int DH, int REP>
+__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
+                                            uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
+                                            Misc* misc, uint32_t ii) {
+  constexpr int DC = DH / 8;                 // 16-byte chunks per K/V row
+  constexpr int PL = kPageBytes / (4 * DH);  // positions per KV page
+  constexpr int JP = PL / 32;                // score rows per lane
+  constexpr int DPL = DH / 32;               // output dims per lane
+  constexpr int CS = DH + 2;                 // partial record: o[DH], m, l
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
+  const uint32_t NP = (uint32_t)p.ring_pages;
+  float4* qlo = reinterpret_cast<float4*>(act);
+  float4* qhi = qlo + REP * DC;
+  float* pbuf = act + REP * DH + cw * PL * REP;
+  float* comb = act + REP * DH + kConsumerWarps * PL * REP;
+  const float scale = 1.0f / sqrtf((float)DH);
+  uint32_t used = 0;
+
+  for (uint32_t k = 0; k < I.n_units; ++k) {
+    const uint32_t u = p.units[I.unit_off + k];
+    const int b = u >> 24, g = (u >> 16) & 0xFF, s = u & 0xFFFF;
+    const int pos = p.pos[b], npg = pos / PL + 1;
+    const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
+    const int np_ = pe - pb;
+    for (int e = ct; e < REP * DC; e += 256) {
+      const int h = e / DC, c = e % DC;
+      const float* src = p.q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
+      float4 a0 = ldcg4(src), a1 = ldcg4(src + 4);
+      a0.x *= scale; a0.y *= scale; a0.z *= scale; a0.w *= scale;
+      a1.x *= scale; a1.y *= scale; a1.z *= scale; a1.w *= scale;
+      qlo[h * DC + c] = a0;
+      qhi[h * DC + c] = a1;
+    }
+    cbar();
+
+    float m[REP], l[REP], o[REP][DPL];
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      m[h] = -CUDART_INF_F;
+      l[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
+    }
+    for (int j = cw; j < np_; j += kConsumerWarps) {
+      const uint32_t pidx = page_base + used + j, slot = pidx % NP;
+      bool ok = wait_mbar(p, &full[slot], (pidx / NP) & 1, E_WAIT_FULL, ii, true);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) misc->stop = 1;
+        break;
+      }
+      uint8_t* pg = ring + (size_t)slot * kPageBytes;
+      uint8_t* vpg = pg + PL * DH * 2;
+      const int p0 = (pb + j) * PL;
+      const int cnt = min(PL, pos + 1 - p0);  // valid rows, >= 1
+      const int rcur = pos - p0;              // this step's position, if in this page
+      if (rcur < PL) {
+        const size_t base = kv_offset(p, I.layer, b, pb + j, g) + (size_t)rcur * DH;
+        if constexpr (DH == 64) {
+          reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane] =
+              __ldcg(reinterpret_cast<const unsigned int*>(p.kcache + base) + lane);
+          reinterpret_cast<uint32_t*>(vpg + rcur * DH * 2)[lane] =
+              __ldcg(reinterpret_cast<const unsigned int*>(p.vcache + base) + lane);
+        } else {
+          reinterpret_cast<uint2*>(pg + rcur * DH * 2)[lane] =
+              __ldcg(reinterpret_cast<const uint2*>(p.kcache + base) + lane);
+          reinterpret_cast<uint2*>(vpg + rcur * DH * 2)[lane] =
+              __ldcg(reinterpret_cast<const uint2*>(p.vcache + base) + lane);
+        }
+        __syncwarp();
+      }
+      // scores s[h][row] = (q_h / sqrt(d)) . k_row; rows lane and lane + 32
+      float sc[REP][JP];
+#pragma unroll
+      for (int h = 0; h < REP; ++h)
+#pragma unroll
+        for (int jj = 0; jj < JP; ++jj) sc[h][jj] = 0.f;
+      const uint32_t kb = smem_u32(pg);
+#pragma unroll
+      for (int cc = 0; cc < DC; ++cc) {
+        const int c = (cc + lane) & (DC - 1);  // rotated so a warp's rows hit distinct banks
+        uint4 kw[JP];
+#pragma unroll
+        for (int jj = 0; jj < JP; ++jj) kw[jj] = lds128(kb + (uint32_t)(((lane + 32 * jj) * DC + c) * 16));
+#pragma unroll
+        for (int h = 0; h < REP; ++h) {
+          const float4 ql = qlo[h * DC + c], qh = qhi[h * DC + c];
+#pragma unroll
+          for (int jj = 0; jj < JP; ++jj) {
+            float t = sc[h][jj];
+            t = fmaf(bf_lo(kw[jj].x), ql.x, t); t = fmaf(bf_hi(kw[jj].x), ql.y, t);
+            t = fmaf(bf_lo(kw[jj].y), ql.z, t); t = fmaf(bf_hi(kw[jj].y), ql.w, t);
+            t = fmaf(bf_lo(kw[jj].z), qh.x, t); t = fmaf(bf_hi(kw[jj].z), qh.y, t);
+            t = fmaf(bf_lo(kw[jj].w), qh.z, t); t = fmaf(bf_hi(kw[jj].w), qh.w, t);
+            sc[h][jj] = t;
+          }
+        }
+      }
+      // online softmax update
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int jj = 0; jj < JP; ++jj)
+          if (lane + 32 * jj < cnt) mx = fmaxf(mx, sc[h][jj]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        const float mnew = fmaxf(m[h], mx);
+        const float corr = __expf(m[h] - mnew);
+        float ps = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < JP; ++jj) {
+          const int row = lane + 32 * jj;
+          const float pr = row < cnt ? __expf(sc[h][jj] - mnew) : 0.f;
+          pbuf[row * REP + h] = pr;
+          ps += pr;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
+        l[h] = l[h] * corr + ps;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
+        m[h] = mnew;
+      }
+      __syncwarp();
+      // o[h][dims of this lane] += p[h][row] * v[row][dims]
+      const uint8_t* vrow = vpg + lane * DPL * 2;
+      for (int r = 0; r < cnt; ++r) {
+        float pv[REP];
+        if constexpr (REP % 4 == 0) {
+#pragma unroll
+          for (int h = 0; h < REP; h += 4) {
+            const float4 t = *reinterpret_cast<const float4*>(pbuf + r * REP + h);
+            pv[h] = t.x; pv[h + 1] = t.y; pv[h + 2] = t.z; pv[h + 3] = t.w;
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < REP; ++h) pv[h] = pbuf[r * REP + h];
+        }
+        float vv[DPL];
+        if constexpr (DPL == 2) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(vrow + r * DH * 2);
+          vv[0] = bf_lo(w); vv[1] = bf_hi(w);
+        } else {
+          const uint2 w = *reinterpret_cast<const uint2*>(vrow + r * DH * 2);
+          vv[0] = bf_lo(w.x); vv[1] = bf_hi(w.x); vv[2] = bf_lo(w.y); vv[3] = bf_hi(w.y);
+        }
+#pragma unroll
+        for (int h = 0; h < REP; ++h)
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pv[h], vv[e], o[h][e]);
+      }
+      __syncwarp();
+      if (rcur < PL) fence_proxy_async_smem();  // generic writes before the next bulk copy
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    // combine the warps' partials into this slice's partial
+    float* mine = comb + cw * REP * CS;
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) mine[h * CS + lane * DPL + e] = o[h][e];
+      if (lane == 0) { mine[h * CS + DH] = m[h]; mine[h * CS + DH + 1] = l[h]; }
+    }
+    cbar();
+    if (misc->stop) { cbar(); break; }
+    float* part = p.part + ((size_t)(b * D.Hkv + g) * p.S + s) * REP * CS;
+    for (int e = ct; e < REP * DH; e += 256) {
+      const int h = e / DH, i = e % DH;
+      float M = -CUDART_INF_F;
+      for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * REP + h) * CS + DH]);
+      float L = 0.f, O = 0.f;
+      if (M > -CUDART_INF_F)
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = comb[(w * REP + h) * CS + DH];
+          if (mw > -CUDART_INF_F) {
+            const float f = __expf(mw - M);
+            L += comb[(w * REP + h) * CS + DH + 1] * f;
+            O += comb[(w * REP + h) * CS + i] * f;
+          }
+        }
+      part[h * CS + i] = O;
+      if (i == 0) { part[h * CS + DH] = M; part[h * CS + DH + 1] = L; }
+    }
+    __threadfence();
+    cbar();
+    if (ct == 0) {
+      const uint32_t old = atom_acq_rel_add(p.ctr + ctr_part(D, I.layer, b, g), 1u);
+      misc->last = (old == (uint32_t)p.S - 1);
+    }
+    cbar();
+    if (misc->last) {
+      const float* pp = p.part + (size_t)(b * D.Hkv + g) * p.S * REP * CS;
+      for (int e = ct; e < REP * DH; e += 256) {
+        const int h = e / DH, i = e % DH;
+        float M = -CUDART_INF_F;
+        for (int t = 0; t < p.S; ++t) M = fmaxf(M, __ldcg(pp + (t * REP + h) * CS + DH));
+        float L = 0.f, O = 0.f;
+        for (int t = 0; t < p.S; ++t) {
+          const float mt = __ldcg(pp + (t * REP + h) * CS + DH);
+          if (mt > -CUDART_INF_F) {
+            const float f = __expf(mt - M);
+            L += __ldcg(pp + (t * REP + h) * CS + DH + 1) * f;
+            O += __ldcg(pp + (t * REP + h) * CS + i) * f;
+          }
+        }
+        p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
+      }
+      __threadfence();
+      cbar();
+      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+    }
+    used += (uint32_t)np_;
+    cbar();
+  }
+  return used;
+}
+
+// ---------------------------------------------------------------- consumers: ops
+
+template <int OPK, int NBT>
+__device__ __forceinline__ void mv_dispatch(int rt, const KParams& p, const Instr& I, uint32_t pb,
+                                            uint8_t* ring, const float* act, int K, uint64_t* full,
+                                            uint64_t* empty, Misc* misc, uint32_t ii) {
+  switch (rt) {
+    case 1: if constexpr (OPK != OP_QKV && OPK != OP_GU) mv_units<OPK, 1, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 2: mv_units<OPK, 2, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 4: mv_units<OPK, 4, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 8: mv_units<OPK, 8, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+  }
+}
+
+template <int DH>
+__device__ __forceinline__ uint32_t attn_dispatch(const KParams& p, const Instr& I, uint32_t pb,
+                                                  uint8_t* ring, float* act, uint64_t* full,
+                                                  uint64_t* empty, Misc* misc, uint32_t ii) {
+  switch (p.D.rep) {
+    case 1: return attn_units<DH, 1>(p, I, pb, ring, act, full, empty, misc, ii);
+    case 2: return attn_units<DH, 2>(p, I, pb, ring, act, full, empty, misc, ii);
+    case 4: return attn_units<DH, 4>(p, I, pb, ring, act, full, empty, misc, ii);
+    default: return attn_units<DH, 8>(p, I, pb, ring, act, full, empty, misc, ii);
+  }
+}
+
+template <int NBT>
+__device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* act, uint64_t* full,
+                                      uint64_t* empty, Misc* misc) {
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32;
+  const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
+  uint32_t page_base = 0;
+  for (uint32_t ii = i0; ii < i1; ++ii) {
+    const Instr I = p.instrs[ii];
+    long long* rec = (p.prof && ct == 0) ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 8 : nullptr;
+    if (rec) {
+      rec[0] = (long long)I.op | ((long long)I.layer << 8) | ((long long)I.n_units << 24);
+      rec[1] = (long long)globaltimer_ns();
+    }
+    if (ct == 0 && I.dep != kNoCounter)
+      if (!wait_counter(p, p.ctr + I.dep, I.dep_target, ii)) misc->stop = 1;
+    cbar();
+    if (rec) rec[2] = (long long)globaltimer_ns();
+    if (misc->stop) break;
+    uint32_t used = I.n_units;  // one page per unit, except attention
+    switch (I.op) {
+      case OP_QKV: {
+        const LayerW& W = p.layers[I.layer];
+        if (I.layer == 0) {
+          if (ct < NBT) {
+            int t = ct < p.nb ? p.tokens[ct] : 0;
+            if (t < 0 || t >= D.V) {
+              raise_error(p, E_BAD_TOKEN, ii, (uint32_t)t, false);
+              t = 0;
+            }
+            misc->tok[ct] = t;
+          }
+          cbar();
+          stage<NBT, true, true>(p, act, misc, nullptr, 0, D.H, W.attn_norm, (int)I.aux0, (int)I.aux1);
+        } else {
+          stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, W.attn_norm, 0, 0);
+        }
+        mv_dispatch<OP_QKV, NBT>(2 * D.RP, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
+        break;
+      }
+      case OP_ATTN:
+        used = D.d == 64 ? attn_dispatch<64>(p, I, page_base, ring, act, full, empty, misc, ii)
+                         : attn_dispatch<128>(p, I, page_base, ring, act, full, empty, misc, ii);
+        break;
+      case OP_O:
+        stage<NBT, false, false>(p, act, misc, p.o, D.qdim, D.qdim, nullptr, 0, 0);
+        mv_dispatch<OP_O, NBT>(D.Ro, p, I, page_base, ring, act, D.qdim, full, empty, misc, ii);
+        break;
+      case OP_GU:
+        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, p.layers[I.layer].mlp_norm, 0, 0);
+        mv_dispatch<OP_GU, NBT>(2 * D.Rgu, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
+        break;
+      case OP_DOWN:
+        stage<NBT, false, false>(p, act, misc, p.a + (size_t)I.arg * D.KS, D.F, D.KS, nullptr, 0, 0);
+        mv_dispatch<OP_DOWN, NBT>(D.Rdn, p, I, page_base, ring, act, D.KS, full, empty, misc, ii);
+        break;
+      case OP_LM:
+        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, p.final_norm, 0, 0);
+        mv_dispatch<OP_LM, NBT>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
+        break;
+    }
+    page_base += used;
+    if (rec) rec[3] = (long long)globaltimer_ns();
+    __threadfence();
+    cbar();
+    if (misc->stop) break;
+    if (ct == 0 && I.sig != kNoCounter) red_release_add(p.ctr + I.sig, 1u);
+    if (rec) rec[4] = (long long)globaltimer_ns();
+  }
+}
+
+// ---------------------------------------------------------------- the kernel
+
+template <int NBT>
+__global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
+  Misc* misc = reinterpret_cast<Misc*>(smem + p.misc_off);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
+  uint64_t* empty = full + 64;
+  // the next step's counters start from zero (this step's were zeroed by the previous one)
+  for (int i = blockIdx.x * kThreads + threadIdx.x; i < p.n_counters; i += gridDim.x * kThreads)
+    p.ctr_next[i] = 0u;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < p.ring_pages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    misc->stop = 0;
+    misc->last = 0;
+    misc->issued = 0;
+    misc->entry_abort = aborted(p) ? 1 : 0;
+  }
+  __syncthreads();
+  if (!misc->entry_abort) {
+    if (threadIdx.x < 32) {
+      if (threadIdx.x == 0) producer(p, smem, full, empty, misc);
+    } else {
+      consumer<NBT>(p, smem, reinterpret_cast<float*>(smem + p.act_off), full, empty, misc);
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace mk

@@ -1,0 +1,120 @@
+// mk_plan.h -- the instruction tape format shared by the host scheduler and the
+// persistent kernel, plus the shape parameters both derive from a config.
+//
+// The per-SM "execution plan" of the Hazy megakernel article (section
+// "Megakernel: a deep-fusion design from scratch"): an ordered list of fused
+// instructions per SM whose dependencies are fixed before the run.  Here an
+// instruction names an op, a layer, a list of work units (each unit is exactly
+// one shared-memory page of weights, or one attention slice), the counter it
+// waits on with its target, and the counter it bumps when done.
+#pragma once
+
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#if defined(__CUDACC__)
+#define MK_HD __host__ __device__
+#else
+#define MK_HD
+#endif
+
+namespace mk {
+
+enum Op : uint8_t {
+  OP_QKV = 1,   // RMSNorm(x) -> rows of Wq|Wk|Wv -> RoPE -> q scratch / K,V cache
+  OP_ATTN = 2,  // one slice of a (lane, kv head) over a range of KV pages -> partial; last merges
+  OP_O = 3,     // rows of Wo . o -> x += (red.add)
+  OP_GU = 4,    // RMSNorm(x) -> rows of Wgate and Wup -> a = silu(g) * u
+  OP_DOWN = 5,  // rows of Wdown over one K slice . a -> x += (red.add)
+  OP_LM = 6,    // RMSNorm(x) -> rows of the LM head -> logits, running argmax; last reduces
+};
+
+constexpr int kPageBytes = 16384;      // one ring page
+constexpr int kMaxNB = 8;              // lanes (sequences) per step
+constexpr int kConsumerWarps = 8;      // warps that compute; warp 0 loads
+constexpr int kThreads = 32 * (1 + kConsumerWarps);
+constexpr int kActFloatsMax = 16384;   // max_batch * K of the staged activation
+constexpr uint16_t kNoCounter = 0xFFFF;
+
+// counters of one layer
+enum : int { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, kCountersPerLayer = 5 };
+
+struct Instr {            // 32 bytes
+  uint8_t op;
+  uint8_t arg;            // OP_DOWN: K-slice index
+  uint16_t layer;
+  uint32_t unit_off;      // first unit in the tape's unit array
+  uint32_t n_units;
+  uint16_t dep;           // counter waited on before the instruction (kNoCounter: none)
+  uint16_t sig;           // counter incremented once when the instruction is done
+  uint32_t dep_target;    // value `dep` must reach in this step
+  uint32_t aux0, aux1;    // OP_QKV at layer 0: residual rows [aux0, aux1) this SM seeds
+  uint32_t pad;
+};
+static_assert(sizeof(Instr) == 32, "Instr layout");
+
+// Shape parameters of one handle (identical for every tape of the handle).
+struct Dims {
+  int L, H, Hq, Hkv, d, F, V, qdim, kvdim, rep;
+  int RP;         // QKV: half-split pairs per unit (unit rows = 2*RP)
+  int Ro, Rgu, Rdn, Rlm;  // rows per unit of O, gate/up (each), down, LM head
+  int n_ks, KS;   // down projection: K slices and their width
+  int PL;         // positions per KV page
+  int pages_per_seq;
+  int n_phys_pages;   // KV pages per layer per kv head (all slots)
+  int max_batch, max_seq;
+  int n_qkv, n_o, n_gu, n_dn, n_lm;   // units per op per layer (n_dn per K slice)
+  float eps;
+  int tied;
+};
+
+// One tape: the instruction lists of every SM for one active batch size.
+struct Tape {
+  int nb = 0;
+  int S = 1;                      // attention slices per (lane, kv head)
+  int n_counters = 0;
+  std::vector<uint32_t> sm_off;   // n_sm + 1 offsets into instrs
+  std::vector<Instr> instrs;
+  std::vector<uint32_t> units;
+};
+
+// lanes the kernel is instantiated for: the batch size rounded up to 1, 2, 4 or 8
+MK_HD inline int lanes_template(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
+
+MK_HD inline int ctr_layer(int layer, int kind) { return layer * kCountersPerLayer + kind; }
+MK_HD inline int ctr_part(const Dims& D, int layer, int b, int g) {
+  return D.L * kCountersPerLayer + (layer * kMaxNB + b) * D.Hkv + g;
+}
+MK_HD inline int ctr_lm(const Dims& D) { return D.L * kCountersPerLayer + D.L * kMaxNB * D.Hkv; }
+MK_HD inline int n_counters(const Dims& D) { return ctr_lm(D) + 1; }
+
+MK_HD inline uint32_t attn_unit(int b, int g, int s) { return (uint32_t(b) << 24) | (uint32_t(g) << 16) | uint32_t(s); }
+
+// Shape derivation and tape lowering (mk_sched.cpp).
+std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                        int ffn, int vocab, int tied, float eps, int max_batch, int max_seq,
+                        int n_sm, Dims* out);
+int attn_slices(const Dims& D, int n_sm, int nb);
+Tape lower(const Dims& D, int n_sm, int nb);
+
+struct SimReport {
+  bool deadlock_free = false, coverage_ok = false, targets_ok = false;
+  int max_instr_per_sm = 0, n_instr_total = 0;
+  int64_t bytes_min = 0, bytes_max = 0;
+  std::string error;
+};
+SimReport simulate(const Dims& D, int n_sm, const Tape& t);
+
+// Dynamic shared memory layout of the kernel.
+struct SmemLayout {
+  int ring_pages;
+  int act_bytes;     // activation / attention scratch region
+  int bar_off;       // mbarriers
+  int misc_off;      // small reduction scratch
+  int total;
+};
+SmemLayout smem_layout(const Dims& D, int nb_max, int max_dyn_smem, int want_pages);
+
+}  // namespace mk

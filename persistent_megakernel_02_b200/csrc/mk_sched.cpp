@@ -1,0 +1,342 @@
+// mk_sched.cpp -- host scheduler: lowers a decoder shape into per-SM instruction
+// tapes with counter targets, and a CPU simulator that runs a tape to prove it is
+// deadlock-free, covers every output exactly once and waits on full fan-in.
+//
+// The Hazy megakernel article (section "Megakernel: a deep-fusion design from
+// scratch") says the dependencies between instructions are analysed and laid
+// out before the run, and each SM gets its own ordered execution plan; the
+// forum post "Two thousand four hundred kernel launches per token" (tail-effect
+// example: 512 work blocks on 148 SMs leave 80 idle in the last wave) is why
+// units are assigned by cumulative bytes per SM rather than in waves.
+#include <algorithm>
+#include <cstdio>
+#include <queue>
+#include <string>
+#include <vector>
+
+#include "mk_plan.h"
+
+namespace mk {
+
+static int pow2_floor(long long x) {
+  if (x < 1) return 1;
+  int p = 1;
+  while ((long long)p * 2 <= x) p *= 2;
+  return p;
+}
+
+// rows of length k (bf16) that fit one page, at most 8, a power of two
+static int page_rows(int k) { return std::min(8, pow2_floor(kPageBytes / (2LL * k))); }
+
+std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, int head_dim,
+                        int ffn, int vocab, int tied, float eps, int max_batch, int max_seq,
+                        int n_sm, Dims* out) {
+  char buf[256];
+  if (n_layers < 1 || n_layers > 4096) return "n_layers out of range";
+  if (head_dim != 64 && head_dim != 128) return "head_dim must be 64 or 128";
+  if (n_heads < 1 || n_kv_heads < 1 || n_heads % n_kv_heads) return "n_heads must be a multiple of n_kv_heads";
+  int rep = n_heads / n_kv_heads;
+  if (rep != 1 && rep != 2 && rep != 4 && rep != 8) return "n_heads / n_kv_heads must be 1, 2, 4 or 8";
+  if (n_kv_heads > 255) return "n_kv_heads too large";
+  if (hidden < 8 || hidden % 8) return "hidden must be a positive multiple of 8";
+  if (hidden > 4096) return "hidden > 4096 is not supported (two rows per 16 KiB page)";
+  if (ffn < 8 || ffn % 8) return "ffn must be a positive multiple of 8";
+  int qdim = n_heads * head_dim, kvdim = n_kv_heads * head_dim;
+  if (qdim > 8192) return "n_heads * head_dim > 8192 is not supported";
+  if (vocab < 1) return "vocab must be positive";
+  if (max_batch < 1 || max_batch > kMaxNB) return "max_batch must be in 1..8";
+  if (max_seq < 1 || max_seq > (1 << 24)) return "max_seq out of range";
+  if (n_sm < 1 || n_sm > 4096) return "n_sm out of range";
+  int kact = std::max(hidden, qdim);
+  int nbt = lanes_template(max_batch);
+  if ((long long)nbt * kact > kActFloatsMax) {
+    snprintf(buf, sizeof buf,
+             "max_batch (rounded up to %d) * max(hidden, n_heads*head_dim) = %lld exceeds %d", nbt,
+             (long long)nbt * kact, kActFloatsMax);
+    return buf;
+  }
+  Dims D{};
+  D.L = n_layers; D.H = hidden; D.Hq = n_heads; D.Hkv = n_kv_heads; D.d = head_dim;
+  D.F = ffn; D.V = vocab; D.qdim = qdim; D.kvdim = kvdim; D.rep = rep;
+  D.eps = eps; D.tied = tied ? 1 : 0;
+  D.max_batch = max_batch; D.max_seq = max_seq;
+  // down projection: K slices no wider than the staged activation
+  int n_ks = 0;
+  for (int n = std::max(1, (ffn + kact - 1) / kact); n <= ffn / 8; ++n) {
+    if (ffn % n == 0 && (ffn / n) % 8 == 0 && ffn / n <= kact) { n_ks = n; break; }
+  }
+  if (!n_ks) return "ffn cannot be split into K slices of at most max(hidden, qdim)";
+  D.n_ks = n_ks; D.KS = ffn / n_ks;
+  if (n_ks > 255) return "too many down-projection K slices";
+  // rows per unit: as many as fit a page, but no more than keep every SM busy
+  long long pairs = (long long)(n_heads + 2 * n_kv_heads) * (head_dim / 2);
+  D.RP = std::min(page_rows(hidden) / 2, pow2_floor(pairs / n_sm));
+  if (D.RP < 1) D.RP = 1;
+  while ((head_dim / 2) % D.RP) D.RP /= 2;
+  D.Ro = std::min(page_rows(qdim), pow2_floor(hidden / n_sm));
+  D.Rgu = std::max(1, std::min(page_rows(hidden) / 2, pow2_floor(ffn / n_sm)));
+  D.Rdn = std::min(page_rows(D.KS), pow2_floor((long long)hidden * n_ks / n_sm));
+  D.Rlm = std::min(page_rows(hidden), pow2_floor(vocab / n_sm));
+  D.PL = kPageBytes / (4 * head_dim);
+  D.pages_per_seq = (max_seq + D.PL - 1) / D.PL;
+  D.n_phys_pages = max_batch * D.pages_per_seq;
+  D.n_qkv = (int)(pairs / D.RP);
+  D.n_o = (hidden + D.Ro - 1) / D.Ro;
+  D.n_gu = (ffn + D.Rgu - 1) / D.Rgu;
+  D.n_dn = (hidden + D.Rdn - 1) / D.Rdn;
+  D.n_lm = (vocab + D.Rlm - 1) / D.Rlm;
+  if (n_counters(D) >= kNoCounter) return "too many counters for this shape";
+  *out = D;
+  return "";
+}
+
+int attn_slices(const Dims& D, int n_sm, int nb) {
+  int s = n_sm / (nb * D.Hkv);
+  s = std::max(1, std::min(s, D.pages_per_seq));
+  return std::min(s, 65535);
+}
+
+// bytes one unit streams (weights), or an estimate for an attention slice
+static int64_t unit_bytes(const Dims& D, int op, int S) {
+  switch (op) {
+    case OP_QKV: return 2LL * 2 * D.RP * D.H;
+    case OP_O: return 2LL * D.Ro * D.qdim;
+    case OP_GU: return 2LL * 2 * D.Rgu * D.H;
+    case OP_DOWN: return 2LL * D.Rdn * D.KS;
+    case OP_LM: return 2LL * D.Rlm * D.H;
+    case OP_ATTN: {
+      int pages = (D.pages_per_seq + S - 1) / S;
+      return (int64_t)pages * kPageBytes;
+    }
+  }
+  return 0;
+}
+
+namespace {
+struct Assigner {
+  std::vector<int64_t>& load;
+  explicit Assigner(std::vector<int64_t>& l) : load(l) {}
+  // Give each of n equal units to the least-loaded SM of [lo, hi) (ties: lowest id).
+  std::vector<std::vector<uint32_t>> run(int n, int64_t bytes, int lo, int hi) {
+    using E = std::pair<int64_t, int>;
+    std::priority_queue<E, std::vector<E>, std::greater<E>> pq;
+    for (int s = lo; s < hi; ++s) pq.push({load[s], s});
+    std::vector<std::vector<uint32_t>> out(load.size());
+    for (int u = 0; u < n; ++u) {
+      E e = pq.top();
+      pq.pop();
+      out[e.second].push_back((uint32_t)u);
+      e.first += bytes;
+      load[e.second] = e.first;
+      pq.push(e);
+    }
+    return out;
+  }
+};
+}  // namespace
+
+Tape lower(const Dims& D, int n_sm, int nb) {
+  Tape t;
+  t.nb = nb;
+  t.S = attn_slices(D, n_sm, nb);
+  t.n_counters = n_counters(D);
+  std::vector<int64_t> load(n_sm, 0);
+  Assigner as(load);
+  std::vector<std::vector<Instr>> ins(n_sm);
+  std::vector<std::vector<uint32_t>> uts(n_sm);
+
+  auto emit = [&](int sm, uint8_t op, int layer, const std::vector<uint32_t>& units, uint16_t dep,
+                  uint16_t sig, uint8_t arg) -> Instr& {
+    Instr I{};
+    I.op = op; I.arg = arg; I.layer = (uint16_t)layer;
+    I.unit_off = (uint32_t)uts[sm].size();  // rebased when the tapes are concatenated
+    I.n_units = (uint32_t)units.size();
+    I.dep = dep; I.sig = sig; I.dep_target = 0;
+    uts[sm].insert(uts[sm].end(), units.begin(), units.end());
+    ins[sm].push_back(I);
+    return ins[sm].back();
+  };
+
+  for (int l = 0; l < D.L; ++l) {
+    uint16_t dep_qkv = l ? (uint16_t)ctr_layer(l - 1, C_DOWN) : kNoCounter;
+    // RMSNorm + QKV + RoPE
+    auto a = as.run(D.n_qkv, unit_bytes(D, OP_QKV, t.S), 0, n_sm);
+    std::vector<int> qkv_sms;
+    for (int s = 0; s < n_sm; ++s)
+      if (!a[s].empty()) qkv_sms.push_back(s);
+    for (size_t k = 0; k < qkv_sms.size(); ++k) {
+      int s = qkv_sms[k];
+      Instr& I = emit(s, OP_QKV, l, a[s], dep_qkv, (uint16_t)ctr_layer(l, C_QKV), 0);
+      if (l == 0) {  // these SMs seed the residual with the embedding rows
+        I.aux0 = (uint32_t)((long long)D.H * k / qkv_sms.size());
+        I.aux1 = (uint32_t)((long long)D.H * (k + 1) / qkv_sms.size());
+      }
+    }
+    // attention slices (lane, kv head, slice)
+    {
+      int n = nb * D.Hkv * t.S;
+      auto at = as.run(n, unit_bytes(D, OP_ATTN, t.S), 0, n_sm);
+      for (int s = 0; s < n_sm; ++s) {
+        if (at[s].empty()) continue;
+        std::vector<uint32_t> u;
+        for (uint32_t i : at[s]) {
+          int b = i / (D.Hkv * t.S), g = (i / t.S) % D.Hkv, sl = i % t.S;
+          u.push_back(attn_unit(b, g, sl));
+        }
+        emit(s, OP_ATTN, l, u, (uint16_t)ctr_layer(l, C_QKV), kNoCounter, 0);
+      }
+    }
+    // O projection + residual
+    auto o = as.run(D.n_o, unit_bytes(D, OP_O, t.S), 0, n_sm);
+    for (int s = 0; s < n_sm; ++s)
+      if (!o[s].empty()) emit(s, OP_O, l, o[s], (uint16_t)ctr_layer(l, C_ATTN), (uint16_t)ctr_layer(l, C_O), 0);
+    // RMSNorm + gate/up + SwiGLU
+    auto gu = as.run(D.n_gu, unit_bytes(D, OP_GU, t.S), 0, n_sm);
+    for (int s = 0; s < n_sm; ++s)
+      if (!gu[s].empty()) emit(s, OP_GU, l, gu[s], (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0);
+    // down projection + residual: SMs split into one group per K slice
+    for (int ks = 0; ks < D.n_ks; ++ks) {
+      int lo = (int)((long long)n_sm * ks / D.n_ks), hi = (int)((long long)n_sm * (ks + 1) / D.n_ks);
+      if (hi <= lo) hi = lo + 1;  // more slices than SMs: share
+      lo %= n_sm; hi = std::min(hi, n_sm);
+      auto dn = as.run(D.n_dn, unit_bytes(D, OP_DOWN, t.S), lo, hi);
+      for (int s = lo; s < hi; ++s)
+        if (!dn[s].empty())
+          emit(s, OP_DOWN, l, dn[s], (uint16_t)ctr_layer(l, C_GU), (uint16_t)ctr_layer(l, C_DOWN), (uint8_t)ks);
+    }
+  }
+  // final norm + LM head + argmax: every SM takes part (possibly with no rows)
+  auto lm = as.run(D.n_lm, unit_bytes(D, OP_LM, t.S), 0, n_sm);
+  for (int s = 0; s < n_sm; ++s)
+    emit(s, OP_LM, D.L, lm[s], (uint16_t)ctr_layer(D.L - 1, C_DOWN), kNoCounter, 0);
+
+  // wait targets = how many instructions signal the counter in one step
+  std::vector<uint32_t> fan(t.n_counters, 0);
+  for (int s = 0; s < n_sm; ++s)
+    for (auto& I : ins[s])
+      if (I.sig != kNoCounter) fan[I.sig]++;
+  for (int l = 0; l < D.L; ++l) fan[ctr_layer(l, C_ATTN)] = (uint32_t)(nb * D.Hkv);
+  for (int s = 0; s < n_sm; ++s)
+    for (auto& I : ins[s])
+      if (I.dep != kNoCounter) I.dep_target = fan[I.dep];
+
+  // concatenate
+  t.sm_off.assign(n_sm + 1, 0);
+  for (int s = 0; s < n_sm; ++s) {
+    t.sm_off[s] = (uint32_t)t.instrs.size();
+    uint32_t base = (uint32_t)t.units.size();
+    for (auto I : ins[s]) {
+      I.unit_off += base;
+      t.instrs.push_back(I);
+    }
+    t.units.insert(t.units.end(), uts[s].begin(), uts[s].end());
+  }
+  t.sm_off[n_sm] = (uint32_t)t.instrs.size();
+  return t;
+}
+
+SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
+  SimReport r;
+  std::vector<int64_t> ctr(t.n_counters, 0), signals(t.n_counters, 0);
+  std::vector<int64_t> part((size_t)D.L * kMaxNB * D.Hkv, 0);
+  const int nb = t.nb, S = t.S;
+  // coverage: per layer and op, how often each output tile was produced
+  std::vector<int> cq((size_t)D.L * D.n_qkv, 0), co((size_t)D.L * D.n_o, 0),
+      cg((size_t)D.L * D.n_gu, 0), cd((size_t)D.L * D.n_ks * D.n_dn, 0),
+      ca((size_t)D.L * nb * D.Hkv * S, 0), cl(D.n_lm, 0);
+  std::vector<uint32_t> ip(n_sm);
+  r.bytes_min = INT64_MAX; r.bytes_max = 0;
+  for (int s = 0; s < n_sm; ++s) {
+    ip[s] = t.sm_off[s];
+    int n = (int)(t.sm_off[s + 1] - t.sm_off[s]);
+    r.max_instr_per_sm = std::max(r.max_instr_per_sm, n);
+    int64_t by = 0;
+    for (uint32_t i = t.sm_off[s]; i < t.sm_off[s + 1]; ++i)
+      by += unit_bytes(D, t.instrs[i].op, S) * t.instrs[i].n_units;
+    r.bytes_min = std::min(r.bytes_min, by);
+    r.bytes_max = std::max(r.bytes_max, by);
+  }
+  r.n_instr_total = (int)t.instrs.size();
+  bool cover_err = false;
+  auto bump = [&](std::vector<int>& v, size_t i) {
+    if (i >= v.size()) { cover_err = true; return; }
+    v[i]++;
+  };
+  bool progress = true;
+  while (progress) {
+    progress = false;
+    for (int s = 0; s < n_sm; ++s) {
+      while (ip[s] < t.sm_off[s + 1]) {
+        const Instr& I = t.instrs[ip[s]];
+        if (I.dep != kNoCounter && ctr[I.dep] < (int64_t)I.dep_target) break;
+        int l = I.layer;
+        for (uint32_t k = 0; k < I.n_units; ++k) {
+          uint32_t u = t.units[I.unit_off + k];
+          switch (I.op) {
+            case OP_QKV: bump(cq, (size_t)l * D.n_qkv + u); break;
+            case OP_O: bump(co, (size_t)l * D.n_o + u); break;
+            case OP_GU: bump(cg, (size_t)l * D.n_gu + u); break;
+            case OP_DOWN: bump(cd, ((size_t)l * D.n_ks + I.arg) * D.n_dn + u); break;
+            case OP_LM: bump(cl, u); break;
+            case OP_ATTN: {
+              int b = u >> 24, g = (u >> 16) & 0xFF, sl = u & 0xFFFF;
+              if (b >= nb || g >= D.Hkv || sl >= S) { cover_err = true; break; }
+              bump(ca, (((size_t)l * nb + b) * D.Hkv + g) * S + sl);
+              size_t pi = ((size_t)l * kMaxNB + b) * D.Hkv + g;
+              ctr[ctr_part(D, l, b, g)]++;
+              if (++part[pi] == S) { ctr[ctr_layer(l, C_ATTN)]++; signals[ctr_layer(l, C_ATTN)]++; }
+              break;
+            }
+          }
+        }
+        if (I.op == OP_LM) { ctr[ctr_lm(D)]++; signals[ctr_lm(D)]++; }
+        if (I.sig != kNoCounter) { ctr[I.sig]++; signals[I.sig]++; }
+        ip[s]++;
+        progress = true;
+      }
+    }
+  }
+  r.deadlock_free = true;
+  for (int s = 0; s < n_sm; ++s)
+    if (ip[s] != t.sm_off[s + 1]) {
+      r.deadlock_free = false;
+      char b[128];
+      snprintf(b, sizeof b, "SM %d stuck at instruction %u", s, ip[s] - t.sm_off[s]);
+      r.error = b;
+      break;
+    }
+  auto all_one = [](const std::vector<int>& v) {
+    for (int x : v)
+      if (x != 1) return false;
+    return true;
+  };
+  r.coverage_ok = !cover_err && all_one(cq) && all_one(co) && all_one(cg) && all_one(cd) &&
+                  all_one(ca) && all_one(cl);
+  r.targets_ok = true;
+  for (const Instr& I : t.instrs)
+    if (I.dep != kNoCounter && signals[I.dep] != (int64_t)I.dep_target) r.targets_ok = false;
+  if (signals[ctr_lm(D)] != n_sm) r.targets_ok = false;
+  if (!r.coverage_ok && r.error.empty()) r.error = "coverage";
+  if (!r.targets_ok && r.error.empty()) r.error = "targets";
+  return r;
+}
+
+SmemLayout smem_layout(const Dims& D, int nb_max, int max_dyn_smem, int want_pages) {
+  SmemLayout s{};
+  int act = nb_max * std::max(std::max(D.H, D.qdim), D.KS) * 4;
+  // attention scratch: q (rep x d), per-warp probabilities (PL x rep), per-warp partials
+  int attn = D.rep * D.d * 4 + kConsumerWarps * D.PL * D.rep * 4 +
+             kConsumerWarps * D.rep * (D.d + 2) * 4;
+  s.act_bytes = (std::max(act, attn) + 1023) / 1024 * 1024;
+  int misc = 4096;  // mbarriers, reduction scratch, flags
+  int avail = max_dyn_smem - s.act_bytes - misc;
+  int np = avail / kPageBytes;
+  if (want_pages > 0) np = std::min(np, want_pages);
+  s.ring_pages = np;
+  s.bar_off = np * kPageBytes + s.act_bytes;
+  s.misc_off = s.bar_off + 2 * 8 * 64;  // room for up to 64 full + 64 empty barriers
+  s.total = np * kPageBytes + s.act_bytes + misc;
+  return s;
+}
+
+}  // namespace mk

@@ -1,0 +1,67 @@
+"""Summaries of the per-instruction timestamps the kernel records in profile mode.
+
+Create the handle with ``profile=1``; after a step, ``Megakernel.profile_records()``
+returns int64 [n_sm, stride, 8] records (see ``mk_profile_read`` in include/mk.h).
+This module turns them into the time breakdown of one step: per op, how long
+SMs waited on counters, staged activations, computed, and when the last SM of
+each (layer, op) finished -- the critical path through the layer chain.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+OPS = {1: "qkv", 2: "attn", 3: "o", 4: "gu", 5: "down", 6: "lm"}
+
+
+def flatten(rec: np.ndarray) -> list[dict]:
+    rows = []
+    n_sm, stride, _ = rec.shape
+    for s in range(n_sm):
+        for i in range(stride):
+            r = rec[s, i]
+            if r[1] == 0:
+                continue
+            rows.append(dict(sm=s, op=OPS.get(int(r[0]) & 0xFF, "?"), layer=int(r[0] >> 8) & 0xFFFF,
+                             units=int(r[0] >> 24), t_start=int(r[1]), t_dep=int(r[2]),
+                             t_done=int(r[3]), t_sig=int(r[4]), p_first=int(r[5]), p_last=int(r[6])))
+    return rows
+
+
+def summarize(rec: np.ndarray) -> dict:
+    """Aggregate one step's records (nanoseconds; 'critical' is the per-(layer, op)
+    window from the first SM passing its wait to the last SM signalling)."""
+    rows = flatten(rec)
+    if not rows:
+        return {}
+    t0 = min(r["t_start"] for r in rows)
+    t1 = max(r["t_sig"] for r in rows)
+    per_op = {}
+    for r in rows:
+        d = per_op.setdefault(r["op"], dict(n=0, wait=0, work=0, signal=0))
+        d["n"] += 1
+        d["wait"] += r["t_dep"] - r["t_start"]
+        d["work"] += r["t_done"] - r["t_dep"]
+        d["signal"] += r["t_sig"] - r["t_done"]
+    for d in per_op.values():
+        for k in ("wait", "work", "signal"):
+            d[k + "_us_mean"] = d[k] / d["n"] / 1e3
+    phases = {}
+    for r in rows:
+        key = (r["layer"], r["op"])
+        ph = phases.setdefault(key, dict(first_dep=r["t_dep"], last_sig=r["t_sig"], last_dep=r["t_dep"]))
+        ph["first_dep"] = min(ph["first_dep"], r["t_dep"])
+        ph["last_dep"] = max(ph["last_dep"], r["t_dep"])
+        ph["last_sig"] = max(ph["last_sig"], r["t_sig"])
+    crit = {}
+    for (layer, op), ph in phases.items():
+        c = crit.setdefault(op, [])
+        c.append((ph["last_sig"] - ph["first_dep"]) / 1e3)
+    return {
+        "step_us": (t1 - t0) / 1e3,
+        "per_op": {k: {kk: round(vv, 3) if isinstance(vv, float) else vv for kk, vv in v.items()}
+                   for k, v in per_op.items()},
+        "phase_us_mean": {op: round(float(np.mean(v)), 3) for op, v in crit.items()},
+        "phase_end_us": sorted(((ph["last_sig"] - t0) / 1e3, layer, op)
+                               for (layer, op), ph in phases.items()),
+    }
