@@ -25,11 +25,9 @@ struct mk_ctx {
   struct DevTape {
     Instr* instrs = nullptr;
     uint32_t* sm_off = nullptr;
-    uint32_t* units = nullptr;
   };
   std::vector<DevTape> dtapes;
-  LayerW* d_layers = nullptr;
-  const uint16_t *embed = nullptr, *lm = nullptr, *final_norm = nullptr;
+  const uint16_t* embed = nullptr;
   float *x = nullptr, *q = nullptr, *o = nullptr, *a = nullptr, *part = nullptr;
   int2* lm_part = nullptr;
   uint16_t *kcache = nullptr, *vcache = nullptr;
@@ -131,40 +129,38 @@ mk_status check_weights(const mk_config* c, const mk_weights* w) {
   return MK_OK;
 }
 
+// Resolve the device pointers each instruction streams from (see Instr::ptr).
+void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w) {
+  const void* lm = D.tied ? w->embed : w->lm_head;
+  for (Instr& I : t.instrs) {
+    const int l = I.layer;
+    I.ptr[0] = I.ptr[1] = I.ptr[2] = I.ptr[3] = nullptr;
+    switch (I.op) {
+      case OP_QKV: I.ptr[0] = w->wq[l]; I.ptr[1] = w->wk[l]; I.ptr[2] = w->wv[l]; I.ptr[3] = w->attn_norm[l]; break;
+      case OP_O: I.ptr[0] = w->wo[l]; break;
+      case OP_GU: I.ptr[0] = w->w_gate[l]; I.ptr[1] = w->w_up[l]; I.ptr[3] = w->mlp_norm[l]; break;
+      case OP_DOWN: I.ptr[0] = w->w_down[l]; break;
+      case OP_LM: I.ptr[0] = lm; I.ptr[3] = w->final_norm; break;
+      default: break;
+    }
+  }
+}
+
 mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   const Dims& D = h->D;
   // tapes, one per active batch size
   for (int nb = 1; nb <= D.max_batch; ++nb) {
     h->tapes.push_back(lower(D, h->n_sm, nb));
-    const Tape& t = h->tapes.back();
+    Tape& t = h->tapes.back();
+    resolve_pointers(t, D, w);
     mk_ctx::DevTape dt;
     MK_TRY(dalloc(h, &dt.instrs, t.instrs.size()));
     MK_TRY(dalloc(h, &dt.sm_off, t.sm_off.size()));
-    MK_TRY(dalloc(h, &dt.units, t.units.size()));
     MK_TRY(from_cuda(cudaMemcpy(dt.instrs, t.instrs.data(), t.instrs.size() * sizeof(Instr), cudaMemcpyHostToDevice)));
     MK_TRY(from_cuda(cudaMemcpy(dt.sm_off, t.sm_off.data(), t.sm_off.size() * 4, cudaMemcpyHostToDevice)));
-    if (!t.units.empty())
-      MK_TRY(from_cuda(cudaMemcpy(dt.units, t.units.data(), t.units.size() * 4, cudaMemcpyHostToDevice)));
     h->dtapes.push_back(dt);
   }
-  // weights
-  std::vector<LayerW> lw(D.L);
-  for (int l = 0; l < D.L; ++l) {
-    lw[l].attn_norm = (const uint16_t*)w->attn_norm[l];
-    lw[l].wq = (const uint16_t*)w->wq[l];
-    lw[l].wk = (const uint16_t*)w->wk[l];
-    lw[l].wv = (const uint16_t*)w->wv[l];
-    lw[l].wo = (const uint16_t*)w->wo[l];
-    lw[l].mlp_norm = (const uint16_t*)w->mlp_norm[l];
-    lw[l].w_gate = (const uint16_t*)w->w_gate[l];
-    lw[l].w_up = (const uint16_t*)w->w_up[l];
-    lw[l].w_down = (const uint16_t*)w->w_down[l];
-  }
-  MK_TRY(dalloc(h, &h->d_layers, D.L));
-  MK_TRY(from_cuda(cudaMemcpy(h->d_layers, lw.data(), D.L * sizeof(LayerW), cudaMemcpyHostToDevice)));
   h->embed = (const uint16_t*)w->embed;
-  h->lm = D.tied ? h->embed : (const uint16_t*)w->lm_head;
-  h->final_norm = (const uint16_t*)w->final_norm;
   // scratch and state
   const int S1 = h->tapes[0].S;  // nb = 1 has the most slices
   MK_TRY(dalloc(h, &h->x, (size_t)kMaxNB * D.H));
@@ -199,7 +195,7 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   int max_dyn = 0;
   MK_TRY(from_cuda(cudaDeviceGetAttribute(&max_dyn, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev)));
   h->sm = smem_layout(D, h->nbt, max_dyn, want_pages);
-  if (h->sm.ring_pages < 2) return MK_ERR_UNSUPPORTED;
+  if (h->sm.ring_pages < kConsumerWarps) return MK_ERR_UNSUPPORTED;
   if (h->sm.ring_pages > 64) return MK_ERR_UNSUPPORTED;
   const void* kfn[4] = {(const void*)mk_decode_kernel<1>, (const void*)mk_decode_kernel<2>,
                         (const void*)mk_decode_kernel<4>, (const void*)mk_decode_kernel<8>};
@@ -229,12 +225,8 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   KParams p{};
   p.instrs = dt.instrs;
   p.sm_off = dt.sm_off;
-  p.units = dt.units;
   p.S = t.S;
-  p.layers = h->d_layers;
   p.embed = h->embed;
-  p.lm_head = h->lm;
-  p.final_norm = h->final_norm;
   p.x = h->x; p.q = h->q; p.o = h->o; p.a = h->a; p.part = h->part; p.lm_part = h->lm_part;
   p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
   const int par = (int)(h->step & 1);
@@ -346,7 +338,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
     for (const Tape& t : h->tapes)
       for (int sm = 0; sm < h->n_sm; ++sm) stride = std::max(stride, (int)(t.sm_off[sm + 1] - t.sm_off[sm]));
     h->prof_stride = stride;
-    s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * 8);
+    s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * 16);
   }
   if (s == MK_OK && o.debug_fault == 1) {
     // test hook: one wait (the first layer-0 O projection of SM 0's tape for every
@@ -467,11 +459,12 @@ extern "C" mk_status mk_profile_read(mk_handle h, int64_t* out, int64_t cap, int
   *n_sm = h->n_sm;
   *stride = h->prof_stride;
   if (!h->prof) return MK_ERR_INVALID_ARG;
-  const int64_t need = (int64_t)h->n_sm * h->prof_stride * 8;
+  const int64_t need = (int64_t)h->n_sm * h->prof_stride * 16;
   if (!out || cap < need) return MK_ERR_INVALID_ARG;
   cudaSetDevice(h->dev);
   MK_TRY(from_cuda(cudaDeviceSynchronize()));
-  return from_cuda(cudaMemcpy(out, h->prof, need * sizeof(int64_t), cudaMemcpyDeviceToHost));
+  MK_TRY(from_cuda(cudaMemcpy(out, h->prof, need * sizeof(int64_t), cudaMemcpyDeviceToHost)));
+  return from_cuda(cudaMemset(h->prof, 0, need * sizeof(int64_t)));  // accumulators restart
 }
 
 extern "C" mk_status mk_get_error(mk_handle h, char* buf, int32_t len) {

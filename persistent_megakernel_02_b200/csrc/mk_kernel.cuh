@@ -58,13 +58,9 @@ struct KParams {
   // tape of this step's batch size
   const Instr* instrs;
   const uint32_t* sm_off;
-  const uint32_t* units;
   int S;  // attention slices per (lane, kv head)
-  // weights
-  const LayerW* layers;
+  // the embedding table (layer-0 inputs); all other weights are named by the instructions
   const uint16_t* embed;
-  const uint16_t* lm_head;  // == embed when tied
-  const uint16_t* final_norm;
   // state
   float* x;     // [8][H] residual stream
   float* q;     // [8][qdim] rotated queries
@@ -105,6 +101,8 @@ struct Misc {
   uint32_t issued;
   int entry_abort;
 };
+// the misc region is what smem_layout leaves after the barriers: 4096 - 8 * (128 + 64)
+static_assert(sizeof(Misc) <= 4096 - 8 * (128 + 64), "Misc does not fit its shared-memory region");
 
 // ---------------------------------------------------------------- errors & waits
 
@@ -128,7 +126,7 @@ __device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, u
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ld_acquire_u32(c) >= target) return true;
-    if ((it & 15) == 0) {
+    if ((it & 63) == 0) {
       if (aborted(p)) return false;
       if (globaltimer_ns() - t0 > p.wait_limit_ns) {
         raise_error(p, E_WAIT_COUNTER, instr, target, true);
@@ -139,23 +137,46 @@ __device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, u
   }
 }
 
-// Wait for an mbarrier phase.  honor_abort = false is used by the exit drain,
+// Wait for an mbarrier phase.  The abort flag (an L2 load) and the clock are
+// only consulted once a wait has lasted a while, so a page that lands during a
+// short wait is seen at once.  honor_abort = false is used by the exit drain,
 // which must wait for copies in flight even after an abort.
 __device__ __forceinline__ bool wait_mbar(const KParams& p, uint64_t* bar, uint32_t parity,
                                           uint32_t code, uint32_t instr, bool honor_abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 7) == 0) {
+    if ((it & 255) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
       if (honor_abort && aborted(p)) return false;
-      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+      if (now - t0 > p.wait_limit_ns) {
         raise_error(p, code, instr, parity, true);
         return false;
       }
     }
   }
 }
+
+// Position of a page in the ring protocol (see the kernel): its slot and the
+// parity of the slot's use count, its full barrier and that barrier's parity.
+// Advanced incrementally so the hot loops divide by the ring size only once.
+struct RingPos {
+  uint32_t slot, sphase, fidx, fphase;
+  __device__ __forceinline__ void init(uint32_t page, uint32_t NP) {
+    slot = page % NP;
+    sphase = (page / NP) & 1u;
+    fidx = page % (2 * NP);
+    fphase = (page / (2 * NP)) & 1u;
+  }
+  __device__ __forceinline__ void advance(uint32_t n, uint32_t NP) {  // n <= NP
+    slot += n;
+    if (slot >= NP) { slot -= NP; sphase ^= 1u; }
+    fidx += n;
+    if (fidx >= 2 * NP) { fidx -= 2 * NP; fphase ^= 1u; }
+  }
+};
 
 __device__ __forceinline__ size_t kv_offset(const KParams& p, int layer, int b, int page, int g) {
   const Dims& D = p.D;
@@ -170,14 +191,11 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
   const Dims& D = p.D;
   switch (I.op) {
     case OP_QKV: {
-      const LayerW& W = p.layers[I.layer];
       const int half = D.d / 2;
       const int P0 = (int)u * D.RP, hg = P0 / half, i0 = P0 % half;
-      const uint16_t* w;
-      int hh;
-      if (hg < D.Hq) { w = W.wq; hh = hg; }
-      else if (hg < D.Hq + D.Hkv) { w = W.wk; hh = hg - D.Hq; }
-      else { w = W.wv; hh = hg - D.Hq - D.Hkv; }
+      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
+      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+      const uint16_t* w = static_cast<const uint16_t*>(I.ptr[sec]);
       const size_t r0 = (size_t)hh * D.d + i0;
       const uint32_t bytes = (uint32_t)D.RP * D.H * 2;
       mbar_arrive_expect_tx(bar, 2 * bytes);
@@ -189,22 +207,22 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
       const int r0 = (int)u * D.Ro, nr = min(D.Ro, D.H - r0);
       const uint32_t bytes = (uint32_t)nr * D.qdim * 2;
       mbar_arrive_expect_tx(bar, bytes);
-      bulk_g2s(dst, p.layers[I.layer].wo + (size_t)r0 * D.qdim, bytes, bar, pol);
+      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)r0 * D.qdim, bytes, bar, pol);
       break;
     }
     case OP_GU: {
-      const LayerW& W = p.layers[I.layer];
       const int r0 = (int)u * D.Rgu, nr = min(D.Rgu, D.F - r0);
       const uint32_t bytes = (uint32_t)nr * D.H * 2;
       mbar_arrive_expect_tx(bar, 2 * bytes);
-      bulk_g2s(dst, W.w_gate + (size_t)r0 * D.H, bytes, bar, pol);
-      bulk_g2s(dst + (size_t)D.Rgu * D.H * 2, W.w_up + (size_t)r0 * D.H, bytes, bar, pol);
+      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)r0 * D.H, bytes, bar, pol);
+      bulk_g2s(dst + (size_t)D.Rgu * D.H * 2, static_cast<const uint16_t*>(I.ptr[1]) + (size_t)r0 * D.H,
+               bytes, bar, pol);
       break;
     }
     case OP_DOWN: {
       const int r0 = (int)u * D.Rdn, nr = min(D.Rdn, D.H - r0);
       const uint32_t rb = (uint32_t)D.KS * 2;
-      const uint16_t* w = p.layers[I.layer].w_down + (size_t)I.arg * D.KS;
+      const uint16_t* w = static_cast<const uint16_t*>(I.ptr[0]) + (size_t)I.arg * D.KS;
       mbar_arrive_expect_tx(bar, nr * rb);
       for (int r = 0; r < nr; ++r) bulk_g2s(dst + r * rb, w + (size_t)(r0 + r) * D.F, rb, bar, pol);
       break;
@@ -213,12 +231,16 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
       const int r0 = (int)u * D.Rlm, nr = min(D.Rlm, D.V - r0);
       const uint32_t bytes = (uint32_t)nr * D.H * 2;
       mbar_arrive_expect_tx(bar, bytes);
-      bulk_g2s(dst, p.lm_head + (size_t)r0 * D.H, bytes, bar, pol);
+      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)r0 * D.H, bytes, bar, pol);
       break;
     }
   }
 }
 
+// The producer walks this SM's tape and issues every unit's page in order.  It
+// touches global memory only for the tape (the next instruction is loaded while
+// the current one is issued) and the page table; every other address comes from
+// the instruction, so the issue loop never stalls on a dependent load.
 __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                       Misc* misc) {
   const Dims& D = p.D;
@@ -226,48 +248,59 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
   const uint64_t pol = l2_evict_first_policy();
   const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
   uint32_t pidx = 0;
+  RingPos rp;
+  rp.init(0, NP);
   bool ok = true;
+  Instr I;
+  if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1 && ok; ++ii) {
-    const Instr I = p.instrs[ii];
-    long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 8 : nullptr;
-    for (uint32_t k = 0; k < I.n_units && ok; ++k) {
-      const uint32_t u = p.units[I.unit_off + k];
-      if (rec && k == 0) rec[5] = (long long)globaltimer_ns();
-      if (rec && k + 1 == I.n_units) rec[6] = (long long)globaltimer_ns();
-      if (I.op == OP_ATTN) {
-        const int b = u >> 24, g = (u >> 16) & 0xFF, s = u & 0xFFFF;
+    const Instr In = ii + 1 < i1 ? p.instrs[ii + 1] : I;
+    long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 16 : nullptr;
+    long long acc_wait = 0, acc_pages = 0;
+    if (rec) rec[5] = (long long)globaltimer_ns();
+    if (I.op == OP_ATTN) {
+      for (uint32_t k = 0; k < I.n_units && ok; ++k) {
+        int b, g, s;
+        attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
         const int pos = p.pos[b], npg = pos / D.PL + 1;
         const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
         for (int j = pb; j < pe; ++j) {
-          const uint32_t slot = pidx % NP;
-          if (!(ok = wait_mbar(p, &empty[slot], ((pidx / NP) & 1) ^ 1, E_WAIT_EMPTY, ii, true))) break;
+          if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
           // only positions written by earlier steps; the current one is patched in by the consumer
           const int n_old = min(D.PL, pos - j * D.PL);
+          uint64_t* fb = &full[rp.fidx];
           if (n_old > 0) {
             const size_t base = kv_offset(p, I.layer, b, j, g);
             const uint32_t bytes = (uint32_t)n_old * D.d * 2;
-            uint8_t* dst = ring + (size_t)slot * kPageBytes;
-            mbar_arrive_expect_tx(&full[slot], 2 * bytes);
-            bulk_g2s(dst, p.kcache + base, bytes, &full[slot], pol);
-            bulk_g2s(dst + (size_t)D.PL * D.d * 2, p.vcache + base, bytes, &full[slot], pol);
+            uint8_t* dst = ring + (size_t)rp.slot * kPageBytes;
+            mbar_arrive_expect_tx(fb, 2 * bytes);
+            bulk_g2s(dst, p.kcache + base, bytes, fb, pol);
+            bulk_g2s(dst + (size_t)D.PL * D.d * 2, p.vcache + base, bytes, fb, pol);
           } else {
-            mbar_arrive(&full[slot]);
+            mbar_arrive(fb);
           }
           ++pidx;
+          rp.advance(1, NP);
         }
-      } else {
-        const uint32_t slot = pidx % NP;
-        if (!(ok = wait_mbar(p, &empty[slot], ((pidx / NP) & 1) ^ 1, E_WAIT_EMPTY, ii, true))) break;
-        issue_matvec_page(p, I, u, ring + (size_t)slot * kPageBytes, &full[slot], pol);
+      }
+    } else {
+      for (uint32_t k = 0; k < I.n_units; ++k) {
+        const long long tw = rec ? (long long)globaltimer_ns() : 0;
+        if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
+        if (rec) { acc_wait += (long long)globaltimer_ns() - tw; acc_pages += 1; }
+        issue_matvec_page(p, I, I.u0 + k, ring + (size_t)rp.slot * kPageBytes, &full[rp.fidx], pol);
         ++pidx;
+        rp.advance(1, NP);
       }
     }
+    if (rec) { rec[6] = (long long)globaltimer_ns(); rec[9] += acc_wait; rec[10] += acc_pages; }
+    I = In;
   }
   misc->issued = pidx;
   // every copy issued must land before the CTA exits (also after an abort)
   const uint32_t first = pidx > NP ? pidx - NP : 0;
   for (uint32_t q = first; q < pidx; ++q)
-    if (!wait_mbar(p, &full[q % NP], (q / NP) & 1, E_DRAIN, q, false)) break;
+    if (!wait_mbar(p, &full[q % (2 * NP)], (q / (2 * NP)) & 1, E_DRAIN, q, false)) break;
 }
 
 // ---------------------------------------------------------------- consumers: staging
@@ -289,6 +322,12 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
 #pragma unroll
   for (int b = 0; b < NBT; ++b) ss[b] = 0.f;
   for (int c = ct; c < nch; c += 256) {
+    float g[8];
+    if (NORM) {  // the gain is applied here; the 1/rms scale after the reduction
+      const uint4 gw = ldnc16(gain + c * 8);
+      g[0] = bf_lo(gw.x); g[1] = bf_hi(gw.x); g[2] = bf_lo(gw.y); g[3] = bf_hi(gw.y);
+      g[4] = bf_lo(gw.z); g[5] = bf_hi(gw.z); g[6] = bf_lo(gw.w); g[7] = bf_hi(gw.w);
+    }
 #pragma unroll
     for (int b = 0; b < NBT; ++b) {
       float v[8];
@@ -314,7 +353,10 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
       }
       if (NORM) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss[b] = fmaf(v[e], v[e], ss[b]);
+        for (int e = 0; e < 8; ++e) {
+          ss[b] = fmaf(v[e], v[e], ss[b]);
+          v[e] *= g[e];
+        }
       }
       lo[b * nch + c] = make_float4(v[0], v[1], v[2], v[3]);
       hi[b * nch + c] = make_float4(v[4], v[5], v[6], v[7]);
@@ -323,10 +365,10 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
   if (NORM) {
 #pragma unroll
     for (int b = 0; b < NBT; ++b) {
-      float s = ss[b];
+      float t = ss[b];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-      if (lane == 0) misc->red[cw][b] = s;
+      for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+      if (lane == 0) misc->red[cw][b] = t;
     }
     cbar();
     float rinv[NBT];
@@ -338,15 +380,12 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
       rinv[b] = 1.0f / sqrtf(t / (float)K + p.D.eps);
     }
     for (int c = ct; c < nch; c += 256) {
-      const uint4 gw = ldnc16(gain + c * 8);
-      const float g0 = bf_lo(gw.x), g1 = bf_hi(gw.x), g2 = bf_lo(gw.y), g3 = bf_hi(gw.y);
-      const float g4 = bf_lo(gw.z), g5 = bf_hi(gw.z), g6 = bf_lo(gw.w), g7 = bf_hi(gw.w);
 #pragma unroll
       for (int b = 0; b < NBT; ++b) {
         float4 l4 = lo[b * nch + c], h4 = hi[b * nch + c];
         const float r = rinv[b];
-        l4.x = l4.x * r * g0; l4.y = l4.y * r * g1; l4.z = l4.z * r * g2; l4.w = l4.w * r * g3;
-        h4.x = h4.x * r * g4; h4.y = h4.y * r * g5; h4.z = h4.z * r * g6; h4.w = h4.w * r * g7;
+        l4.x *= r; l4.y *= r; l4.z *= r; l4.w *= r;
+        h4.x *= r; h4.y *= r; h4.z *= r; h4.w *= r;
         lo[b * nch + c] = l4;
         hi[b * nch + c] = h4;
       }
@@ -357,34 +396,86 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
 
 // ---------------------------------------------------------------- consumers: matvec
 
-// acc[r][b] += sum_k W[r][k] * act[b][k] over this lane's 8-element chunks.
+// acc[r][b] += W[r][k] * act[b][k] over this lane's 8-element chunks c = lane,
+// lane + 32, ...; two partial sums per row (packed FP32 FMA, FFMA2).  The tile
+// is RT rows of nch chunks in shared memory; act is staged in the split layout.
 template <int RT, int NBT>
-__device__ __forceinline__ void mv_core(uint32_t tile, int nch, const float4* alo, const float4* ahi,
-                                        int lane, float (&acc)[RT][NBT]) {
-#pragma unroll 2
+__device__ __forceinline__ void mv_core(uint32_t tile, uint32_t alo, uint32_t ahi, int nch, int lane,
+                                        float2 (&acc)[RT][NBT]) {
+#pragma unroll 4
   for (int c = lane; c < nch; c += 32) {
-    float4 xl[NBT], xh[NBT];
+    float2 x[NBT][4];
 #pragma unroll
     for (int b = 0; b < NBT; ++b) {
-      xl[b] = alo[b * nch + c];
-      xh[b] = ahi[b * nch + c];
+      const float4 l = lds128f(alo + (uint32_t)(b * nch + c) * 16u);
+      const float4 h = lds128f(ahi + (uint32_t)(b * nch + c) * 16u);
+      x[b][0] = make_float2(l.x, l.y);
+      x[b][1] = make_float2(l.z, l.w);
+      x[b][2] = make_float2(h.x, h.y);
+      x[b][3] = make_float2(h.z, h.w);
     }
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       const uint4 w = lds128(tile + (uint32_t)(r * nch + c) * 16u);
-      const float f0 = bf_lo(w.x), f1 = bf_hi(w.x), f2 = bf_lo(w.y), f3 = bf_hi(w.y);
-      const float f4 = bf_lo(w.z), f5 = bf_hi(w.z), f6 = bf_lo(w.w), f7 = bf_hi(w.w);
+      const float2 w0 = make_float2(bf_lo(w.x), bf_hi(w.x)), w1 = make_float2(bf_lo(w.y), bf_hi(w.y));
+      const float2 w2 = make_float2(bf_lo(w.z), bf_hi(w.z)), w3 = make_float2(bf_lo(w.w), bf_hi(w.w));
 #pragma unroll
       for (int b = 0; b < NBT; ++b) {
-        float s = acc[r][b];
-        s = fmaf(f0, xl[b].x, s); s = fmaf(f1, xl[b].y, s);
-        s = fmaf(f2, xl[b].z, s); s = fmaf(f3, xl[b].w, s);
-        s = fmaf(f4, xh[b].x, s); s = fmaf(f5, xh[b].y, s);
-        s = fmaf(f6, xh[b].z, s); s = fmaf(f7, xh[b].w, s);
+        float2 s = acc[r][b];
+        s = __ffma2_rn(w0, x[b][0], s);
+        s = __ffma2_rn(w1, x[b][1], s);
+        s = __ffma2_rn(w2, x[b][2], s);
+        s = __ffma2_rn(w3, x[b][3], s);
         acc[r][b] = s;
       }
     }
   }
+}
+
+// Warp reduce-scatter of N per-lane values: while more than KEEP values remain,
+// each lane keeps the half picked by its lane bit and adds its partner's copy of
+// that half; the remaining lane bits are reduced in full.  Afterwards every lane
+// holds rs_left(N, KEEP) totals, the first with index rs_base(N, KEEP, lane), and
+// lanes that differ only in the bits of rs_dup_mask hold the same totals.
+template <int N, int n, int KEEP, int O>
+__device__ __forceinline__ void warp_rs(float (&v)[N], int lane) {
+  if constexpr (O > 0) {
+    if constexpr (n > KEEP) {
+      const bool up = (lane & O) != 0;
+#pragma unroll
+      for (int i = 0; i < n / 2; ++i) {
+        const float a = v[i], b = v[i + n / 2];
+        v[i] = (up ? b : a) + __shfl_xor_sync(0xFFFFFFFFu, up ? a : b, O);
+      }
+      warp_rs<N, n / 2, KEEP, O / 2>(v, lane);
+    } else {
+#pragma unroll
+      for (int i = 0; i < n; ++i) v[i] += __shfl_xor_sync(0xFFFFFFFFu, v[i], O);
+      warp_rs<N, n, KEEP, O / 2>(v, lane);
+    }
+  }
+}
+__host__ __device__ constexpr int rs_left(int n, int keep) {
+  for (int o = 16; o >= 1; o >>= 1)
+    if (n > keep) n /= 2;
+  return n;
+}
+__host__ __device__ constexpr int rs_dup_mask(int n, int keep) {
+  int m = 0;
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (n > keep) n /= 2;
+    else m |= o;
+  }
+  return m;
+}
+__device__ __forceinline__ int rs_base(int n, int keep, int lane) {
+  int idx = 0;
+  for (int o = 16; o >= 1; o >>= 1)
+    if (n > keep) {
+      if (lane & o) idx += n / 2;
+      n /= 2;
+    }
+  return idx;
 }
 
 __device__ __forceinline__ bool lm_better(float v, int i, float bv, int bi) {
@@ -400,110 +491,134 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const uint32_t NP = (uint32_t)p.ring_pages;
   const int nch = K >> 3;
-  const float4* alo = reinterpret_cast<const float4*>(act);
-  const float4* ahi = alo + NBT * nch;
+  const uint32_t alo = smem_u32(act);
+  const uint32_t ahi = alo + (uint32_t)(NBT * nch) * 16u;
+  constexpr bool PAIRED = (OPK == OP_QKV || OPK == OP_GU);
+  constexpr int P = PAIRED ? RT / 2 : RT;  // output rows of a unit
+  constexpr int NV = RT * NBT;
+  constexpr int KEEP = PAIRED ? 2 : 1;
+  constexpr int NL = rs_left(NV, KEEP);
+  const int vbase = rs_base(NV, KEEP, lane);
+  const bool writer = (lane & rs_dup_mask(NV, KEEP)) == 0;
   float bestv[NBT];
   int besti[NBT];
 #pragma unroll
   for (int b = 0; b < NBT; ++b) { bestv[b] = -CUDART_INF_F; besti[b] = 0x7FFFFFFF; }
+  long long* prec = (p.prof && cw == 0)
+                        ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - p.sm_off[blockIdx.x])) * 16
+                        : nullptr;
+  long long c_wait = 0, c_pages = 0;
 
-  for (uint32_t k = cw; k < I.n_units; k += kConsumerWarps) {
-    const uint32_t pidx = page_base + k, slot = pidx % NP;
-    bool ok = wait_mbar(p, &full[slot], (pidx / NP) & 1, E_WAIT_FULL, ii, true);
+  RingPos rp;
+  rp.init(page_base + cw, NP);
+  for (uint32_t k = cw; k < I.n_units; k += kConsumerWarps, rp.advance(kConsumerWarps, NP)) {
+    const uint32_t u = I.u0 + k;
+    const uint32_t slot = rp.slot;
+    const long long tw = prec ? (long long)globaltimer_ns() : 0;
+    bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+    if (prec) { c_wait += (long long)globaltimer_ns() - tw; c_pages += 1; }
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) misc->stop = 1;
       break;
     }
-    float acc[RT][NBT];
+    float2 acc[RT][NBT];
 #pragma unroll
     for (int r = 0; r < RT; ++r)
 #pragma unroll
-      for (int b = 0; b < NBT; ++b) acc[r][b] = 0.f;
-    mv_core<RT, NBT>(smem_u32(ring + (size_t)slot * kPageBytes), nch, alo, ahi, lane, acc);
+      for (int b = 0; b < NBT; ++b) acc[r][b] = make_float2(0.f, 0.f);
+    mv_core<RT, NBT>(smem_u32(ring + (size_t)slot * kPageBytes), alo, ahi, nch, lane, acc);
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[slot]);
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int b = 0; b < NBT; ++b) {
-        float s = acc[r][b];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-        acc[r][b] = s;
-      }
-    const uint32_t u = p.units[I.unit_off + k];
+    if (lane == 0) mbar_arrive_cnt(&empty[slot], kConsumerWarps);
 
-    if constexpr (OPK == OP_QKV) {
-      constexpr int RP = RT / 2;
-      const int half = D.d / 2;
-      const int P0 = (int)u * RP, hg = P0 / half, i0 = P0 % half;
-      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
-      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+    float v[NV];
+    if constexpr (PAIRED) {
 #pragma unroll
-      for (int j = 0; j < RP; ++j)
+      for (int j = 0; j < P; ++j)
 #pragma unroll
-        for (int b = 0; b < NBT; ++b) {
-          if (lane != ((j * NBT + b) & 31) || b >= p.nb) continue;
-          const float v1 = acc[j][b], v2 = acc[RP + j][b];
-          const int i = i0 + j, pos = p.pos[b];
-          float r1 = v1, r2 = v2;
-          if (sec < 2) {
-            const float2 cs = p.rope[(size_t)pos * half + i];
-            r1 = v1 * cs.x - v2 * cs.y;
-            r2 = v2 * cs.x + v1 * cs.y;
-          }
-          if (sec == 0) {
-            float* qq = p.q + (size_t)b * D.qdim + hh * D.d;
-            qq[i] = r1;
-            qq[i + half] = r2;
-          } else {
-            const size_t idx = kv_offset(p, I.layer, b, pos / D.PL, hh) + (size_t)(pos % D.PL) * D.d + i;
-            uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
-            cache[idx] = f2bf(r1);
-            cache[idx + half] = f2bf(r2);
-          }
-        }
-    } else if constexpr (OPK == OP_O || OPK == OP_DOWN) {
-      const int R = OPK == OP_O ? D.Ro : D.Rdn;
-      const int r0 = (int)u * R, nr = min(R, D.H - r0);
+        for (int b = 0; b < NBT; ++b)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) v[(j * NBT + b) * 2 + h] = acc[j + h * P][b].x + acc[j + h * P][b].y;
+    } else {
 #pragma unroll
       for (int r = 0; r < RT; ++r)
 #pragma unroll
-        for (int b = 0; b < NBT; ++b)
-          if (lane == ((r * NBT + b) & 31) && r < nr && b < p.nb)
-            red_add_f32(p.x + (size_t)b * D.H + r0 + r, acc[r][b]);
+        for (int b = 0; b < NBT; ++b) v[r * NBT + b] = acc[r][b].x + acc[r][b].y;
+    }
+    warp_rs<NV, NV, KEEP, 16>(v, lane);
+
+    if constexpr (OPK == OP_QKV) {
+      const int half = D.d / 2;
+      const int P0 = (int)u * P, hg = P0 / half, i0 = P0 % half;
+      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
+      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+#pragma unroll
+      for (int m = 0; m < NL / 2; ++m) {
+        const int pi = vbase / 2 + m, j = pi / NBT, b = pi % NBT;
+        if (!writer || b >= p.nb) continue;
+        const float v1 = v[2 * m], v2 = v[2 * m + 1];
+        const int i = i0 + j, pos = p.pos[b];
+        float r1 = v1, r2 = v2;
+        if (sec < 2) {
+          const float2 cs = p.rope[(size_t)pos * half + i];
+          r1 = v1 * cs.x - v2 * cs.y;
+          r2 = v2 * cs.x + v1 * cs.y;
+        }
+        if (sec == 0) {
+          float* qq = p.q + (size_t)b * D.qdim + hh * D.d;
+          qq[i] = r1;
+          qq[i + half] = r2;
+        } else {
+          const size_t idx = kv_offset(p, I.layer, b, pos / D.PL, hh) + (size_t)(pos % D.PL) * D.d + i;
+          uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
+          cache[idx] = f2bf(r1);
+          cache[idx + half] = f2bf(r2);
+        }
+      }
     } else if constexpr (OPK == OP_GU) {
-      constexpr int R = RT / 2;
-      const int r0 = (int)u * R, nr = min(R, D.F - r0);
+      const int r0 = (int)u * P, nr = min(P, D.F - r0);
 #pragma unroll
-      for (int r = 0; r < R; ++r)
+      for (int m = 0; m < NL / 2; ++m) {
+        const int pi = vbase / 2 + m, r = pi / NBT, b = pi % NBT;
+        if (!writer || r >= nr || b >= p.nb) continue;
+        const float g = v[2 * m], up = v[2 * m + 1];
+        p.a[(size_t)b * D.F + r0 + r] = g / (1.0f + __expf(-g)) * up;
+      }
+    } else if constexpr (OPK == OP_O || OPK == OP_DOWN) {
+      const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
 #pragma unroll
-        for (int b = 0; b < NBT; ++b)
-          if (lane == ((r * NBT + b) & 31) && r < nr && b < p.nb) {
-            const float g = acc[r][b], up = acc[R + r][b];
-            p.a[(size_t)b * D.F + r0 + r] = g / (1.0f + __expf(-g)) * up;
-          }
+      for (int m = 0; m < NL; ++m) {
+        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
+        if (writer && r < nr && b < p.nb) red_add_f32(p.x + (size_t)b * D.H + r0 + r, v[m]);
+      }
     } else if constexpr (OPK == OP_LM) {
       const int r0 = (int)u * RT, nr = min(RT, D.V - r0);
 #pragma unroll
-      for (int r = 0; r < RT; ++r) {
-        if (r >= nr) break;
+      for (int m = 0; m < NL; ++m) {
+        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
+        if (r >= nr || b >= p.nb) continue;
 #pragma unroll
-        for (int b = 0; b < NBT; ++b) {
-          if (b >= p.nb) continue;
-          const float v = acc[r][b];
-          if (lm_better(v, r0 + r, bestv[b], besti[b])) { bestv[b] = v; besti[b] = r0 + r; }
-          if (p.logits && lane == ((r * NBT + b) & 31)) p.logits[(size_t)b * D.V + r0 + r] = v;
-        }
+        for (int bb = 0; bb < NBT; ++bb)
+          if (bb == b && lm_better(v[m], r0 + r, bestv[bb], besti[bb])) { bestv[bb] = v[m]; besti[bb] = r0 + r; }
+        if (writer && p.logits) p.logits[(size_t)b * D.V + r0 + r] = v[m];
       }
     }
   }
 
+  if (prec && lane == 0) { prec[7] += c_wait; prec[8] += c_pages; }
   if constexpr (OPK == OP_LM) {
-    // combine the warps' running argmax, publish this SM's, the last SM reduces
-    if (lane == 0)
+    // combine the lanes' and warps' running argmax, publish this SM's, the last SM reduces
 #pragma unroll
-      for (int b = 0; b < NBT; ++b) { misc->lmv[cw][b] = bestv[b]; misc->lmi[cw][b] = besti[b]; }
+    for (int b = 0; b < NBT; ++b) {
+      float bv = bestv[b];
+      int bi = besti[b];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (lm_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+      }
+      if (lane == 0) { misc->lmv[cw][b] = bv; misc->lmi[cw][b] = bi; }
+    }
     cbar();
     if (ct < NBT) {
       float bv = -CUDART_INF_F;
@@ -512,9 +627,9 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         if (lm_better(misc->lmv[w][ct], misc->lmi[w][ct], bv, bi)) { bv = misc->lmv[w][ct]; bi = misc->lmi[w][ct]; }
       p.lm_part[blockIdx.x * kMaxNB + ct] = make_int2(__float_as_int(bv), bi);
     }
-    __threadfence();
     cbar();
     if (ct == 0) {
+      __threadfence();
       const uint32_t old = atom_acq_rel_add(p.ctr + ctr_lm(D), 1u);
       misc->last = (old == gridDim.x - 1) && !misc->stop;
     }
@@ -524,8 +639,8 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
       int bi = 0x7FFFFFFF;
       for (int s = 0; s < (int)gridDim.x; ++s) {
         const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
-        const float v = __int_as_float(e.x);
-        if (lm_better(v, e.y, bv, bi)) { bv = v; bi = e.y; }
+        const float val = __int_as_float(e.x);
+        if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
       }
       p.ids[ct] = (bi >= 0 && bi < D.V) ? bi : 0;
     }
@@ -535,10 +650,12 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
 // ---------------------------------------------------------------- consumers: attention
 
 // Split-KV GQA decode attention for the slices of this instruction.  A slice
-// covers a contiguous range of KV pages of one (lane, kv head); the 8 warps take
-// its pages round-robin, each keeping an online-softmax partial (running max m,
-// sum l, unnormalised output o) for the REP query heads of the group; the CTA
-// combines them into one slice partial, and the last slice to finish (atomic
+// covers a contiguous range of KV pages of one (lane, kv head).  Every page is
+// shared by the 8 warps, each taking PL/8 of its positions: a lane scores one
+// (position, query head) pair, then each warp folds its positions into an
+// online-softmax partial (running max m, sum l, unnormalised o) for the REP
+// query heads of the group.  After the slice the CTA combines the warps'
+// partials into the slice partial, and the last slice to finish (atomic
 // counter) merges all slices of the (lane, kv head) into o.
 template <int DH, int REP>
 __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
@@ -546,22 +663,26 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
                                             Misc* misc, uint32_t ii) {
   constexpr int DC = DH / 8;                 // 16-byte chunks per K/V row
   constexpr int PL = kPageBytes / (4 * DH);  // positions per KV page
-  constexpr int JP = PL / 32;                // score rows per lane
+  constexpr int RPW = PL / kConsumerWarps;   // positions of a page per warp
+  constexpr int PAIRS = RPW * REP;           // (position, head) scores per warp
+  constexpr int SPL = (PAIRS + 31) / 32;     // scores per lane
   constexpr int DPL = DH / 32;               // output dims per lane
   constexpr int CS = DH + 2;                 // partial record: o[DH], m, l
+  static_assert(32 % REP == 0, "REP must divide 32");
   const Dims& D = p.D;
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const uint32_t NP = (uint32_t)p.ring_pages;
   float4* qlo = reinterpret_cast<float4*>(act);
   float4* qhi = qlo + REP * DC;
-  float* pbuf = act + REP * DH + cw * PL * REP;
-  float* comb = act + REP * DH + kConsumerWarps * PL * REP;
+  const uint32_t sqlo = smem_u32(qlo), sqhi = smem_u32(qhi);
+  float* comb = act + REP * DH;
   const float scale = 1.0f / sqrtf((float)DH);
+  const int myh = lane % REP;  // the query head of every score this lane computes
   uint32_t used = 0;
 
   for (uint32_t k = 0; k < I.n_units; ++k) {
-    const uint32_t u = p.units[I.unit_off + k];
-    const int b = u >> 24, g = (u >> 16) & 0xFF, s = u & 0xFFFF;
+    int b, g, s;
+    attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
     const int pos = p.pos[b], npg = pos / PL + 1;
     const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
     const int np_ = pe - pb;
@@ -584,9 +705,11 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
 #pragma unroll
       for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
     }
-    for (int j = cw; j < np_; j += kConsumerWarps) {
-      const uint32_t pidx = page_base + used + j, slot = pidx % NP;
-      bool ok = wait_mbar(p, &full[slot], (pidx / NP) & 1, E_WAIT_FULL, ii, true);
+    RingPos rp;
+    rp.init(page_base + used, NP);
+    for (int j = 0; j < np_; ++j, rp.advance(1, NP)) {
+      const uint32_t slot = rp.slot;
+      bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         if (lane == 0) misc->stop = 1;
         break;
@@ -594,9 +717,11 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
       uint8_t* pg = ring + (size_t)slot * kPageBytes;
       uint8_t* vpg = pg + PL * DH * 2;
       const int p0 = (pb + j) * PL;
-      const int cnt = min(PL, pos + 1 - p0);  // valid rows, >= 1
+      const int cnt = min(PL, pos + 1 - p0);  // valid positions, >= 1
       const int rcur = pos - p0;              // this step's position, if in this page
-      if (rcur < PL) {
+      const int r0 = cw * RPW;
+      const bool patch = rcur >= r0 && rcur < r0 + RPW;
+      if (patch) {  // this step's K/V, written by the QKV instruction, replace the stale copy
         const size_t base = kv_offset(p, I.layer, b, pb + j, g) + (size_t)rcur * DH;
         if constexpr (DH == 64) {
           reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane] =
@@ -611,90 +736,83 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         }
         __syncwarp();
       }
-      // scores s[h][row] = (q_h / sqrt(d)) . k_row; rows lane and lane + 32
-      float sc[REP][JP];
-#pragma unroll
-      for (int h = 0; h < REP; ++h)
-#pragma unroll
-        for (int jj = 0; jj < JP; ++jj) sc[h][jj] = 0.f;
+      // scores: lane -> pair pi = lane + 32 t -> (position r0 + pi / REP, head pi % REP)
+      float sc[SPL];
       const uint32_t kb = smem_u32(pg);
 #pragma unroll
-      for (int cc = 0; cc < DC; ++cc) {
-        const int c = (cc + lane) & (DC - 1);  // rotated so a warp's rows hit distinct banks
-        uint4 kw[JP];
+      for (int t = 0; t < SPL; ++t) {
+        const int pi = lane + 32 * t, row = r0 + pi / REP;
+        float sv = -CUDART_INF_F;
+        if (pi < PAIRS && row < cnt) {
+          float2 a2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int jj = 0; jj < JP; ++jj) kw[jj] = lds128(kb + (uint32_t)(((lane + 32 * jj) * DC + c) * 16));
-#pragma unroll
-        for (int h = 0; h < REP; ++h) {
-          const float4 ql = qlo[h * DC + c], qh = qhi[h * DC + c];
-#pragma unroll
-          for (int jj = 0; jj < JP; ++jj) {
-            float t = sc[h][jj];
-            t = fmaf(bf_lo(kw[jj].x), ql.x, t); t = fmaf(bf_hi(kw[jj].x), ql.y, t);
-            t = fmaf(bf_lo(kw[jj].y), ql.z, t); t = fmaf(bf_hi(kw[jj].y), ql.w, t);
-            t = fmaf(bf_lo(kw[jj].z), qh.x, t); t = fmaf(bf_hi(kw[jj].z), qh.y, t);
-            t = fmaf(bf_lo(kw[jj].w), qh.z, t); t = fmaf(bf_hi(kw[jj].w), qh.w, t);
-            sc[h][jj] = t;
+          for (int cc = 0; cc < DC; ++cc) {
+            const int c = (cc + lane) & (DC - 1);  // lanes of a phase hit distinct banks
+            const uint4 kw = lds128(kb + (uint32_t)((row * DC + c) * 16));
+            const float4 ql = lds128f(sqlo + (uint32_t)((myh * DC + c) * 16));
+            const float4 qh = lds128f(sqhi + (uint32_t)((myh * DC + c) * 16));
+            a2 = __ffma2_rn(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(ql.x, ql.y), a2);
+            a2 = __ffma2_rn(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(ql.z, ql.w), a2);
+            a2 = __ffma2_rn(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(qh.x, qh.y), a2);
+            a2 = __ffma2_rn(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(qh.z, qh.w), a2);
           }
+          sv = a2.x + a2.y;
         }
+        sc[t] = sv;
       }
-      // online softmax update
+      // per-head max over the warp's positions (lanes with equal lane % REP share a head)
+      float mx = sc[0];
+#pragma unroll
+      for (int t = 1; t < SPL; ++t) mx = fmaxf(mx, sc[t]);
+#pragma unroll
+      for (int off = REP; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      float mnew_mine = fmaxf(m[0], mx);
+#pragma unroll
+      for (int h = 1; h < REP; ++h)
+        if (h == myh) mnew_mine = fmaxf(m[h], mx);
+      float pr[SPL], ps = 0.f;
+#pragma unroll
+      for (int t = 0; t < SPL; ++t) {
+        pr[t] = sc[t] > -CUDART_INF_F ? __expf(sc[t] - mnew_mine) : 0.f;
+        ps += pr[t];
+      }
+#pragma unroll
+      for (int off = REP; off < 32; off <<= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
+      // fold into the running state of every head (lane h holds head h's values)
 #pragma unroll
       for (int h = 0; h < REP; ++h) {
-        float mx = -CUDART_INF_F;
-#pragma unroll
-        for (int jj = 0; jj < JP; ++jj)
-          if (lane + 32 * jj < cnt) mx = fmaxf(mx, sc[h][jj]);
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-        const float mnew = fmaxf(m[h], mx);
-        const float corr = __expf(m[h] - mnew);
-        float ps = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < JP; ++jj) {
-          const int row = lane + 32 * jj;
-          const float pr = row < cnt ? __expf(sc[h][jj] - mnew) : 0.f;
-          pbuf[row * REP + h] = pr;
-          ps += pr;
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
-        l[h] = l[h] * corr + ps;
+        const float mh = __shfl_sync(0xFFFFFFFFu, mnew_mine, h);
+        const float sh = __shfl_sync(0xFFFFFFFFu, ps, h);
+        const float corr = mh > -CUDART_INF_F ? __expf(m[h] - mh) : 1.f;
+        l[h] = l[h] * corr + sh;
 #pragma unroll
         for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
-        m[h] = mnew;
+        m[h] = mh;
       }
-      __syncwarp();
-      // o[h][dims of this lane] += p[h][row] * v[row][dims]
-      const uint8_t* vrow = vpg + lane * DPL * 2;
-      for (int r = 0; r < cnt; ++r) {
-        float pv[REP];
-        if constexpr (REP % 4 == 0) {
+      // o[h][dims of this lane] += p[h][position] * v[position][dims]
+      const uint32_t vb = smem_u32(vpg) + (uint32_t)(lane * DPL * 2);
 #pragma unroll
-          for (int h = 0; h < REP; h += 4) {
-            const float4 t = *reinterpret_cast<const float4*>(pbuf + r * REP + h);
-            pv[h] = t.x; pv[h + 1] = t.y; pv[h + 2] = t.z; pv[h + 3] = t.w;
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < REP; ++h) pv[h] = pbuf[r * REP + h];
-        }
+      for (int rr = 0; rr < RPW; ++rr) {
+        if (r0 + rr >= cnt) break;
         float vv[DPL];
         if constexpr (DPL == 2) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(vrow + r * DH * 2);
+          const uint32_t w = lds32(vb + (uint32_t)((r0 + rr) * DH * 2));
           vv[0] = bf_lo(w); vv[1] = bf_hi(w);
         } else {
-          const uint2 w = *reinterpret_cast<const uint2*>(vrow + r * DH * 2);
+          const uint2 w = lds64(vb + (uint32_t)((r0 + rr) * DH * 2));
           vv[0] = bf_lo(w.x); vv[1] = bf_hi(w.x); vv[2] = bf_lo(w.y); vv[3] = bf_hi(w.y);
         }
 #pragma unroll
-        for (int h = 0; h < REP; ++h)
+        for (int h = 0; h < REP; ++h) {
+          const int pi = rr * REP + h;
+          const float ph = __shfl_sync(0xFFFFFFFFu, pr[pi / 32], pi % 32);
 #pragma unroll
-          for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pv[h], vv[e], o[h][e]);
+          for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(ph, vv[e], o[h][e]);
+        }
       }
       __syncwarp();
-      if (rcur < PL) fence_proxy_async_smem();  // generic writes before the next bulk copy
-      if (lane == 0) mbar_arrive(&empty[slot]);
+      if (patch) fence_proxy_async_smem();  // generic writes before the next bulk copy
+      if (lane == 0) mbar_arrive_cnt(&empty[slot], 1u);  // one of the 8 warps
     }
     // combine the warps' partials into this slice's partial
     float* mine = comb + cw * REP * CS;
@@ -724,9 +842,9 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
       part[h * CS + i] = O;
       if (i == 0) { part[h * CS + DH] = M; part[h * CS + DH + 1] = L; }
     }
-    __threadfence();
     cbar();
     if (ct == 0) {
+      __threadfence();
       const uint32_t old = atom_acq_rel_add(p.ctr + ctr_part(D, I.layer, b, g), 1u);
       misc->last = (old == (uint32_t)p.S - 1);
     }
@@ -748,9 +866,11 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         }
         p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
       }
-      __threadfence();
       cbar();
-      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      if (ct == 0) {
+        __threadfence();
+        red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      }
     }
     used += (uint32_t)np_;
     cbar();
@@ -791,9 +911,11 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   const int ct = threadIdx.x - 32;
   const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
   uint32_t page_base = 0;
+  Instr I;
+  if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1; ++ii) {
-    const Instr I = p.instrs[ii];
-    long long* rec = (p.prof && ct == 0) ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 8 : nullptr;
+    const Instr In = ii + 1 < i1 ? p.instrs[ii + 1] : I;  // loaded while this one runs
+    long long* rec = (p.prof && ct == 0) ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 16 : nullptr;
     if (rec) {
       rec[0] = (long long)I.op | ((long long)I.layer << 8) | ((long long)I.n_units << 24);
       rec[1] = (long long)globaltimer_ns();
@@ -806,7 +928,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     uint32_t used = I.n_units;  // one page per unit, except attention
     switch (I.op) {
       case OP_QKV: {
-        const LayerW& W = p.layers[I.layer];
+        const uint16_t* gain = static_cast<const uint16_t*>(I.ptr[3]);
         if (I.layer == 0) {
           if (ct < NBT) {
             int t = ct < p.nb ? p.tokens[ct] : 0;
@@ -817,9 +939,9 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
             misc->tok[ct] = t;
           }
           cbar();
-          stage<NBT, true, true>(p, act, misc, nullptr, 0, D.H, W.attn_norm, (int)I.aux0, (int)I.aux1);
+          stage<NBT, true, true>(p, act, misc, nullptr, 0, D.H, gain, (int)I.aux0, (int)I.aux1);
         } else {
-          stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, W.attn_norm, 0, 0);
+          stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, gain, 0, 0);
         }
         mv_dispatch<OP_QKV, NBT>(2 * D.RP, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
@@ -833,7 +955,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         mv_dispatch<OP_O, NBT>(D.Ro, p, I, page_base, ring, act, D.qdim, full, empty, misc, ii);
         break;
       case OP_GU:
-        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, p.layers[I.layer].mlp_norm, 0, 0);
+        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), 0, 0);
         mv_dispatch<OP_GU, NBT>(2 * D.Rgu, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
       case OP_DOWN:
@@ -841,16 +963,19 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         mv_dispatch<OP_DOWN, NBT>(D.Rdn, p, I, page_base, ring, act, D.KS, full, empty, misc, ii);
         break;
       case OP_LM:
-        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, p.final_norm, 0, 0);
+        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), 0, 0);
         mv_dispatch<OP_LM, NBT>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
     }
     page_base += used;
     if (rec) rec[3] = (long long)globaltimer_ns();
-    __threadfence();
     cbar();
     if (misc->stop) break;
-    if (ct == 0 && I.sig != kNoCounter) red_release_add(p.ctr + I.sig, 1u);
+    if (ct == 0 && I.sig != kNoCounter) {
+      __threadfence();  // publishes the CTA's writes (ordered before it by the barrier)
+      red_release_add(p.ctr + I.sig, 1u);
+    }
+    I = In;
     if (rec) rec[4] = (long long)globaltimer_ns();
   }
 }
@@ -861,16 +986,21 @@ template <int NBT>
 __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Misc* misc = reinterpret_cast<Misc*>(smem + p.misc_off);
+  // Ring protocol.  Page i (in this SM's stream order) goes to slot i % NP and
+  // completes full barrier i % (2 NP), phase parity (i / (2 NP)) & 1; its slot is
+  // released on empty barrier i % NP by 8 warp arrivals.  A consumer only waits on
+  // page i after page i - NP was issued (NP >= 8 consumer warps, each taking
+  // pages in order), so page i - 2 NP -- the previous user of the same full
+  // barrier -- has been consumed and the parity wait cannot alias an older phase,
+  // even when bulk copies land out of order.
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
-  uint64_t* empty = full + 64;
+  uint64_t* empty = full + 128;
   // the next step's counters start from zero (this step's were zeroed by the previous one)
   for (int i = blockIdx.x * kThreads + threadIdx.x; i < p.n_counters; i += gridDim.x * kThreads)
     p.ctr_next[i] = 0u;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < p.ring_pages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
+    for (int i = 0; i < 2 * p.ring_pages; ++i) mbar_init(&full[i], 1);
+    for (int i = 0; i < p.ring_pages; ++i) mbar_init(&empty[i], kConsumerWarps);
     fence_barrier_init();
     fence_proxy_async_smem();
     misc->stop = 0;

@@ -4,9 +4,10 @@
 // The per-SM "execution plan" of the Hazy megakernel article (section
 // "Megakernel: a deep-fusion design from scratch"): an ordered list of fused
 // instructions per SM whose dependencies are fixed before the run.  Here an
-// instruction names an op, a layer, a list of work units (each unit is exactly
-// one shared-memory page of weights, or one attention slice), the counter it
-// waits on with its target, and the counter it bumps when done.
+// instruction names an op, a layer, a contiguous range of work units (each unit
+// is exactly one shared-memory page of weights, or one attention slice), the
+// counter it waits on with its target, and the counter it bumps when done.
+// Ranges keep the kernel free of per-unit table lookups: a unit id is u0 + k.
 #pragma once
 
 #include <stdint.h>
@@ -41,19 +42,24 @@ constexpr uint16_t kNoCounter = 0xFFFF;
 // counters of one layer
 enum : int { C_QKV = 0, C_ATTN = 1, C_O = 2, C_GU = 3, C_DOWN = 4, kCountersPerLayer = 5 };
 
-struct Instr {            // 32 bytes
+struct Instr {            // 64 bytes
   uint8_t op;
   uint8_t arg;            // OP_DOWN: K-slice index
   uint16_t layer;
-  uint32_t unit_off;      // first unit in the tape's unit array
+  uint32_t u0;            // units of the instruction are u0 .. u0 + n_units - 1
   uint32_t n_units;
   uint16_t dep;           // counter waited on before the instruction (kNoCounter: none)
   uint16_t sig;           // counter incremented once when the instruction is done
   uint32_t dep_target;    // value `dep` must reach in this step
   uint32_t aux0, aux1;    // OP_QKV at layer 0: residual rows [aux0, aux1) this SM seeds
   uint32_t pad;
+  // device pointers resolved when the handle is created, so the kernel needs no
+  // table lookup per instruction: [0..2] the weight matrices the producer
+  // streams (QKV: Wq, Wk, Wv; O: Wo; GU: Wgate, Wup; DOWN: Wdown; LM: the head),
+  // [3] the bf16 RMSNorm gain the consumers stage with (QKV, GU, LM)
+  const void* ptr[4];
 };
-static_assert(sizeof(Instr) == 32, "Instr layout");
+static_assert(sizeof(Instr) == 64, "Instr layout");
 
 // Shape parameters of one handle (identical for every tape of the handle).
 struct Dims {
@@ -77,7 +83,6 @@ struct Tape {
   int n_counters = 0;
   std::vector<uint32_t> sm_off;   // n_sm + 1 offsets into instrs
   std::vector<Instr> instrs;
-  std::vector<uint32_t> units;
 };
 
 // lanes the kernel is instantiated for: the batch size rounded up to 1, 2, 4 or 8
@@ -90,7 +95,13 @@ MK_HD inline int ctr_part(const Dims& D, int layer, int b, int g) {
 MK_HD inline int ctr_lm(const Dims& D) { return D.L * kCountersPerLayer + D.L * kMaxNB * D.Hkv; }
 MK_HD inline int n_counters(const Dims& D) { return ctr_lm(D) + 1; }
 
-MK_HD inline uint32_t attn_unit(int b, int g, int s) { return (uint32_t(b) << 24) | (uint32_t(g) << 16) | uint32_t(s); }
+// attention unit i = (lane * Hkv + kv head) * S + slice
+MK_HD inline void attn_unit(uint32_t i, int Hkv, int S, int* b, int* g, int* s) {
+  *s = (int)(i % (uint32_t)S);
+  const uint32_t bg = i / (uint32_t)S;
+  *g = (int)(bg % (uint32_t)Hkv);
+  *b = (int)(bg / (uint32_t)Hkv);
+}
 
 // Shape derivation and tape lowering (mk_sched.cpp).
 std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, int head_dim,

@@ -116,20 +116,28 @@ namespace {
 struct Assigner {
   std::vector<int64_t>& load;
   explicit Assigner(std::vector<int64_t>& l) : load(l) {}
-  // Give each of n equal units to the least-loaded SM of [lo, hi) (ties: lowest id).
+  // Split n equal units over the SMs of [lo, hi): how many each SM gets is decided
+  // by cumulative bytes (the least-loaded SM takes the next unit, ties: lowest
+  // id), and each SM receives a CONTIGUOUS range of units, in SM order.  Keeping
+  // an SM's weights of one phase contiguous keeps its bulk copies within a few
+  // GPU pages instead of one new page per copy.
   std::vector<std::vector<uint32_t>> run(int n, int64_t bytes, int lo, int hi) {
     using E = std::pair<int64_t, int>;
     std::priority_queue<E, std::vector<E>, std::greater<E>> pq;
     for (int s = lo; s < hi; ++s) pq.push({load[s], s});
-    std::vector<std::vector<uint32_t>> out(load.size());
+    std::vector<int> count(load.size(), 0);
     for (int u = 0; u < n; ++u) {
       E e = pq.top();
       pq.pop();
-      out[e.second].push_back((uint32_t)u);
+      count[e.second]++;
       e.first += bytes;
       load[e.second] = e.first;
       pq.push(e);
     }
+    std::vector<std::vector<uint32_t>> out(load.size());
+    uint32_t u = 0;
+    for (int s = lo; s < hi; ++s)
+      for (int c = 0; c < count[s]; ++c) out[s].push_back(u++);
     return out;
   }
 };
@@ -143,16 +151,17 @@ Tape lower(const Dims& D, int n_sm, int nb) {
   std::vector<int64_t> load(n_sm, 0);
   Assigner as(load);
   std::vector<std::vector<Instr>> ins(n_sm);
-  std::vector<std::vector<uint32_t>> uts(n_sm);
 
+  // units must form one contiguous range per instruction (the Assigner's output)
   auto emit = [&](int sm, uint8_t op, int layer, const std::vector<uint32_t>& units, uint16_t dep,
                   uint16_t sig, uint8_t arg) -> Instr& {
     Instr I{};
     I.op = op; I.arg = arg; I.layer = (uint16_t)layer;
-    I.unit_off = (uint32_t)uts[sm].size();  // rebased when the tapes are concatenated
+    I.u0 = units.empty() ? 0u : units[0];
     I.n_units = (uint32_t)units.size();
+    for (size_t k = 1; k < units.size(); ++k)
+      if (units[k] != units[0] + k) I.n_units = 0xFFFFFFFFu;  // not a range: simulate() reports it
     I.dep = dep; I.sig = sig; I.dep_target = 0;
-    uts[sm].insert(uts[sm].end(), units.begin(), units.end());
     ins[sm].push_back(I);
     return ins[sm].back();
   };
@@ -176,15 +185,8 @@ Tape lower(const Dims& D, int n_sm, int nb) {
     {
       int n = nb * D.Hkv * t.S;
       auto at = as.run(n, unit_bytes(D, OP_ATTN, t.S), 0, n_sm);
-      for (int s = 0; s < n_sm; ++s) {
-        if (at[s].empty()) continue;
-        std::vector<uint32_t> u;
-        for (uint32_t i : at[s]) {
-          int b = i / (D.Hkv * t.S), g = (i / t.S) % D.Hkv, sl = i % t.S;
-          u.push_back(attn_unit(b, g, sl));
-        }
-        emit(s, OP_ATTN, l, u, (uint16_t)ctr_layer(l, C_QKV), kNoCounter, 0);
-      }
+      for (int s = 0; s < n_sm; ++s)
+        if (!at[s].empty()) emit(s, OP_ATTN, l, at[s], (uint16_t)ctr_layer(l, C_QKV), kNoCounter, 0);
     }
     // O projection + residual
     auto o = as.run(D.n_o, unit_bytes(D, OP_O, t.S), 0, n_sm);
@@ -224,12 +226,7 @@ Tape lower(const Dims& D, int n_sm, int nb) {
   t.sm_off.assign(n_sm + 1, 0);
   for (int s = 0; s < n_sm; ++s) {
     t.sm_off[s] = (uint32_t)t.instrs.size();
-    uint32_t base = (uint32_t)t.units.size();
-    for (auto I : ins[s]) {
-      I.unit_off += base;
-      t.instrs.push_back(I);
-    }
-    t.units.insert(t.units.end(), uts[s].begin(), uts[s].end());
+    t.instrs.insert(t.instrs.end(), ins[s].begin(), ins[s].end());
   }
   t.sm_off[n_sm] = (uint32_t)t.instrs.size();
   return t;
@@ -252,7 +249,7 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
     r.max_instr_per_sm = std::max(r.max_instr_per_sm, n);
     int64_t by = 0;
     for (uint32_t i = t.sm_off[s]; i < t.sm_off[s + 1]; ++i)
-      by += unit_bytes(D, t.instrs[i].op, S) * t.instrs[i].n_units;
+      if (t.instrs[i].n_units != 0xFFFFFFFFu) by += unit_bytes(D, t.instrs[i].op, S) * t.instrs[i].n_units;
     r.bytes_min = std::min(r.bytes_min, by);
     r.bytes_max = std::max(r.bytes_max, by);
   }
@@ -270,8 +267,9 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
         const Instr& I = t.instrs[ip[s]];
         if (I.dep != kNoCounter && ctr[I.dep] < (int64_t)I.dep_target) break;
         int l = I.layer;
+        if (I.n_units == 0xFFFFFFFFu) { cover_err = true; ip[s]++; progress = true; continue; }
         for (uint32_t k = 0; k < I.n_units; ++k) {
-          uint32_t u = t.units[I.unit_off + k];
+          uint32_t u = I.u0 + k;
           switch (I.op) {
             case OP_QKV: bump(cq, (size_t)l * D.n_qkv + u); break;
             case OP_O: bump(co, (size_t)l * D.n_o + u); break;
@@ -279,7 +277,8 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
             case OP_DOWN: bump(cd, ((size_t)l * D.n_ks + I.arg) * D.n_dn + u); break;
             case OP_LM: bump(cl, u); break;
             case OP_ATTN: {
-              int b = u >> 24, g = (u >> 16) & 0xFF, sl = u & 0xFFFF;
+              int b, g, sl;
+              attn_unit(u, D.Hkv, S, &b, &g, &sl);
               if (b >= nb || g >= D.Hkv || sl >= S) { cover_err = true; break; }
               bump(ca, (((size_t)l * nb + b) * D.Hkv + g) * S + sl);
               size_t pi = ((size_t)l * kMaxNB + b) * D.Hkv + g;
@@ -324,17 +323,17 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
 SmemLayout smem_layout(const Dims& D, int nb_max, int max_dyn_smem, int want_pages) {
   SmemLayout s{};
   int act = nb_max * std::max(std::max(D.H, D.qdim), D.KS) * 4;
-  // attention scratch: q (rep x d), per-warp probabilities (PL x rep), per-warp partials
-  int attn = D.rep * D.d * 4 + kConsumerWarps * D.PL * D.rep * 4 +
-             kConsumerWarps * D.rep * (D.d + 2) * 4;
+  // attention scratch: q (rep x d) and the per-warp partials (rep x (d + 2))
+  int attn = D.rep * D.d * 4 + kConsumerWarps * D.rep * (D.d + 2) * 4;
   s.act_bytes = (std::max(act, attn) + 1023) / 1024 * 1024;
-  int misc = 4096;  // mbarriers, reduction scratch, flags
+  int misc = 4096;  // mbarriers (128 full + 64 empty), reduction scratch, flags
   int avail = max_dyn_smem - s.act_bytes - misc;
-  int np = avail / kPageBytes;
-  if (want_pages > 0) np = std::min(np, want_pages);
+  int np = std::min(64, avail / kPageBytes);
+  // the ring protocol needs at least one page per consumer warp
+  if (want_pages > 0) np = std::min(np, std::max(want_pages, kConsumerWarps));
   s.ring_pages = np;
   s.bar_off = np * kPageBytes + s.act_bytes;
-  s.misc_off = s.bar_off + 2 * 8 * 64;  // room for up to 64 full + 64 empty barriers
+  s.misc_off = s.bar_off + 8 * (128 + 64);  // 2 NP full + NP empty barriers, NP <= 64
   s.total = np * kPageBytes + s.act_bytes + misc;
   return s;
 }

@@ -24,7 +24,8 @@ def flatten(rec: np.ndarray) -> list[dict]:
                 continue
             rows.append(dict(sm=s, op=OPS.get(int(r[0]) & 0xFF, "?"), layer=int(r[0] >> 8) & 0xFFFF,
                              units=int(r[0] >> 24), t_start=int(r[1]), t_dep=int(r[2]),
-                             t_done=int(r[3]), t_sig=int(r[4]), p_first=int(r[5]), p_last=int(r[6])))
+                             t_done=int(r[3]), t_sig=int(r[4]), p_first=int(r[5]), p_last=int(r[6]),
+                             c_wait=int(r[7]), c_pages=int(r[8]), p_wait=int(r[9]), p_pages=int(r[10])))
     return rows
 
 
@@ -38,14 +39,19 @@ def summarize(rec: np.ndarray) -> dict:
     t1 = max(r["t_sig"] for r in rows)
     per_op = {}
     for r in rows:
-        d = per_op.setdefault(r["op"], dict(n=0, wait=0, work=0, signal=0))
+        d = per_op.setdefault(r["op"], dict(n=0, wait=0, work=0, signal=0, c_wait=0, c_pages=0,
+                                            p_wait=0, p_pages=0))
         d["n"] += 1
+        for k in ("c_wait", "c_pages", "p_wait", "p_pages"):
+            d[k] += r[k]
         d["wait"] += r["t_dep"] - r["t_start"]
         d["work"] += r["t_done"] - r["t_dep"]
         d["signal"] += r["t_sig"] - r["t_done"]
     for d in per_op.values():
         for k in ("wait", "work", "signal"):
             d[k + "_us_mean"] = d[k] / d["n"] / 1e3
+        d["c_wait_us_per_page"] = d["c_wait"] / max(1, d["c_pages"]) / 1e3
+        d["p_wait_us_per_page"] = d["p_wait"] / max(1, d["p_pages"]) / 1e3
     phases = {}
     for r in rows:
         key = (r["layer"], r["op"])
