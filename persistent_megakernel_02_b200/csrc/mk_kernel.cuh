@@ -84,7 +84,7 @@ struct KParams {
   float* logits;  // device [nb][V] or null
   int* ids;       // device [nb]
   unsigned long long wait_limit_ns;
-  long long* prof;   // profile records [n_sm][prof_stride][8] or null
+  long long* prof;   // profile records [n_sm][prof_stride][16] or null
   int prof_stride;
   // shared memory layout
   int ring_pages, act_off, bar_off, misc_off;
@@ -98,7 +98,7 @@ struct Misc {
   int tok[kMaxNB];
   volatile int stop;
   volatile int last;
-  uint32_t issued;
+  uint32_t issued;  // pages the ring producer issued
   int entry_abort;
 };
 // the misc region is what smem_layout leaves after the barriers: 4096 - 8 * (128 + 64)
@@ -177,6 +177,11 @@ struct RingPos {
     if (fidx >= 2 * NP) { fidx -= 2 * NP; fphase ^= 1u; }
   }
 };
+
+// Slices actually used for a (lane, kv head) with npg KV pages: about one per
+// two pages, at most the tape's S.  A short context is then one slice, which
+// writes its output directly instead of through partials and a merge.
+__device__ __forceinline__ int attn_slices_used(int S, int npg) { return max(1, min(S, npg / 2)); }
 
 __device__ __forceinline__ size_t kv_offset(const KParams& p, int layer, int b, int page, int g) {
   const Dims& D = p.D;
@@ -262,8 +267,9 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
       for (uint32_t k = 0; k < I.n_units && ok; ++k) {
         int b, g, s;
         attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-        const int pos = p.pos[b], npg = pos / D.PL + 1;
-        const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
+        const int pos = p.pos[b], npg = pos / D.PL + 1, se = attn_slices_used(p.S, npg);
+        if (s >= se) continue;
+        const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
         for (int j = pb; j < pe; ++j) {
           if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
           // only positions written by earlier steps; the current one is patched in by the consumer
@@ -629,7 +635,6 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
     }
     cbar();
     if (ct == 0) {
-      __threadfence();
       const uint32_t old = atom_acq_rel_add(p.ctr + ctr_lm(D), 1u);
       misc->last = (old == gridDim.x - 1) && !misc->stop;
     }
@@ -683,8 +688,9 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
   for (uint32_t k = 0; k < I.n_units; ++k) {
     int b, g, s;
     attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-    const int pos = p.pos[b], npg = pos / PL + 1;
-    const int pb = (int)((long long)s * npg / p.S), pe = (int)((long long)(s + 1) * npg / p.S);
+    const int pos = p.pos[b], npg = pos / PL + 1, se = attn_slices_used(p.S, npg);
+    if (s >= se) continue;  // uniform: this slice is not needed at this context length
+    const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
     const int np_ = pe - pb;
     for (int e = ct; e < REP * DC; e += 256) {
       const int h = e / DC, c = e % DC;
@@ -824,6 +830,29 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     }
     cbar();
     if (misc->stop) { cbar(); break; }
+    if (se == 1) {
+      // the only slice: normalise and write the output, then signal
+      for (int e = ct; e < REP * DH; e += 256) {
+        const int h = e / DH, i = e % DH;
+        float M = -CUDART_INF_F;
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * REP + h) * CS + DH]);
+        float L = 0.f, O = 0.f;
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float mw = comb[(w * REP + h) * CS + DH];
+          if (mw > -CUDART_INF_F) {
+            const float f = __expf(mw - M);
+            L += comb[(w * REP + h) * CS + DH + 1] * f;
+            O += comb[(w * REP + h) * CS + i] * f;
+          }
+        }
+        p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
+      }
+      cbar();
+      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      used += (uint32_t)np_;
+      cbar();
+      continue;
+    }
     float* part = p.part + ((size_t)(b * D.Hkv + g) * p.S + s) * REP * CS;
     for (int e = ct; e < REP * DH; e += 256) {
       const int h = e / DH, i = e % DH;
@@ -844,9 +873,8 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     }
     cbar();
     if (ct == 0) {
-      __threadfence();
       const uint32_t old = atom_acq_rel_add(p.ctr + ctr_part(D, I.layer, b, g), 1u);
-      misc->last = (old == (uint32_t)p.S - 1);
+      misc->last = (old == (uint32_t)se - 1);
     }
     cbar();
     if (misc->last) {
@@ -854,9 +882,9 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
       for (int e = ct; e < REP * DH; e += 256) {
         const int h = e / DH, i = e % DH;
         float M = -CUDART_INF_F;
-        for (int t = 0; t < p.S; ++t) M = fmaxf(M, __ldcg(pp + (t * REP + h) * CS + DH));
+        for (int t = 0; t < se; ++t) M = fmaxf(M, __ldcg(pp + (t * REP + h) * CS + DH));
         float L = 0.f, O = 0.f;
-        for (int t = 0; t < p.S; ++t) {
+        for (int t = 0; t < se; ++t) {
           const float mt = __ldcg(pp + (t * REP + h) * CS + DH);
           if (mt > -CUDART_INF_F) {
             const float f = __expf(mt - M);
@@ -867,10 +895,7 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
       }
       cbar();
-      if (ct == 0) {
-        __threadfence();
-        red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
-      }
+      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
     }
     used += (uint32_t)np_;
     cbar();
@@ -971,10 +996,9 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     if (rec) rec[3] = (long long)globaltimer_ns();
     cbar();
     if (misc->stop) break;
-    if (ct == 0 && I.sig != kNoCounter) {
-      __threadfence();  // publishes the CTA's writes (ordered before it by the barrier)
-      red_release_add(p.ctr + I.sig, 1u);
-    }
+    // the barrier orders every consumer thread's writes before thread 0's release,
+    // which is cumulative, so one release publishes the whole CTA's results
+    if (ct == 0 && I.sig != kNoCounter) red_release_add(p.ctr + I.sig, 1u);
     I = In;
     if (rec) rec[4] = (long long)globaltimer_ns();
   }
@@ -1010,9 +1034,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   }
   __syncthreads();
   if (!misc->entry_abort) {
-    if (threadIdx.x < 32) {
+    const int warp = threadIdx.x >> 5;
+    if (warp == 0) {
       if (threadIdx.x == 0) producer(p, smem, full, empty, misc);
-    } else {
+    } else if (warp <= kConsumerWarps) {
       consumer<NBT>(p, smem, reinterpret_cast<float*>(smem + p.act_off), full, empty, misc);
     }
   }

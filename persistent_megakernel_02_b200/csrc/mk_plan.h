@@ -34,7 +34,7 @@ enum Op : uint8_t {
 
 constexpr int kPageBytes = 16384;      // one ring page
 constexpr int kMaxNB = 8;              // lanes (sequences) per step
-constexpr int kConsumerWarps = 8;      // warps that compute; warp 0 loads
+constexpr int kConsumerWarps = 8;      // warps 1..8 compute; warp 0 loads the ring
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
 constexpr int kActFloatsMax = 16384;   // max_batch * K of the staged activation
 constexpr uint16_t kNoCounter = 0xFFFF;

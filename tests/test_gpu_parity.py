@@ -89,6 +89,27 @@ def test_tiny_batch_of_three_lanes():
             H.compare_ids(ids[t, b], w_steps[t])
 
 
+@pytest.mark.parametrize("lens", [[300], [520, 130]])
+def test_tiny_long_context_split_attention(lens):
+    """Contexts of several KV pages are split over SMs and merged (online-softmax
+    partials); lanes of one step use different splits."""
+    nb = len(lens)
+    cfg = configs.model_config("tiny", max_batch=nb, max_seq=max(lens) + 8)
+    w = H.gpu_weights(cfg)
+    prompts = [synth.prompt_tokens(cfg, b, n).numpy() for b, n in enumerate(lens)]
+    teacher = [synth.teacher_tokens(cfg, b, 6).numpy() for b in range(nb)]
+    mk = _mk(cfg, w)
+    pre, lg, ids = H.run_teacher_forced(mk, cfg, prompts, teacher, 6)
+    mk.close()
+    orc = H.oracle_for(cfg, w)
+    for b in range(nb):
+        w_pre, w_steps = H.oracle_teacher_forced(orc, prompts[b], teacher[b], 6)
+        H.compare_logits(pre[b], w_pre, f"lane {b} prefill")
+        for t in range(6):
+            H.compare_logits(lg[t, b], w_steps[t], f"lane {b} step {t}")
+            H.compare_ids(ids[t, b], w_steps[t])
+
+
 def test_tiny_free_run_greedy_chained_on_device():
     wlc = configs.WORKLOADS["tiny"]
     cfg = configs.model_config("tiny")
