@@ -96,13 +96,15 @@ struct Misc {
   float lmv[kConsumerWarps][kMaxNB];
   int lmi[kConsumerWarps][kMaxNB];
   int tok[kMaxNB];
+  int cur_phys[kMaxNB];  // physical KV page holding each lane's position this step
+  float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
   volatile int stop;
   volatile int last;
   uint32_t issued;  // pages the ring producer issued
   int entry_abort;
 };
-// the misc region is what smem_layout leaves after the barriers: 4096 - 8 * (128 + 64)
-static_assert(sizeof(Misc) <= 4096 - 8 * (128 + 64), "Misc does not fit its shared-memory region");
+// the misc region is what smem_layout leaves after the barriers: 8192 - 8 * (128 + 64)
+static_assert(sizeof(Misc) <= 8192 - 8 * (128 + 64), "Misc does not fit its shared-memory region");
 
 // ---------------------------------------------------------------- errors & waits
 
@@ -182,12 +184,6 @@ struct RingPos {
 // two pages, at most the tape's S.  A short context is then one slice, which
 // writes its output directly instead of through partials and a merge.
 __device__ __forceinline__ int attn_slices_used(int S, int npg) { return max(1, min(S, npg / 2)); }
-
-__device__ __forceinline__ size_t kv_offset(const KParams& p, int layer, int b, int page, int g) {
-  const Dims& D = p.D;
-  const int phys = p.page_table[p.slot[b] * D.pages_per_seq + page];
-  return (((size_t)layer * D.n_phys_pages + phys) * D.Hkv + g) * (size_t)(D.PL * D.d);
-}
 
 // ---------------------------------------------------------------- producer
 
@@ -270,13 +266,17 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
         const int pos = p.pos[b], npg = pos / D.PL + 1, se = attn_slices_used(p.S, npg);
         if (s >= se) continue;
         const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
+        const int* pt = p.page_table + p.slot[b] * D.pages_per_seq;
+        int phys_next = pb < pe ? pt[pb] : 0;
         for (int j = pb; j < pe; ++j) {
+          const int phys = phys_next;
+          if (j + 1 < pe) phys_next = pt[j + 1];  // in flight while this page is issued
           if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
           // only positions written by earlier steps; the current one is patched in by the consumer
           const int n_old = min(D.PL, pos - j * D.PL);
           uint64_t* fb = &full[rp.fidx];
           if (n_old > 0) {
-            const size_t base = kv_offset(p, I.layer, b, j, g);
+            const size_t base = (((size_t)I.layer * D.n_phys_pages + phys) * D.Hkv + g) * (size_t)(D.PL * D.d);
             const uint32_t bytes = (uint32_t)n_old * D.d * 2;
             uint8_t* dst = ring + (size_t)rp.slot * kPageBytes;
             mbar_arrive_expect_tx(fb, 2 * bytes);
@@ -565,7 +565,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         const int i = i0 + j, pos = p.pos[b];
         float r1 = v1, r2 = v2;
         if (sec < 2) {
-          const float2 cs = p.rope[(size_t)pos * half + i];
+          const float2 cs = misc->rope_cs[b][i];
           r1 = v1 * cs.x - v2 * cs.y;
           r2 = v2 * cs.x + v1 * cs.y;
         }
@@ -574,7 +574,8 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
           qq[i] = r1;
           qq[i + half] = r2;
         } else {
-          const size_t idx = kv_offset(p, I.layer, b, pos / D.PL, hh) + (size_t)(pos % D.PL) * D.d + i;
+          const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
+                                 (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
           uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
           cache[idx] = f2bf(r1);
           cache[idx + half] = f2bf(r2);
@@ -692,6 +693,20 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     if (s >= se) continue;  // uniform: this slice is not needed at this context length
     const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
     const int np_ = pe - pb;
+    // the warp owning this step's position (if this slice holds it) fetches its
+    // freshly written K/V row now, overlapping the q load
+    const int rcur_all = pos - (npg - 1) * PL;  // row of pos within the last page
+    const bool own_cur = pe == npg && rcur_all / RPW == cw;
+    uint32_t kcur[DH / 64], vcur[DH / 64];
+    if (own_cur) {
+      const size_t base = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + g) *
+                              (size_t)(PL * DH) + (size_t)rcur_all * DH;
+#pragma unroll
+      for (int e = 0; e < DH / 64; ++e) {
+        kcur[e] = __ldcg(reinterpret_cast<const unsigned int*>(p.kcache + base) + lane * (DH / 64) + e);
+        vcur[e] = __ldcg(reinterpret_cast<const unsigned int*>(p.vcache + base) + lane * (DH / 64) + e);
+      }
+    }
     for (int e = ct; e < REP * DC; e += 256) {
       const int h = e / DC, c = e % DC;
       const float* src = p.q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
@@ -728,17 +743,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
       const int r0 = cw * RPW;
       const bool patch = rcur >= r0 && rcur < r0 + RPW;
       if (patch) {  // this step's K/V, written by the QKV instruction, replace the stale copy
-        const size_t base = kv_offset(p, I.layer, b, pb + j, g) + (size_t)rcur * DH;
-        if constexpr (DH == 64) {
-          reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane] =
-              __ldcg(reinterpret_cast<const unsigned int*>(p.kcache + base) + lane);
-          reinterpret_cast<uint32_t*>(vpg + rcur * DH * 2)[lane] =
-              __ldcg(reinterpret_cast<const unsigned int*>(p.vcache + base) + lane);
-        } else {
-          reinterpret_cast<uint2*>(pg + rcur * DH * 2)[lane] =
-              __ldcg(reinterpret_cast<const uint2*>(p.kcache + base) + lane);
-          reinterpret_cast<uint2*>(vpg + rcur * DH * 2)[lane] =
-              __ldcg(reinterpret_cast<const uint2*>(p.vcache + base) + lane);
+#pragma unroll
+        for (int e = 0; e < DH / 64; ++e) {
+          reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane * (DH / 64) + e] = kcur[e];
+          reinterpret_cast<uint32_t*>(vpg + rcur * DH * 2)[lane * (DH / 64) + e] = vcur[e];
         }
         __syncwarp();
       }
@@ -936,6 +944,15 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   const int ct = threadIdx.x - 32;
   const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
   uint32_t page_base = 0;
+  // per-step constants: RoPE (cos, sin) at each lane's position, and the KV page
+  // that position lives in
+  const int half = D.d / 2;
+  for (int e = ct; e < p.nb * half; e += 256) {
+    const int b = e / half, i = e % half;
+    misc->rope_cs[b][i] = p.rope[(size_t)p.pos[b] * half + i];
+  }
+  if (ct < p.nb) misc->cur_phys[ct] = p.page_table[p.slot[ct] * D.pages_per_seq + p.pos[ct] / D.PL];
+  cbar();
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1; ++ii) {
