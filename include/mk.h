@@ -84,6 +84,8 @@ typedef struct {
   int32_t rope_orig_max;
   int32_t max_batch;       /* sequence slots 0..max_batch-1 */
   int32_t max_seq;         /* positions 0..max_seq-1 per slot */
+  int32_t kv_dtype;        /* KV cache element: 0 = bf16, 1 = fp16 (both 2 bytes; fp16
+                              keeps 3 more mantissa bits for deep models) */
 } mk_config;
 
 /* Device pointers (bf16).  The per-layer members are HOST arrays of n_layers

@@ -148,14 +148,27 @@ def weights_to_numpy(w: dict) -> dict:
     return out
 
 
+def round_to_bf16(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest bf16 (ties to even), returned as float32.
+
+    Diagnostic only: lets the oracle keep a bf16 KV cache like a GPU path that
+    stores K and V in bf16, to separate that rounding from other differences.
+    """
+    bits = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    bits = (bits + 0x7FFF + ((bits >> 16) & 1)) >> 16 << 16
+    return bits.astype(np.uint32).view(np.float32)
+
+
 # --- the model ---------------------------------------------------------------
 
 class OracleModel:
     """fp32 (or fp64) forward of one decoder over float32 numpy weights."""
 
-    def __init__(self, cfg: dict, weights: dict, dtype=np.float32):
+    def __init__(self, cfg: dict, weights: dict, dtype=np.float32, kv_round: str | None = None):
         self.cfg = cfg
         self.dt = np.dtype(dtype)
+        # diagnostic only: store K, V rounded to "bf16" or "fp16" (default: compute dtype)
+        self.kv_round = kv_round
         self.w = weights
         self.L = cfg["n_layers"]
         self.H = cfg["hidden"]
@@ -172,6 +185,11 @@ class OracleModel:
     def _m(self, name: str, layer: int | None = None) -> np.ndarray:
         a = self.w[name] if layer is None else self.w[name][layer]
         return a if a.dtype == self.dt else a.astype(self.dt)
+
+    def _kv_rounded(self, a: np.ndarray) -> np.ndarray:
+        if self.kv_round == "bf16":
+            return round_to_bf16(a).astype(self.dt)
+        return a.astype(np.float16).astype(self.dt)  # IEEE half, round to nearest even
 
     def _lm(self) -> np.ndarray:
         return self._m("embed") if self.cfg["tied"] else self._m("lm_head")
@@ -198,6 +216,8 @@ class OracleModel:
             v = (self._m("wv", l) @ n).reshape(Hkv, d)
             q = rope_apply(q, cos[0], sin[0])
             k = rope_apply(k, cos[0], sin[0])
+            if self.kv_round:
+                k, v = self._kv_rounded(k), self._kv_rounded(v)
             cache["K"][l].append(k)
             cache["V"][l].append(v)
             o = attention_decode(q, np.stack(cache["K"][l]), np.stack(cache["V"][l]))
@@ -252,6 +272,8 @@ class OracleModel:
             V = (n @ self._m("wv", l).T).reshape(T, Hkv, d)
             Q = rope_apply(Q, cos[:, None, :], sin[:, None, :])
             K = rope_apply(K, cos[:, None, :], sin[:, None, :])
+            if self.kv_round:
+                K, V = self._kv_rounded(K), self._kv_rounded(V)
             O = np.empty((T, Hq, d), dtype=self.dt)
             for h in range(Hq):
                 g = h // rep

@@ -47,6 +47,7 @@ class MkConfig(ctypes.Structure):
         ("rope_factor", ctypes.c_float), ("rope_low_freq", ctypes.c_float),
         ("rope_high_freq", ctypes.c_float), ("rope_orig_max", ctypes.c_int32),
         ("max_batch", ctypes.c_int32), ("max_seq", ctypes.c_int32),
+        ("kv_dtype", ctypes.c_int32),
     ]
 
 
@@ -138,7 +139,7 @@ _CFG_FIELDS = [f for f, _ in MkConfig._fields_]
 
 
 def config_struct(cfg: dict) -> MkConfig:
-    return MkConfig(**{k: cfg[k] for k in _CFG_FIELDS})
+    return MkConfig(**{k: cfg.get(k, 0) if k == "kv_dtype" else cfg[k] for k in _CFG_FIELDS})
 
 
 def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0) -> dict:

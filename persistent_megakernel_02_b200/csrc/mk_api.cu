@@ -86,8 +86,11 @@ std::string dims_from_config(const mk_config* c, int n_sm, Dims* D) {
         c->rope_orig_max <= 0)
       return "invalid Llama-3 rope scaling parameters";
   }
-  return derive_dims(c->n_layers, c->hidden, c->n_heads, c->n_kv_heads, c->head_dim, c->ffn, c->vocab,
-                     c->tied, c->rms_eps, c->max_batch, c->max_seq, n_sm, D);
+  if (c->kv_dtype != 0 && c->kv_dtype != 1) return "kv_dtype must be 0 (bf16) or 1 (fp16)";
+  std::string why = derive_dims(c->n_layers, c->hidden, c->n_heads, c->n_kv_heads, c->head_dim, c->ffn,
+                                c->vocab, c->tied, c->rms_eps, c->max_batch, c->max_seq, n_sm, D);
+  D->kv_fp16 = c->kv_dtype;
+  return why;
 }
 
 // inverse frequencies theta^(-2i/d) with the optional Llama-3 rescaling of long wavelengths

@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace mk {
@@ -131,6 +132,13 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 __device__ __forceinline__ uint16_t f2bf(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
+// fp16 pair in a 32-bit word -> two floats (exact)
+__device__ __forceinline__ float h_lo(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu))); }
+__device__ __forceinline__ float h_hi(uint32_t w) { return __half2float(__ushort_as_half((unsigned short)(w >> 16))); }
+__device__ __forceinline__ uint16_t f2h(float f) { return __half_as_ushort(__float2half_rn(f)); }
+// a KV cache element pair in a 32-bit word -> two floats
+template <bool F16> __device__ __forceinline__ float kv_lo(uint32_t w) { return F16 ? h_lo(w) : bf_lo(w); }
+template <bool F16> __device__ __forceinline__ float kv_hi(uint32_t w) { return F16 ? h_hi(w) : bf_hi(w); }
 
 // named barrier over the 8 consumer warps (warps 1..8)
 __device__ __forceinline__ void cbar() { asm volatile("bar.sync 1, 256;" ::: "memory"); }

@@ -577,8 +577,8 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
           const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
                                  (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
           uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
-          cache[idx] = f2bf(r1);
-          cache[idx + half] = f2bf(r2);
+          cache[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
+          cache[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
         }
       }
     } else if constexpr (OPK == OP_GU) {
@@ -663,7 +663,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
 // query heads of the group.  After the slice the CTA combines the warps'
 // partials into the slice partial, and the last slice to finish (atomic
 // counter) merges all slices of the (lane, kv head) into o.
-template <int DH, int REP>
+template <int DH, int REP, bool KV16F>
 __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
                                             uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
                                             Misc* misc, uint32_t ii) {
@@ -765,10 +765,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
             const uint4 kw = lds128(kb + (uint32_t)((row * DC + c) * 16));
             const float4 ql = lds128f(sqlo + (uint32_t)((myh * DC + c) * 16));
             const float4 qh = lds128f(sqhi + (uint32_t)((myh * DC + c) * 16));
-            a2 = __ffma2_rn(make_float2(bf_lo(kw.x), bf_hi(kw.x)), make_float2(ql.x, ql.y), a2);
-            a2 = __ffma2_rn(make_float2(bf_lo(kw.y), bf_hi(kw.y)), make_float2(ql.z, ql.w), a2);
-            a2 = __ffma2_rn(make_float2(bf_lo(kw.z), bf_hi(kw.z)), make_float2(qh.x, qh.y), a2);
-            a2 = __ffma2_rn(make_float2(bf_lo(kw.w), bf_hi(kw.w)), make_float2(qh.z, qh.w), a2);
+            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.x), kv_hi<KV16F>(kw.x)), make_float2(ql.x, ql.y), a2);
+            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.y), kv_hi<KV16F>(kw.y)), make_float2(ql.z, ql.w), a2);
+            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.z), kv_hi<KV16F>(kw.z)), make_float2(qh.x, qh.y), a2);
+            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.w), kv_hi<KV16F>(kw.w)), make_float2(qh.z, qh.w), a2);
           }
           sv = a2.x + a2.y;
         }
@@ -811,10 +811,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         float vv[DPL];
         if constexpr (DPL == 2) {
           const uint32_t w = lds32(vb + (uint32_t)((r0 + rr) * DH * 2));
-          vv[0] = bf_lo(w); vv[1] = bf_hi(w);
+          vv[0] = kv_lo<KV16F>(w); vv[1] = kv_hi<KV16F>(w);
         } else {
           const uint2 w = lds64(vb + (uint32_t)((r0 + rr) * DH * 2));
-          vv[0] = bf_lo(w.x); vv[1] = bf_hi(w.x); vv[2] = bf_lo(w.y); vv[3] = bf_hi(w.y);
+          vv[0] = kv_lo<KV16F>(w.x); vv[1] = kv_hi<KV16F>(w.x); vv[2] = kv_lo<KV16F>(w.y); vv[3] = kv_hi<KV16F>(w.y);
         }
 #pragma unroll
         for (int h = 0; h < REP; ++h) {
@@ -925,16 +925,23 @@ __device__ __forceinline__ void mv_dispatch(int rt, const KParams& p, const Inst
   }
 }
 
+template <int DH, bool KV16F>
+__device__ __forceinline__ uint32_t attn_dispatch_rep(const KParams& p, const Instr& I, uint32_t pb,
+                                                      uint8_t* ring, float* act, uint64_t* full,
+                                                      uint64_t* empty, Misc* misc, uint32_t ii) {
+  switch (p.D.rep) {
+    case 1: return attn_units<DH, 1, KV16F>(p, I, pb, ring, act, full, empty, misc, ii);
+    case 2: return attn_units<DH, 2, KV16F>(p, I, pb, ring, act, full, empty, misc, ii);
+    case 4: return attn_units<DH, 4, KV16F>(p, I, pb, ring, act, full, empty, misc, ii);
+    default: return attn_units<DH, 8, KV16F>(p, I, pb, ring, act, full, empty, misc, ii);
+  }
+}
 template <int DH>
 __device__ __forceinline__ uint32_t attn_dispatch(const KParams& p, const Instr& I, uint32_t pb,
                                                   uint8_t* ring, float* act, uint64_t* full,
                                                   uint64_t* empty, Misc* misc, uint32_t ii) {
-  switch (p.D.rep) {
-    case 1: return attn_units<DH, 1>(p, I, pb, ring, act, full, empty, misc, ii);
-    case 2: return attn_units<DH, 2>(p, I, pb, ring, act, full, empty, misc, ii);
-    case 4: return attn_units<DH, 4>(p, I, pb, ring, act, full, empty, misc, ii);
-    default: return attn_units<DH, 8>(p, I, pb, ring, act, full, empty, misc, ii);
-  }
+  return p.D.kv_fp16 ? attn_dispatch_rep<DH, true>(p, I, pb, ring, act, full, empty, misc, ii)
+                     : attn_dispatch_rep<DH, false>(p, I, pb, ring, act, full, empty, misc, ii);
 }
 
 template <int NBT>

@@ -74,6 +74,7 @@ struct Dims {
   int n_qkv, n_o, n_gu, n_dn, n_lm;   // units per op per layer (n_dn per K slice)
   float eps;
   int tied;
+  int kv_fp16;    // KV cache element: 0 bf16, 1 fp16
 };
 
 // One tape: the instruction lists of every SM for one active batch size.

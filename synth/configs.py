@@ -19,13 +19,17 @@ _NO_SCALING = dict(rope_scaling=0, rope_factor=1.0, rope_low_freq=1.0,
                    rope_high_freq=1.0, rope_orig_max=0)
 
 TINY = dict(n_layers=2, hidden=256, n_heads=4, n_kv_heads=2, head_dim=64, ffn=1024,
-            vocab=4096, tied=1, rms_eps=1e-5, rope_theta=500000.0, **_NO_SCALING)
+            vocab=4096, tied=1, rms_eps=1e-5, rope_theta=500000.0, kv_dtype=0, **_NO_SCALING)
 
 LLAMA_1B = dict(n_layers=16, hidden=2048, n_heads=32, n_kv_heads=8, head_dim=64, ffn=8192,
-                vocab=128256, tied=1, rms_eps=1e-5, rope_theta=500000.0, **_LLAMA3_SCALING)
+                vocab=128256, tied=1, rms_eps=1e-5, rope_theta=500000.0, kv_dtype=0,
+                **_LLAMA3_SCALING)
 
+# The 8B workload states no KV-cache type; bf16 K/V rounding alone moves its
+# 32-layer logits past the parity tolerance against the fp32 oracle, so its
+# cache is fp16 (same bytes, 3 more mantissa bits).  kv_dtype: 0 bf16, 1 fp16.
 LLAMA_8B = dict(n_layers=32, hidden=4096, n_heads=32, n_kv_heads=8, head_dim=128, ffn=14336,
-                vocab=128256, tied=0, rms_eps=1e-5, rope_theta=500000.0, **_NO_SCALING)
+                vocab=128256, tied=0, rms_eps=1e-5, rope_theta=500000.0, kv_dtype=1, **_NO_SCALING)
 
 
 def _wl(name, model, batch, prompt_lens, decode_steps, desc):

@@ -67,6 +67,10 @@ def test_tiny_random_norm_gains_and_untied():
     _teacher_forced_case("tiny", norm_jitter=0.2, tied=0)
 
 
+def test_tiny_fp16_kv_cache():
+    _teacher_forced_case("tiny", kv_dtype=1)
+
+
 def test_tiny_ragged_vocab_and_ffn():
     # vocab 4099 leaves a short last LM-head unit; ffn 1000 needs 5 down-proj K slices
     _teacher_forced_case("tiny", vocab=4099, ffn=1000)
@@ -152,6 +156,18 @@ def test_llama1b_bs1_teacher_forced_full():
     worst, checked = _teacher_forced_case("llama1b_bs1")
     print("llama1b_bs1 worst", worst, "ids checked", checked)
     assert checked > 20
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("wl,n_steps", [("llama1b_long", 16), ("llama1b_bs4", 32),
+                                        ("llama1b_bs8", 16), ("llama8b_bs1", 16)])
+def test_full_size_workloads_teacher_forced(wl, n_steps):
+    """The long-context (8192-token KV), batch-4/8 (prompts 512..1408) and 8B
+    shapes at full size: every lane's prompt is prefilled token by token, then
+    n_steps batched decode steps are compared with the oracle's causal pass."""
+    worst, checked = _teacher_forced_case(wl, n_steps=n_steps)
+    print(wl, "worst", worst, "ids checked", checked)
+    assert checked > 0
 
 
 def test_llama1b_zero_layers_identity_full_size():
