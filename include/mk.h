@@ -205,6 +205,40 @@ typedef struct {
 mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
                         mk_plan_report* rep);
 
+/* ---- greedy head without allocation ----
+ *
+ * No counterpart in the pages: a convenience entry point of this library.
+ *
+ * The last stage of a decode step as a stand-alone call on the current CUDA
+ * device: for lanes b < nb,
+ *   logits[b][v] = lm_head[v] . (x_b / sqrt(mean(x_b^2) + rms_eps) * final_norm)
+ *   ids[b]       = argmax_v logits[b][v], lowest index on ties,
+ * from a caller-provided hidden state.  It is for callers that run the decoder
+ * layers themselves and cannot allocate device memory on their call path: code
+ * inside a framework whose caching allocator already owns the GPU's memory, where
+ * a raw cudaMalloc can fail or make the whole device wait, and latency-critical
+ * loops that allow no allocation once started.  It calls no cudaMalloc/cudaFree.
+ *
+ * Its only working memory (the per-block argmax partials and a completion
+ * counter) is one static device array of MK_NOALLOC_SCRATCH_BYTES, held on every
+ * GPU that loads the library until the process exits.  Every call shares it and
+ * it keeps the last call's contents; the kernel returns its counter to zero
+ * itself.  Calls that overlap on the GPU (e.g. on two streams) race on it: order
+ * them on one stream.  The first call on a device looks up the array's device
+ * address with that device current; make that first call before any stream
+ * capture.
+ *
+ *   hidden_dev   device float[nb][hidden]
+ *   final_norm   device bf16[hidden];   lm_head  device bf16[vocab][hidden] (16-byte aligned)
+ *   logits_dev   device float[nb][vocab] or NULL;   ids_dev  device int32[nb]
+ * Limits: 1 <= nb <= 8 and nb * hidden <= 16384 -- larger requests return
+ * MK_ERR_UNSUPPORTED without launching; hidden must be a multiple of 8.
+ * Asynchronous on `stream`. */
+#define MK_NOALLOC_SCRATCH_BYTES 65536
+mk_status mk_greedy_head_noalloc(const float* hidden_dev, int32_t nb, int32_t hidden,
+                                 const void* final_norm, const void* lm_head, int32_t vocab,
+                                 float rms_eps, float* logits_dev, int32_t* ids_dev, void* stream);
+
 /* Library version string (static storage). */
 const char* mk_version(void);
 

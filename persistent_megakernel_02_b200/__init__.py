@@ -17,7 +17,8 @@ import os
 
 from .build import LIB
 
-__all__ = ["Megakernel", "MkError", "plan_check", "version", "lib", "STATUS"]
+__all__ = ["Megakernel", "MkError", "plan_check", "version", "lib", "STATUS",
+           "greedy_head_noalloc"]
 
 STATUS = {
     0: "MK_OK",
@@ -104,6 +105,10 @@ _SIGS = {
     "mk_profile_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.POINTER(ctypes.c_int32),
                                        ctypes.POINTER(ctypes.c_int32)]),
+    "mk_greedy_head_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                              ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                              ctypes.c_void_p]),
     "mk_version": (ctypes.c_char_p, []),
 }
 
@@ -148,6 +153,23 @@ def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0) -> dict:
     c = config_struct(cfg)
     _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, ctypes.byref(rep)), "mk_plan_check")
     return {f: getattr(rep, f) for f, _ in MkPlanReport._fields_}
+
+
+def greedy_head_noalloc(hidden, final_norm, lm_head, rms_eps, ids, logits=None, stream=None):
+    """Final RMSNorm + LM head + greedy argmax through ``mk_greedy_head_noalloc``.
+
+    For callers that cannot allocate device memory on their call path: the call
+    uses only a static scratch array inside the library.  ``hidden`` is a CUDA
+    float32 [nb, H] tensor, ``final_norm`` bf16 [H], ``lm_head`` bf16 [V, H],
+    ``ids`` int32 [nb], ``logits`` float32 [nb, V] or None.  Asynchronous; raises
+    MkError on a rejected request.
+    """
+    nb, H = hidden.shape
+    _check(lib().mk_greedy_head_noalloc(hidden.data_ptr(), nb, H, final_norm.data_ptr(),
+                                        lm_head.data_ptr(), lm_head.shape[0], rms_eps,
+                                        None if logits is None else logits.data_ptr(),
+                                        ids.data_ptr(), _stream_handle(stream)),
+           "mk_greedy_head_noalloc")
 
 
 def _i32_array(values):
