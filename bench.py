@@ -104,6 +104,18 @@ def _dist():
     return ws, rank, local
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The largest value any rank reports (device time of the slowest replica).
+    ``dist`` is torch.distributed with an initialised group, or None for one rank."""
+    if dist is None:
+        return float(value)
+    import torch
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def oracle_sample(cfg, prompt, n_steps, w_host=None, time_budget_s=25.0):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload:
     the prompt is run untimed, then up to n_steps greedy decode steps are timed
@@ -237,11 +249,8 @@ def main():
         ev1.record(stream)
         torch.cuda.synchronize()
     mk.sync(stream)
-    ms = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
     if pg:
-        t_ = torch.tensor([ms], device="cuda")
-        pg.all_reduce(t_, op=pg.ReduceOp.MAX)
-        ms = float(t_.item())
         pg.barrier()
     us_step = 1000.0 * ms / args.steps
     # algorithmic bytes of the timed steps (weights + KV read/write at each step's positions)
@@ -258,10 +267,7 @@ def main():
         mk_ids, _ = mk.decode_step_host(mk_ids, [p + base + t for p in pos0])
     e2e_us = 1e6 * (time.perf_counter() - t0) / e2e_steps
     mk.close()
-    if pg:
-        t_ = torch.tensor([e2e_us], device="cuda")
-        pg.all_reduce(t_, op=pg.ReduceOp.MAX)
-        e2e_us = float(t_.item())
+    e2e_us = max_over_ranks(e2e_us, pg, "cuda")
 
     peak, peak_kind = _peaks()
     line = {

@@ -1,0 +1,90 @@
+"""The C-ABI library on the host (no GPU): exports, tape lowering and simulation,
+fault detection by the simulator, and host-side argument checks."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import persistent_megakernel_02_b200 as mk
+from persistent_megakernel_02_b200 import build
+from synth import configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "mk.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:mk_status|const char\*)\s+(mk_\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert {"mk_create", "mk_decode_step", "mk_prefill", "mk_destroy"} <= set(names)
+    lib = ctypes.CDLL(build.LIB)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(mk._SIGS), "binding misses a declared entry point"
+
+
+def test_version_string():
+    assert "megakernel" in mk.version()
+
+
+@pytest.mark.parametrize("wl", list(configs.WORKLOADS))
+@pytest.mark.parametrize("n_sm", [148, 132, 37])
+def test_tapes_are_deadlock_free_and_cover_every_output(wl, n_sm):
+    cfg = configs.model_config(wl)
+    for nb in sorted({1, cfg["max_batch"]}):
+        r = mk.plan_check(cfg, n_sm, nb)
+        assert r["deadlock_free"] and r["coverage_ok"] and r["targets_ok"], (wl, n_sm, nb, r)
+        # bytes per SM balanced to within one attention slice + one page
+        assert r["bytes_max_sm"] - r["bytes_min_sm"] <= 2 * 16384 * (1 + 130 // r["attn_slices"])
+        assert r["ring_pages"] >= 8
+
+
+def test_ragged_shapes_lower_cleanly():
+    cfg = configs.model_config("tiny", vocab=4099, ffn=1000, max_batch=3, max_seq=77)
+    for nb in (1, 2, 3):
+        r = mk.plan_check(cfg, 148, nb)
+        assert r["deadlock_free"] and r["coverage_ok"] and r["targets_ok"]
+
+
+@pytest.mark.parametrize("fault", [1, 2])
+def test_simulator_reports_planted_faults(fault):
+    """1: a dropped signal, 2: a wait target one too high -- both leave SMs stuck."""
+    r = mk.plan_check(configs.model_config("tiny"), 148, 1, fault=fault)
+    assert not r["deadlock_free"]
+    assert not r["targets_ok"]
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=96), dict(hidden=4104), dict(n_heads=12, n_kv_heads=4),
+                                 dict(max_batch=9), dict(ffn=1001), dict(n_kv_heads=3),
+                                 dict(kv_dtype=2), dict(max_batch=8, hidden=4096)])
+def test_unsupported_configs_are_rejected(bad):
+    cfg = configs.model_config("tiny", **bad)
+    with pytest.raises(mk.MkError, match="UNSUPPORTED"):
+        mk.plan_check(cfg, 148, 1)
+
+
+def test_create_rejects_missing_weights_before_touching_the_gpu():
+    c = mk.config_struct(configs.model_config("tiny"))
+    w = mk.MkWeights()  # all NULL
+    h = ctypes.c_void_p()
+    st = mk.lib().mk_create(ctypes.byref(c), ctypes.byref(w), None, ctypes.byref(h))
+    assert mk.STATUS[st] == "MK_ERR_INVALID_ARG"
+
+
+def test_noalloc_head_rejects_bad_arguments_on_the_host():
+    f = mk.lib().mk_greedy_head_noalloc
+    ids = ctypes.c_void_p(16)
+    assert mk.STATUS[f(None, 1, 64, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_INVALID_ARG"
+    assert mk.STATUS[f(ids, 0, 64, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_INVALID_ARG"
+    assert mk.STATUS[f(ids, 9, 64, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_UNSUPPORTED"
+    assert mk.STATUS[f(ids, 8, 4096, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_UNSUPPORTED"
