@@ -97,6 +97,36 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+KERNEL_SOURCES = ["mk_kernel.cuh", "mk_device.cuh", "mk_plan.h", "mk_sched.cpp", "mk_api.cu"]
+
+
+def kernel_src_hash() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "persistent_megakernel_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on this
+    workload with the current kernel sources; otherwise None."""
+    p = os.path.join(ROOT, "profiles", f"mk_decode_kernel_{workload}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    with open(p) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+    if kv.get("kernel_src_sha256_16") != kernel_src_hash():
+        return None
+    return float(kv["dram_bytes_per_launch"])
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -281,7 +311,8 @@ def main():
         "bytes_per_step": int(bytes_step),
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
-                     "traffic": args.traffic_bytes,
+                     "traffic": args.traffic_bytes if args.traffic_bytes is not None
+                     else recorded_traffic(args.workload),
                      "kernel": "mk::mk_decode_kernel<1>" if nb == 1 else f"mk::mk_decode_kernel<{nb}>"},
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": 4 * nb,
                 "d2h_bytes_per_step": 4 * nb},

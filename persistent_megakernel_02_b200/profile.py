@@ -9,6 +9,10 @@ each (layer, op) finished -- the critical path through the layer chain.
 
 from __future__ import annotations
 
+import argparse
+import json
+import sys
+
 import numpy as np
 
 OPS = {1: "qkv", 2: "attn", 3: "o", 4: "gu", 5: "down", 6: "lm"}
@@ -71,3 +75,45 @@ def summarize(rec: np.ndarray) -> dict:
         "phase_end_us": sorted(((ph["last_sig"] - t0) / 1e3, layer, op)
                                for (layer, op), ph in phases.items()),
     }
+
+
+def main(argv=None):
+    """Profile one steady-state decode step of a workload and print its breakdown.
+
+    python -m persistent_megakernel_02_b200.profile [--workload llama1b_bs1]
+    """
+    import os
+
+    import torch
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import synth
+    from synth import configs
+
+    from . import Megakernel
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", default="llama1b_bs1")
+    ap.add_argument("--ring-pages", type=int, default=0)
+    args = ap.parse_args(argv)
+    wl = configs.WORKLOADS[args.workload]
+    nb, P = wl["batch"], max(wl["prompt_lens"])
+    cfg = configs.model_config(args.workload, max_seq=P + 8)
+    w = synth.make_weights(cfg, device="cuda")
+    mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages)
+    prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
+    ids = torch.tensor([mk.prefill(b, prompts[b]) for b in range(nb)], dtype=torch.int32, device="cuda")
+    pos = [len(p) for p in prompts]
+    for t in range(2):
+        mk.decode_step(ids, [p + t for p in pos], ids)
+    mk.sync()
+    mk.profile_records()  # resets the accumulators
+    mk.decode_step(ids, [p + 2 for p in pos], ids)
+    s = summarize(mk.profile_records())
+    mk.close()
+    out = {k: v for k, v in s.items() if k != "phase_end_us"}
+    print(json.dumps(out, indent=1))
+
+
+if __name__ == "__main__":
+    main()
