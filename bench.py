@@ -232,7 +232,7 @@ def main():
     nb = wl["batch"]
     P = max(wl["prompt_lens"])
     e2e_steps = min(args.steps, 32)
-    max_seq = P + args.warmup + args.steps + e2e_steps + 8
+    max_seq = P + args.warmup + args.steps + 8 + e2e_steps + 8
     cfg = configs.model_config(args.workload, max_seq=max_seq)
 
     if args.impl == "reference":
@@ -262,11 +262,14 @@ def main():
     ids = torch.tensor(firsts, dtype=torch.int32, device="cuda")
     pos0 = [len(p) for p in prompts]
 
-    def step(t):
-        mk.decode_step(ids, [p + t for p in pos0], ids, stream=stream)
+    out = torch.empty((max(args.steps, args.warmup), nb), dtype=torch.int32, device="cuda")
 
-    for t in range(args.warmup):
-        step(t)
+    def steps(t0, n):
+        """n chained decode steps in one launch, starting at step t0 (ids fed back)."""
+        mk.decode_steps(ids, [p + t0 for p in pos0], n, out, stream=stream)
+        ids.copy_(out[n - 1])
+
+    steps(0, args.warmup)
     mk.sync(stream)
     if pg:
         pg.barrier()
@@ -274,8 +277,7 @@ def main():
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         ev0.record(stream)
-        for t in range(args.warmup, args.warmup + args.steps):
-            step(t)
+        steps(args.warmup, args.steps)
         ev1.record(stream)
         torch.cuda.synchronize()
     mk.sync(stream)
@@ -289,8 +291,19 @@ def main():
     bytes_step = total_bytes / args.steps
     gbs = total_bytes / (ms * 1e-3) / 1e9
 
+    # the same steps launched one at a time (for comparison; not the headline)
+    base1 = args.warmup + args.steps
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for t in range(8):
+        mk.decode_step(ids, [p + base1 + t for p in pos0], ids, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us_single = 1000.0 * e0.elapsed_time(e1) / 8
+
     # end to end through the C ABI with host buffers (H2D tokens, D2H ids per step)
-    base = args.warmup + args.steps
+    base = args.warmup + args.steps + 8
     mk_ids = list(firsts)
     t0 = time.perf_counter()
     for t in range(e2e_steps):
@@ -316,7 +329,8 @@ def main():
                      "kernel": "mk::mk_decode_kernel<1>" if nb == 1 else f"mk::mk_decode_kernel<{nb}>"},
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": 4 * nb,
                 "d2h_bytes_per_step": 4 * nb},
-        "gpu_launches": args.steps,
+        "gpu_launches": 1,
+        "us_per_step_one_launch_per_step": round(us_single, 2),
         "clocks": clk.summary(),
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:

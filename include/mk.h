@@ -139,6 +139,17 @@ mk_status mk_decode_step(mk_handle h, int32_t nb, const int32_t* tokens_dev,
                          const int32_t* positions, float* logits_dev, int32_t* ids_dev,
                          void* stream);
 
+/* n_steps greedy decode steps in ONE launch, lanes b = 0..nb-1 in slots b.
+ * Step 0 reads tokens_dev[b] at positions[b]; step t > 0 reads the id step t-1
+ * produced, at positions[b] + t.  ids_dev (device int32[n_steps][nb]) receives
+ * every step's ids; logits_dev is NULL or device float[n_steps][nb][vocab].
+ * Requires positions[b] + n_steps <= max_seq.  Asynchronous.  The kernel keeps
+ * streaming weights across step boundaries, so this is faster per step than
+ * n_steps calls of mk_decode_step. */
+mk_status mk_decode_steps(mk_handle h, int32_t nb, int32_t n_steps, const int32_t* tokens_dev,
+                          const int32_t* positions, float* logits_dev, int32_t* ids_dev,
+                          void* stream);
+
 /* The same step with HOST buffers: copies tokens in, runs the step, copies ids
  * (and logits when logits_host != NULL, float[nb, vocab]) back, and waits for
  * the stream.  Returns the step's device status. */
@@ -147,7 +158,7 @@ mk_status mk_decode_step_host(mk_handle h, int32_t nb, const int32_t* tokens_hos
                               int32_t* ids_host, void* stream);
 
 /* Prefill sequence slot `seq` with n HOST tokens at positions start_pos ..
- * start_pos+n-1, one decode step per token.  logits_last_dev (device
+ * start_pos+n-1: one launch that runs one decode step per token.  logits_last_dev (device
  * float[vocab], nullable) and id_last_host (host int32*, nullable) receive the
  * last position's logits and greedy id; when id_last_host is non-NULL the call
  * waits for the stream.  The prompt is copied before the call returns. */

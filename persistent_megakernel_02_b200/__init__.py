@@ -89,6 +89,9 @@ _SIGS = {
     "mk_decode_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
                                       ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p,
                                       ctypes.c_void_p, ctypes.c_void_p]),
+    "mk_decode_steps": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p,
+                                       ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_void_p]),
     "mk_decode_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int32,
                                            ctypes.POINTER(ctypes.c_int32),
                                            ctypes.POINTER(ctypes.c_int32), ctypes.c_void_p,
@@ -223,6 +226,14 @@ class Megakernel:
         _check(lib().mk_decode_step(self._h, nb, tokens.data_ptr(), _i32_array(positions),
                                     None if logits is None else logits.data_ptr(), ids.data_ptr(),
                                     _stream_handle(stream)), "mk_decode_step")
+
+    def decode_steps(self, tokens, positions, n_steps, ids, logits=None, stream=None):
+        """n_steps chained greedy steps in one launch; ids int32 [n_steps, nb] (device),
+        logits None or float32 [n_steps, nb, V]."""
+        nb = len(positions)
+        _check(lib().mk_decode_steps(self._h, nb, n_steps, tokens.data_ptr(), _i32_array(positions),
+                                     None if logits is None else logits.data_ptr(), ids.data_ptr(),
+                                     _stream_handle(stream)), "mk_decode_steps")
 
     def decode_step_host(self, tokens, positions, want_logits=False, stream=None):
         """Step over host buffers; returns (ids list, logits numpy [nb, V] or None)."""

@@ -220,8 +220,10 @@ const void* kernel_for(int nbt) {
   }
 }
 
+// One launch of n_steps decode steps (see KParams for the token / ids / logits modes).
 mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, const int* slot,
-                      float* logits, int* ids, cudaStream_t st) {
+                      float* logits, int* ids, cudaStream_t st, int n_steps = 1, int chain = 1,
+                      int ids_stride = 0, int logits_last = 0) {
   const Dims& D = h->D;
   const Tape& t = h->tapes[nb - 1];
   const mk_ctx::DevTape& dt = h->dtapes[nb - 1];
@@ -239,6 +241,10 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.err = h->err;
   p.rope = h->rope;
   p.nb = nb;
+  p.n_steps = n_steps;
+  p.chain = chain;
+  p.ids_stride = ids_stride;
+  p.logits_last = logits_last;
   p.tokens = tokens_dev;
   for (int b = 0; b < kMaxNB; ++b) {
     p.pos[b] = b < nb ? pos[b] : 0;
@@ -389,6 +395,21 @@ extern "C" mk_status mk_decode_step(mk_handle h, int32_t nb, const int32_t* toke
   return launch_step(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream);
 }
 
+extern "C" mk_status mk_decode_steps(mk_handle h, int32_t nb, int32_t n_steps, const int32_t* tokens_dev,
+                                     const int32_t* positions, float* logits_dev, int32_t* ids_dev,
+                                     void* stream) {
+  if (!h || !tokens_dev || !positions || !ids_dev) return MK_ERR_INVALID_ARG;
+  if (nb < 1 || nb > h->D.max_batch || n_steps < 1) return MK_ERR_INVALID_ARG;
+  int slot[kMaxNB];
+  for (int b = 0; b < nb; ++b) {
+    if (positions[b] < 0 || (long long)positions[b] + n_steps > h->D.max_seq) return MK_ERR_INVALID_ARG;
+    slot[b] = b;
+  }
+  cudaSetDevice(h->dev);
+  return launch_step(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream, n_steps,
+                     /*chain=*/1, /*ids_stride=*/nb, /*logits_last=*/0);
+}
+
 extern "C" mk_status mk_sync(mk_handle h, void* stream) {
   if (!h) return MK_ERR_INVALID_ARG;
   cudaSetDevice(h->dev);
@@ -444,11 +465,11 @@ extern "C" mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_
   // pageable source: the copy completes before the call returns
   MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_stage, tokens_host, sizeof(int) * n, cudaMemcpyHostToDevice, st)));
   MK_TRY(from_cuda(cudaStreamSynchronize(st)));
-  for (int i = 0; i < n; ++i) {
-    int pos = start_pos + i, slot = seq;
-    MK_TRY(launch_step(h, 1, h->tok_stage + i, &pos, &slot, i == n - 1 ? logits_last_dev : nullptr,
-                       h->ids_scratch, st));
-  }
+  // one launch runs the whole prompt: step i takes token i at position start_pos + i;
+  // only the last step's logits are kept, every step overwrites the greedy id
+  int pos = start_pos, slot = seq;
+  MK_TRY(launch_step(h, 1, h->tok_stage, &pos, &slot, logits_last_dev, h->ids_scratch, st, n,
+                     /*chain=*/0, /*ids_stride=*/0, /*logits_last=*/1));
   if (id_last_host) {
     MK_TRY(from_cuda(cudaMemcpyAsync(id_last_host, h->ids_scratch, sizeof(int), cudaMemcpyDeviceToHost, st)));
     return mk_sync(h, stream);

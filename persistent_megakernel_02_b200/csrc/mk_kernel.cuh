@@ -76,13 +76,22 @@ struct KParams {
   int n_counters;
   ErrWord* err;
   const float2* rope;  // [max_seq][d/2] (cos, sin)
-  // step
+  // steps: n_steps decode steps run in this launch, lane b of step t at position
+  // pos[b] + t.  Step t's input tokens: tokens + t * nb when tokens are given
+  // for every step (chain == 0), else step 0 reads tokens and step t > 0 reads the
+  // ids step t - 1 wrote.  Step t writes its ids to ids + t * ids_stride and, when
+  // logits is set, its logits to logits + t * nb * V (logits_last: only the last
+  // step, at logits).
   int nb;
-  const int* tokens;  // device [nb]
+  int n_steps;
+  int chain;
+  int ids_stride;
+  int logits_last;
+  const int* tokens;
   int pos[kMaxNB];
   int slot[kMaxNB];
-  float* logits;  // device [nb][V] or null
-  int* ids;       // device [nb]
+  float* logits;
+  int* ids;
   unsigned long long wait_limit_ns;
   long long* prof;   // profile records [n_sm][prof_stride][16] or null
   int prof_stride;
@@ -96,6 +105,8 @@ struct Misc {
   float lmv[kConsumerWarps][kMaxNB];
   int lmi[kConsumerWarps][kMaxNB];
   int tok[kMaxNB];
+  int pos[kMaxNB];       // each lane's position in the current step
+  int step;              // the current step of this launch
   int cur_phys[kMaxNB];  // physical KV page holding each lane's position this step
   float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
   volatile int stop;
@@ -252,6 +263,7 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
   RingPos rp;
   rp.init(0, NP);
   bool ok = true;
+  for (int t = 0; t < p.n_steps && ok; ++t) {
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1 && ok; ++ii) {
@@ -260,10 +272,15 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
     long long acc_wait = 0, acc_pages = 0;
     if (rec) rec[5] = (long long)globaltimer_ns();
     if (I.op == OP_ATTN) {
+      // KV pages of step t hold the positions earlier steps of this launch wrote:
+      // copy them only once those steps' QKV instructions for this layer are done.
+      // (By then this producer has issued every page of the earlier steps, so the
+      // wait cannot hold up the consumers it depends on.)
+      if (t > 0 && !(ok = wait_counter(p, p.ctr + I.dep, I.dep_target * (uint32_t)t, ii))) break;
       for (uint32_t k = 0; k < I.n_units && ok; ++k) {
         int b, g, s;
         attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-        const int pos = p.pos[b], npg = pos / D.PL + 1, se = attn_slices_used(p.S, npg);
+        const int pos = p.pos[b] + t, npg = pos / D.PL + 1, se = attn_slices_used(p.S, npg);
         if (s >= se) continue;
         const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
         const int* pt = p.page_table + p.slot[b] * D.pages_per_seq;
@@ -301,6 +318,7 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
     }
     if (rec) { rec[6] = (long long)globaltimer_ns(); rec[9] += acc_wait; rec[10] += acc_pages; }
     I = In;
+  }
   }
   misc->issued = pidx;
   // every copy issued must land before the CTA exits (also after an abort)
@@ -514,6 +532,12 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
                         ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - p.sm_off[blockIdx.x])) * 16
                         : nullptr;
   long long c_wait = 0, c_pages = 0;
+  // this step's logits (LM head only)
+  float* lg = nullptr;
+  if (OPK == OP_LM && p.logits) {
+    if (!p.logits_last) lg = p.logits + (size_t)misc->step * p.nb * D.V;
+    else if (misc->step == p.n_steps - 1) lg = p.logits;
+  }
 
   RingPos rp;
   rp.init(page_base + cw, NP);
@@ -562,7 +586,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         const int pi = vbase / 2 + m, j = pi / NBT, b = pi % NBT;
         if (!writer || b >= p.nb) continue;
         const float v1 = v[2 * m], v2 = v[2 * m + 1];
-        const int i = i0 + j, pos = p.pos[b];
+        const int i = i0 + j, pos = misc->pos[b];
         float r1 = v1, r2 = v2;
         if (sec < 2) {
           const float2 cs = misc->rope_cs[b][i];
@@ -606,7 +630,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
 #pragma unroll
         for (int bb = 0; bb < NBT; ++bb)
           if (bb == b && lm_better(v[m], r0 + r, bestv[bb], besti[bb])) { bestv[bb] = v[m]; besti[bb] = r0 + r; }
-        if (writer && p.logits) p.logits[(size_t)b * D.V + r0 + r] = v[m];
+        if (writer && lg) lg[(size_t)b * D.V + r0 + r] = v[m];
       }
     }
   }
@@ -640,15 +664,22 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
       misc->last = (old == gridDim.x - 1) && !misc->stop;
     }
     cbar();
-    if (misc->last && ct < p.nb) {
-      float bv = -CUDART_INF_F;
-      int bi = 0x7FFFFFFF;
-      for (int s = 0; s < (int)gridDim.x; ++s) {
-        const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
-        const float val = __int_as_float(e.x);
-        if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
+    if (misc->last) {
+      if (ct < p.nb) {
+        float bv = -CUDART_INF_F;
+        int bi = 0x7FFFFFFF;
+        for (int s = 0; s < (int)gridDim.x; ++s) {
+          const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
+          const float val = __int_as_float(e.x);
+          if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
+        }
+        p.ids[(size_t)misc->step * p.ids_stride + ct] = (bi >= 0 && bi < D.V) ? bi : 0;
       }
-      p.ids[ct] = (bi >= 0 && bi < D.V) ? bi : 0;
+      cbar();
+      if (ct == 0) {
+        p.ctr[ctr_lm(D)] = 0u;                  // the next step's arrivals count from zero
+        red_release_add(p.ctr + ctr_step(D), 1u);  // this step's ids are written
+      }
     }
   }
 }
@@ -689,7 +720,7 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
   for (uint32_t k = 0; k < I.n_units; ++k) {
     int b, g, s;
     attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-    const int pos = p.pos[b], npg = pos / PL + 1, se = attn_slices_used(p.S, npg);
+    const int pos = misc->pos[b], npg = pos / PL + 1, se = attn_slices_used(p.S, npg);
     if (s >= se) continue;  // uniform: this slice is not needed at this context length
     const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
     const int np_ = pe - pb;
@@ -903,7 +934,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
       }
       cbar();
-      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      if (ct == 0) {
+        p.ctr[ctr_part(D, I.layer, b, g)] = 0u;  // the next step's slices count from zero
+        red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      }
     }
     used += (uint32_t)np_;
     cbar();
@@ -951,14 +985,21 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   const int ct = threadIdx.x - 32;
   const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
   uint32_t page_base = 0;
-  // per-step constants: RoPE (cos, sin) at each lane's position, and the KV page
-  // that position lives in
   const int half = D.d / 2;
+  for (int t = 0; t < p.n_steps; ++t) {
+  // per-step constants: positions, RoPE (cos, sin) at each lane's position, and the
+  // KV page that position lives in
+  if (ct == 0) misc->step = t;
+  if (ct < p.nb) {
+    misc->pos[ct] = p.pos[ct] + t;
+    misc->cur_phys[ct] = p.page_table[p.slot[ct] * D.pages_per_seq + (p.pos[ct] + t) / D.PL];
+  }
   for (int e = ct; e < p.nb * half; e += 256) {
     const int b = e / half, i = e % half;
-    misc->rope_cs[b][i] = p.rope[(size_t)p.pos[b] * half + i];
+    misc->rope_cs[b][i] = p.rope[(size_t)(p.pos[b] + t) * half + i];
   }
-  if (ct < p.nb) misc->cur_phys[ct] = p.page_table[p.slot[ct] * D.pages_per_seq + p.pos[ct] / D.PL];
+  const int* step_tokens = (p.chain && t > 0) ? p.ids + (size_t)(t - 1) * p.ids_stride
+                                              : p.tokens + (size_t)(p.chain ? 0 : t) * p.nb;
   cbar();
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
@@ -969,8 +1010,15 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
       rec[0] = (long long)I.op | ((long long)I.layer << 8) | ((long long)I.n_units << 24);
       rec[1] = (long long)globaltimer_ns();
     }
-    if (ct == 0 && I.dep != kNoCounter)
-      if (!wait_counter(p, p.ctr + I.dep, I.dep_target, ii)) misc->stop = 1;
+    if (ct == 0) {
+      // counters only grow within a launch: step t waits for t + 1 steps' worth
+      bool ok = I.dep == kNoCounter || wait_counter(p, p.ctr + I.dep, I.dep_target * (uint32_t)(t + 1), ii);
+      // step t's first layer starts once step t - 1 wrote its ids (its input
+      // tokens, and the end of every read of the residual)
+      if (ok && t > 0 && I.op == OP_QKV && I.layer == 0)
+        ok = wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, ii);
+      if (!ok) misc->stop = 1;
+    }
     cbar();
     if (rec) rec[2] = (long long)globaltimer_ns();
     if (misc->stop) break;
@@ -980,12 +1028,12 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         const uint16_t* gain = static_cast<const uint16_t*>(I.ptr[3]);
         if (I.layer == 0) {
           if (ct < NBT) {
-            int t = ct < p.nb ? p.tokens[ct] : 0;
-            if (t < 0 || t >= D.V) {
-              raise_error(p, E_BAD_TOKEN, ii, (uint32_t)t, false);
-              t = 0;
+            int tk = ct < p.nb ? __ldcg(step_tokens + ct) : 0;  // may be written in this launch
+            if (tk < 0 || tk >= D.V) {
+              raise_error(p, E_BAD_TOKEN, ii, (uint32_t)tk, false);
+              tk = 0;
             }
-            misc->tok[ct] = t;
+            misc->tok[ct] = tk;
           }
           cbar();
           stage<NBT, true, true>(p, act, misc, nullptr, 0, D.H, gain, (int)I.aux0, (int)I.aux1);
@@ -1025,6 +1073,8 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     if (ct == 0 && I.sig != kNoCounter) red_release_add(p.ctr + I.sig, 1u);
     I = In;
     if (rec) rec[4] = (long long)globaltimer_ns();
+  }
+  if (misc->stop) break;
   }
 }
 

@@ -94,7 +94,9 @@ MK_HD inline int ctr_part(const Dims& D, int layer, int b, int g) {
   return D.L * kCountersPerLayer + (layer * kMaxNB + b) * D.Hkv + g;
 }
 MK_HD inline int ctr_lm(const Dims& D) { return D.L * kCountersPerLayer + D.L * kMaxNB * D.Hkv; }
-MK_HD inline int n_counters(const Dims& D) { return ctr_lm(D) + 1; }
+// steps of the current launch whose greedy ids are written (multi-step launches)
+MK_HD inline int ctr_step(const Dims& D) { return ctr_lm(D) + 1; }
+MK_HD inline int n_counters(const Dims& D) { return ctr_lm(D) + 2; }
 
 // attention unit i = (lane * Hkv + kv head) * S + slice
 MK_HD inline void attn_unit(uint32_t i, int Hkv, int S, int* b, int* g, int* s) {

@@ -139,6 +139,50 @@ def test_tiny_free_run_greedy_chained_on_device():
         assert got[t] == want[t], f"step {t}: {got[t]} != {want[t]}"
 
 
+def test_multi_step_launch_matches_single_steps_and_oracle():
+    """mk_decode_steps runs n chained greedy steps in one launch; its logits equal
+    n launches of mk_decode_step, and its ids follow the oracle's greedy run."""
+    cfg = configs.model_config("tiny", max_batch=3, max_seq=48)
+    w = H.gpu_weights(cfg)
+    lens = [5, 8, 11]
+    prompts = [synth.prompt_tokens(cfg, b, n).tolist() for b, n in enumerate(lens)]
+    n, V = 10, cfg["vocab"]
+    # multi-step: prefill every slot, one launch of n steps (lanes at different positions)
+    mk = _mk(cfg, w)
+    first = [mk.prefill(b, prompts[b]) for b in range(3)]
+    tok = torch.tensor(first, dtype=torch.int32, device="cuda")
+    ids = torch.empty((n, 3), dtype=torch.int32, device="cuda")
+    lg = torch.empty((n, 3, V), dtype=torch.float32, device="cuda")
+    mk.decode_steps(tok, lens, n, ids, lg)
+    mk.sync()
+    mk.close()
+    # the same steps one launch at a time
+    mk1 = _mk(cfg, w)
+    for b in range(3):
+        assert mk1.prefill(b, prompts[b]) == first[b]
+    cur = torch.tensor(first, dtype=torch.int32, device="cuda")
+    out1 = torch.empty(3, dtype=torch.int32, device="cuda")
+    lg1 = torch.empty((3, V), dtype=torch.float32, device="cuda")
+    for t in range(n):
+        mk1.decode_step(cur, [p + t for p in lens], out1, lg1)
+        mk1.sync()
+        np.testing.assert_allclose(lg[t].cpu().numpy(), lg1.cpu().numpy(), atol=2e-3, rtol=0)
+        assert out1.tolist() == ids[t].tolist()
+        cur.copy_(out1)
+    mk1.close()
+    # and the oracle's own greedy run, up to its first near-tie
+    from oracle import top2_margin
+
+    orc = H.oracle_for(cfg, w)
+    for b in range(3):
+        want, want_lg = orc.greedy(np.array(prompts[b]), n)
+        got = [first[b]] + ids[:, b].tolist()
+        for t in range(n + 1):
+            if float(top2_margin(want_lg[t])) <= H.MARGIN:
+                break
+            assert got[t] == want[t], (b, t)
+
+
 def test_zero_layers_greedy_is_identity_tiny():
     cfg = configs.model_config("tiny")
     w = H.gpu_weights(cfg, zero_layers=True)
