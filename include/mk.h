@@ -177,14 +177,20 @@ mk_status mk_get_error(mk_handle h, char* buf, int32_t len);
 mk_status mk_clear_error(mk_handle h);
 
 /* Profile records of the last step (handle created with mk_options.profile = 1).
- * Layout: int64 out[n_sm][stride][16]; record i of SM s describes the i-th
+ * Layout: int64 out[n_sm][stride][32]; record i of SM s describes the i-th
  * instruction of that SM's tape: [0] op | layer << 8 | n_units << 24,
  * [1] consumer start, [2] dependency met, [3] units done, [4] counter signalled,
  * [5] producer issued the first unit's page, [6] producer issued the last
  * unit's page (all %globaltimer ns, 0 where not reached); accumulated since the
- * last read: [7] ns the first consumer warp waited for its matvec pages,
- * [8] pages it took, [9] ns the producer waited for free ring slots, [10] matvec
- * pages it issued; [11..15] unused.  Reading resets the accumulators.
+ * last read: [7] ns the consumer warps waited for their matvec pages,
+ * [8] pages they took, [9] ns the producer waited for free ring slots, [10] matvec
+ * pages it issued; matvec instructions also record [11] activations staged,
+ * [12] the CTA's last warp finished its units, [13] the CTA passed its end
+ * barrier (the counter release follows), and accumulate [14] ns the first
+ * consumer warps spent in page dot products, [15] ns in the reductions and
+ * epilogues, [16] group re-reads of activations not yet written when first
+ * loaded, [17] ns those re-reads took (summed over threads); [18..31] unused.
+ * Reading resets the accumulators.
  * `cap` is the capacity of `out` in int64 elements; *n_sm and *stride are set
  * even when out is NULL, so a first call can size the buffer.  Synchronises
  * the device. */

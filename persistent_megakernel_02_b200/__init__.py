@@ -259,12 +259,12 @@ class Megakernel:
         return out.value if want_id else None
 
     def profile_records(self):
-        """Per-instruction profile records: int64 array [n_sm, stride, 16] (see mk_profile_read)."""
+        """Per-instruction profile records: int64 array [n_sm, stride, 32] (see mk_profile_read)."""
         import numpy as np
 
         n_sm, stride = ctypes.c_int32(), ctypes.c_int32()
         lib().mk_profile_read(self._h, None, 0, ctypes.byref(n_sm), ctypes.byref(stride))
-        out = np.zeros((n_sm.value, stride.value, 16), dtype=np.int64)
+        out = np.zeros((n_sm.value, stride.value, 32), dtype=np.int64)
         _check(lib().mk_profile_read(self._h, out.ctypes.data_as(ctypes.c_void_p), out.size,
                                      ctypes.byref(n_sm), ctypes.byref(stride)), "mk_profile_read")
         return out

@@ -28,7 +28,11 @@ struct mk_ctx {
   };
   std::vector<DevTape> dtapes;
   const uint16_t* embed = nullptr;
-  float *x = nullptr, *q = nullptr, *o = nullptr, *a = nullptr, *part = nullptr;
+  float* acts = nullptr;  // two sets of per-layer activation blocks (see KParams)
+  long long set_floats = 0, layer_floats = 0;
+  int off_q = 0, off_kvn = 0, off_o = 0, off_x1 = 0, off_a = 0, off_p = 0;
+  unsigned long long steps_run = 0;  // decode steps launched (activation-set parity)
+  float* part = nullptr;
   int2* lm_part = nullptr;
   uint16_t *kcache = nullptr, *vcache = nullptr;
   int* page_table = nullptr;
@@ -166,10 +170,20 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   h->embed = (const uint16_t*)w->embed;
   // scratch and state
   const int S1 = h->tapes[0].S;  // nb = 1 has the most slices
-  MK_TRY(dalloc(h, &h->x, (size_t)kMaxNB * D.H));
-  MK_TRY(dalloc(h, &h->q, (size_t)kMaxNB * D.qdim));
-  MK_TRY(dalloc(h, &h->o, (size_t)kMaxNB * D.qdim));
-  MK_TRY(dalloc(h, &h->a, (size_t)kMaxNB * D.F));
+  {
+    const int MB = D.max_batch;
+    long long off = 0;
+    h->off_q = (int)off;   off += (long long)MB * D.qdim;
+    h->off_kvn = (int)off; off += (long long)MB * 2 * D.kvdim;
+    h->off_o = (int)off;   off += (long long)MB * D.qdim;
+    h->off_x1 = (int)off;  off += (long long)MB * D.H;
+    h->off_a = (int)off;   off += (long long)MB * D.F;
+    h->off_p = (int)off;   off += (long long)D.n_ks * MB * D.H;
+    h->layer_floats = (off + 7) / 8 * 8;
+    h->set_floats = h->layer_floats * D.L;
+    MK_TRY(dalloc(h, &h->acts, (size_t)2 * h->set_floats));
+    MK_TRY(from_cuda(cudaMemset(h->acts, 0xFF, sizeof(float) * 2 * h->set_floats)));  // the sentinel
+  }
   MK_TRY(dalloc(h, &h->part, (size_t)kMaxNB * D.Hkv * S1 * D.rep * (D.d + 2)));
   MK_TRY(dalloc(h, &h->lm_part, (size_t)h->n_sm * kMaxNB));
   const size_t kv = (size_t)D.L * D.n_phys_pages * D.Hkv * D.PL * D.d;
@@ -232,7 +246,13 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.sm_off = dt.sm_off;
   p.S = t.S;
   p.embed = h->embed;
-  p.x = h->x; p.q = h->q; p.o = h->o; p.a = h->a; p.part = h->part; p.lm_part = h->lm_part;
+  p.acts = h->acts;
+  p.set_floats = h->set_floats;
+  p.layer_floats = h->layer_floats;
+  p.off_q = h->off_q; p.off_kvn = h->off_kvn; p.off_o = h->off_o;
+  p.off_x1 = h->off_x1; p.off_a = h->off_a; p.off_p = h->off_p;
+  p.parity0 = (int)(h->steps_run & 1);
+  p.part = h->part; p.lm_part = h->lm_part;
   p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
   const int par = (int)(h->step & 1);
   p.ctr = h->counters + (size_t)par * h->n_counters;
@@ -265,6 +285,7 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(nbt), dim3(h->n_sm), dim3(kThreads), args,
                                               (size_t)h->sm.total, st);
   h->step++;
+  if (e == cudaSuccess) h->steps_run += (unsigned long long)n_steps;
   return from_cuda(e);
 }
 
@@ -347,7 +368,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
     for (const Tape& t : h->tapes)
       for (int sm = 0; sm < h->n_sm; ++sm) stride = std::max(stride, (int)(t.sm_off[sm + 1] - t.sm_off[sm]));
     h->prof_stride = stride;
-    s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * 16);
+    s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * kProfSlots);
   }
   if (s == MK_OK && o.debug_fault == 1) {
     // test hook: one wait (the first layer-0 O projection of SM 0's tape for every
@@ -483,7 +504,7 @@ extern "C" mk_status mk_profile_read(mk_handle h, int64_t* out, int64_t cap, int
   *n_sm = h->n_sm;
   *stride = h->prof_stride;
   if (!h->prof) return MK_ERR_INVALID_ARG;
-  const int64_t need = (int64_t)h->n_sm * h->prof_stride * 16;
+  const int64_t need = (int64_t)h->n_sm * h->prof_stride * kProfSlots;
   if (!out || cap < need) return MK_ERR_INVALID_ARG;
   cudaSetDevice(h->dev);
   MK_TRY(from_cuda(cudaDeviceSynchronize()));
@@ -505,6 +526,7 @@ extern "C" mk_status mk_get_error(mk_handle h, char* buf, int32_t len) {
       case E_WAIT_EMPTY: what = "ring page release wait timed out"; break;
       case E_BAD_TOKEN: what = "token out of range"; break;
       case E_DRAIN: what = "in-flight copy drain timed out"; break;
+      case E_WAIT_DATA: what = "activation element wait timed out"; break;
       default: break;
     }
     snprintf(buf, (size_t)len, "%s (code %u, sm %u, instr %u, info %u, abort %u)", what, e.code, e.sm,
@@ -519,5 +541,7 @@ extern "C" mk_status mk_clear_error(mk_handle h) {
   MK_TRY(from_cuda(cudaDeviceSynchronize()));
   MK_TRY(from_cuda(cudaMemset(h->err, 0, sizeof(ErrWord))));
   MK_TRY(from_cuda(cudaMemset(h->counters, 0, sizeof(uint32_t) * 2 * h->n_counters)));
+  // an aborted step may have left written elements behind: every set back to the sentinel
+  MK_TRY(from_cuda(cudaMemset(h->acts, 0xFF, sizeof(float) * 2 * h->set_floats)));
   return from_cuda(cudaDeviceSynchronize());
 }

@@ -20,6 +20,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -88,8 +91,55 @@ __device__ __forceinline__ uint32_t atom_acq_rel_add(uint32_t* p, uint32_t v) {
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(o) : "l"(p), "r"(v) : "memory");
   return o;
 }
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+__device__ __forceinline__ void red_relaxed_add(uint32_t* p, uint32_t v) {
+  asm volatile("red.relaxed.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---- activations published once per step (see the kernel: sentinel protocol) ----
+// An element holds kSentinel until its single write of the step; writers store
+// canonical values only, so a reader that sees anything else has the new value.
+constexpr uint32_t kSentinel = 0xFFFFFFFFu;  // a NaN that arithmetic never produces
+__device__ __forceinline__ float canon(float v) { return v == v ? v : __uint_as_float(0x7FFFFFFFu); }
+__device__ __forceinline__ bool is_sent(float v) { return __float_as_uint(v) == kSentinel; }
+__device__ __forceinline__ bool any_sent(float4 v) {
+  return is_sent(v.x) | is_sent(v.y) | is_sent(v.z) | is_sent(v.w);
+}
+__device__ __forceinline__ bool any_sent(float2 v) { return is_sent(v.x) | is_sent(v.y); }
+// Activation stores carry an L2 evict_last hint: the weight stream passes
+// through L2 with evict_first, and an activation is read again up to a layer
+// later (the residual), which must not cost a DRAM round trip.
+__device__ __forceinline__ uint64_t l2_keep_policy() {
+  uint64_t p;
+  asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void st_relaxed_f32(float* p, float v) {
+  asm volatile("st.relaxed.gpu.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(l2_keep_policy())
+               : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u4(void* p, uint4 v) {
+  asm volatile("st.relaxed.gpu.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x),
+               "r"(v.y), "r"(v.z), "r"(v.w), "l"(l2_keep_policy())
+               : "memory");
+}
+// relaxed loads: every 32-bit element is single-copy atomic; volatile so a retry
+// loop re-reads and no two reads of one address are merged
+__device__ __forceinline__ float4 ld_relaxed_f4(const float* p) {
+  float4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float2 ld_relaxed_f2(const float* p) {
+  float2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ float ld_relaxed_f1(const float* p) {
+  float v;
+  asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p));
+  return v;
 }
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -123,6 +173,9 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   return v;
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
 __device__ __forceinline__ float4 ldcg4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ uint4 ldnc16(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 

@@ -14,8 +14,25 @@
 //                    the activation vector (with RMSNorm where the op fuses
 //                    it), then each warp takes whole pages (units), computes
 //                    the bf16 x fp32 matvec on CUDA cores and runs the op's
-//                    epilogue; at the end one thread bumps the op's counter
-//                    (release), the completion counters of the same article.
+//                    epilogue, and bumps the op's counter when its pages are
+//                    done (the completion counters of the same article).
+//
+// Publishing activations without a fence.  Inside a step every activation
+// element (q, the new K/V row, the attention output, the residual after the O
+// projection, the SwiGLU product, each down-projection K slice) is written
+// exactly once, into a buffer that holds a sentinel NaN until then.  Readers
+// check every element they load and re-read the ones that still hold the
+// sentinel, so a value is trusted by what it is, not by the order it became
+// visible in: the counters are only hints that tell a waiting SM when to start
+// reading (relaxed increments and polls), and no release fence -- which costs
+// microseconds per phase under a full HBM stream -- sits on the layer chain.
+// Buffers alternate between two sets by decode step; during step t every SM
+// refills its share of the other set with the sentinel, after step t - 1 has
+// ended everywhere (the step counter below) and before step t + 1 begins.  The
+// one acquire/release chain per step is the greedy-id reduction of the LM head
+// (acq_rel arrivals, a release of the step counter), which also orders this
+// step's KV-cache writes before the next step's bulk copies of them.
+//
 // Every wait is bounded (globaltimer); on timeout the CTA records an error word,
 // raises a global abort flag that every other waiter polls, drains its in-flight
 // copies and returns, so a bad tape cannot hang the GPU.
@@ -52,6 +69,7 @@ enum DevErr : uint32_t {
   E_WAIT_EMPTY = 3,    // a ring page was not released in time
   E_BAD_TOKEN = 4,     // a lane's token was outside [0, vocab) (treated as 0)
   E_DRAIN = 5,         // in-flight copies did not land before exit
+  E_WAIT_DATA = 6,     // an activation element was not written in time
 };
 
 struct KParams {
@@ -61,11 +79,20 @@ struct KParams {
   int S;  // attention slices per (lane, kv head)
   // the embedding table (layer-0 inputs); all other weights are named by the instructions
   const uint16_t* embed;
-  // state
-  float* x;     // [8][H] residual stream
-  float* q;     // [8][qdim] rotated queries
-  float* o;     // [8][qdim] attention output
-  float* a;     // [8][F] silu(gate) * up
+  // Activations: two sets (by decode-step parity) of L layer blocks of
+  // layer_floats floats.  Inside a block, with MB = max_batch lanes:
+  //   off_q   [MB][qdim]      rotated queries
+  //   off_kvn [MB][2][kvdim]  this step's K and V rows (fp32, before caching)
+  //   off_o   [MB][qdim]      attention output
+  //   off_x1  [MB][H]         residual after the O projection
+  //   off_a   [MB][F]         silu(gate) * up
+  //   off_p   [n_ks][MB][H]   down projection, one partial per K slice
+  // The residual after the down projection is x1 + P_0 + ... + P_{n_ks-1},
+  // summed in that order wherever it is read.
+  float* acts;
+  long long set_floats, layer_floats;
+  int off_q, off_kvn, off_o, off_x1, off_a, off_p;
+  int parity0;  // set of this launch's step 0
   float* part;  // attention partials [8][Hkv][S][rep][d + 2]
   int2* lm_part;  // [n_sm][8] best (value bits, index) per SM
   uint16_t* kcache;
@@ -93,7 +120,7 @@ struct KParams {
   float* logits;
   int* ids;
   unsigned long long wait_limit_ns;
-  long long* prof;   // profile records [n_sm][prof_stride][16] or null
+  long long* prof;   // profile records [n_sm][prof_stride][kProfSlots] or null
   int prof_stride;
   // shared memory layout
   int ring_pages, act_off, bar_off, misc_off;
@@ -101,14 +128,23 @@ struct KParams {
 };
 
 struct Misc {
+  // a copy of the launch parameters: producer and consumers read them through a
+  // reference, and a generic load of the parameter space is a global-memory load
+  KParams kp;
   float red[kConsumerWarps][kMaxNB];
   float lmv[kConsumerWarps][kMaxNB];
   int lmi[kConsumerWarps][kMaxNB];
   int tok[kMaxNB];
+  long long warp_done[kConsumerWarps];  // profile mode: when each warp finished its units
   int pos[kMaxNB];       // each lane's position in the current step
   int step;              // the current step of this launch
   int cur_phys[kMaxNB];  // physical KV page holding each lane's position this step
   float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
+  float* actset;         // the activation set of the current step
+  unsigned int slow_n;   // profile mode: group re-reads of unwritten activations
+  unsigned long long slow_ns;  // and the time they took (summed over threads)
+  long long t_stage_in, t_stage_loaded;  // profile mode: stage entry, thread 0's loads back
+  long long t_sum_x1, t_sum_p;           // profile mode: residual sum, x1 back, partials back
   volatile int stop;
   volatile int last;
   uint32_t issued;  // pages the ring producer issued
@@ -148,6 +184,118 @@ __device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, u
     }
     if (it > 512) __nanosleep(32);
   }
+}
+
+// Spin until the hint counter *c reaches target (relaxed: the data it announces
+// is validated element by element), the abort flag rises, or the time passes.
+__device__ __noinline__ bool wait_hint(const KParams& p, const uint32_t* c, uint32_t target, uint32_t instr) {
+  if (ld_relaxed_u32(c) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_relaxed_u32(c) >= target) return true;
+    if ((it & 63) == 0) {
+      if (aborted(p)) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_COUNTER, instr, target, true);
+        return false;
+      }
+    }
+    if (it > 512) __nanosleep(32);
+  }
+}
+
+// Re-read an activation element group until no element holds the sentinel
+// (bounded; on timeout or abort the CTA stops and zeros are returned).
+__device__ __noinline__ float4 poll4_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    const float4 v = ld_relaxed_f4(src);
+    if (!any_sent(v)) return v;
+    if ((it & 63) == 0) {
+      if (aborted(p)) break;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_DATA, instr, 4, true);
+        break;
+      }
+    }
+  }
+  misc->stop = 1;
+  return make_float4(0.f, 0.f, 0.f, 0.f);
+}
+__device__ __noinline__ float2 poll2_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    const float2 v = ld_relaxed_f2(src);
+    if (!any_sent(v)) return v;
+    if ((it & 63) == 0) {
+      if (aborted(p)) break;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_DATA, instr, 2, true);
+        break;
+      }
+    }
+  }
+  misc->stop = 1;
+  return make_float2(0.f, 0.f);
+}
+__device__ __noinline__ float poll1_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    const float v = ld_relaxed_f1(src);
+    if (!is_sent(v)) return v;
+    if ((it & 63) == 0) {
+      if (aborted(p)) break;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_DATA, instr, 1, true);
+        break;
+      }
+    }
+  }
+  misc->stop = 1;
+  return 0.f;
+}
+// Bookkeeping of a group re-read: true while the group may be read again;
+// false (CTA stopped, error raised on timeout) once it may not.
+struct Spin {
+  uint64_t t0 = 0, tp = 0;
+  uint32_t it = 0;
+  const KParams* pp;
+  Misc* m;
+  __device__ __forceinline__ Spin(const KParams& p, Misc* misc) : pp(&p), m(misc) {
+    if (p.prof) {
+      tp = globaltimer_ns();
+      atomicAdd(&misc->slow_n, 1u);
+    }
+  }
+  __device__ __forceinline__ ~Spin() {
+    if (pp->prof) atomicAdd(&m->slow_ns, (unsigned long long)(globaltimer_ns() - tp));
+  }
+  __device__ __forceinline__ bool again(const KParams& p, uint32_t instr, uint32_t info, Misc* misc) {
+    ++it;
+    if ((it & 15) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      if (aborted(p)) { misc->stop = 1; return false; }
+      if (now - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_DATA, instr, info, true);
+        misc->stop = 1;
+        return false;
+      }
+    }
+    if (it > 4) __nanosleep(64);
+    return true;
+  }
+};
+
+// fast path: the caller issues its loads first, then validates each
+__device__ __forceinline__ void ready(float4& v, const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  if (any_sent(v)) v = poll4_slow(p, src, instr, misc);
+}
+__device__ __forceinline__ void ready(float2& v, const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  if (any_sent(v)) v = poll2_slow(p, src, instr, misc);
+}
+__device__ __forceinline__ void ready(float& v, const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+  if (is_sent(v)) v = poll1_slow(p, src, instr, misc);
 }
 
 // Wait for an mbarrier phase.  The abort flag (an L2 load) and the clock are
@@ -268,15 +416,19 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
   if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1 && ok; ++ii) {
     const Instr In = ii + 1 < i1 ? p.instrs[ii + 1] : I;
-    long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 16 : nullptr;
+    long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * kProfSlots : nullptr;
     long long acc_wait = 0, acc_pages = 0;
     if (rec) rec[5] = (long long)globaltimer_ns();
     if (I.op == OP_ATTN) {
       // KV pages of step t hold the positions earlier steps of this launch wrote:
-      // copy them only once those steps' QKV instructions for this layer are done.
-      // (By then this producer has issued every page of the earlier steps, so the
-      // wait cannot hold up the consumers it depends on.)
-      if (t > 0 && !(ok = wait_counter(p, p.ctr + I.dep, I.dep_target * (uint32_t)t, ii))) break;
+      // copy them only once step t - 1 has ended (its greedy ids are out, which
+      // every SM's KV writes of that step precede).  By then this producer has
+      // issued every page of the earlier steps, so the wait cannot hold up the
+      // consumers it depends on.
+      if (t > 0) {
+        if (!(ok = wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, ii))) break;
+        fence_proxy_async_global();  // the bulk copies below read what the acquire made visible
+      }
       for (uint32_t k = 0; k < I.n_units && ok; ++k) {
         int b, g, s;
         attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
@@ -329,19 +481,91 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
 
 // ---------------------------------------------------------------- consumers: staging
 
+// Slow paths of the staging: some element of the chunk still held the
+// sentinel, so the whole group of loads is issued again (in parallel) until
+// every element is written.  Results come back by value: a fast-path variable
+// whose address escaped would live in local memory and serialise its loads.
+template <int NBT>
+struct Chunk8 {
+  float4 l[NBT], h[NBT];
+};
+template <int NBT>
+__device__ __noinline__ Chunk8<NBT> stage_one_slow(const KParams& p, const float* src, int ld, uint32_t ii,
+                                                   Misc* misc) {
+  Chunk8<NBT> r;
+  Spin sp(p, misc);
+  do {
+    bool bad = false;
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) {
+      r.l[b] = r.h[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b < p.nb) {
+        r.l[b] = ld_relaxed_f4(src + (size_t)b * ld);
+        r.h[b] = ld_relaxed_f4(src + (size_t)b * ld + 4);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < NBT; ++b) bad |= any_sent(r.l[b]) | any_sent(r.h[b]);
+    if (!bad) return r;
+  } while (sp.again(p, ii, 8, misc));
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) r.l[b] = r.h[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+  return r;
+}
+// one 8-element chunk of x1 + P_0 + ... + P_{n_ks-1} (same order of additions)
+__device__ __noinline__ Chunk8<1> resid_chunk_slow(const KParams& p, const float* xs, const float* P0,
+                                                   size_t mbh, size_t off, uint32_t ii, Misc* misc) {
+  Chunk8<1> out;
+  Spin sp(p, misc);
+  do {
+    float4 l = ld_relaxed_f4(xs), h = ld_relaxed_f4(xs + 4);
+    float4 pl[kMaxKS], ph[kMaxKS];
+#pragma unroll
+    for (int s = 0; s < kMaxKS; ++s)
+      if (s < p.D.n_ks) {
+        pl[s] = ld_relaxed_f4(P0 + s * mbh + off);
+        ph[s] = ld_relaxed_f4(P0 + s * mbh + off + 4);
+      }
+    bool bad = any_sent(l) | any_sent(h);
+#pragma unroll
+    for (int s = 0; s < kMaxKS; ++s)
+      if (s < p.D.n_ks) bad |= any_sent(pl[s]) | any_sent(ph[s]);
+    if (!bad) {
+#pragma unroll
+      for (int s = 0; s < kMaxKS; ++s)
+        if (s < p.D.n_ks) {
+          l.x += pl[s].x; l.y += pl[s].y; l.z += pl[s].z; l.w += pl[s].w;
+          h.x += ph[s].x; h.y += ph[s].y; h.z += ph[s].z; h.w += ph[s].w;
+        }
+      out.l[0] = l;
+      out.h[0] = h;
+      return out;
+    }
+  } while (sp.again(p, ii, 9, misc));
+  out.l[0] = out.h[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  return out;
+}
+
 // Stage NBT activation rows of length K into shared memory in the split layout
 // used by the matvec (chunk c of lane b: elements 8c..8c+3 at lo[b*nch + c],
-// 8c+4..8c+7 at hi[b*nch + c]).  Source: fp32 rows (L2, written by other SMs in
-// this step) or, for layer 0, the bf16 embedding rows of the lanes' tokens, which
-// are also written to the residual rows [xlo, xhi).  NORM applies RMSNorm with
-// the bf16 gain.  Lanes >= nb are zero.
-template <int NBT, bool EMB, bool NORM>
-__device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, const float* src,
-                                      int ld, int K, const uint16_t* gain, int xlo, int xhi) {
+// 8c+4..8c+7 at hi[b*nch + c]).  Sources (MODE):
+//   ST_EMB  the bf16 embedding rows of the lanes' tokens (layer 0);
+//   ST_ONE  one fp32 vector per lane at src + b * ld;
+//   ST_SUM  the residual after a down projection: x1 at src + b * H plus the
+//           layer's n_ks partials, added in slice order.
+// fp32 sources are this step's activations: every element is validated against
+// the sentinel (and re-read until written).  NORM applies RMSNorm with the bf16
+// gain.  Lanes >= nb are zero.
+enum { ST_EMB = 0, ST_ONE = 1, ST_SUM = 2 };
+
+template <int NBT, int MODE, bool NORM>
+__device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, const float* src, int ld,
+                                      int K, const uint16_t* gain, uint32_t ii) {
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const int nch = K >> 3;
   float4* lo = reinterpret_cast<float4*>(act);
   float4* hi = lo + NBT * nch;
+  if (p.prof && ct == 0) misc->t_stage_in = (long long)globaltimer_ns();
   float ss[NBT];
 #pragma unroll
   for (int b = 0; b < NBT; ++b) ss[b] = 0.f;
@@ -352,29 +576,86 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
       g[0] = bf_lo(gw.x); g[1] = bf_hi(gw.x); g[2] = bf_lo(gw.y); g[3] = bf_hi(gw.y);
       g[4] = bf_lo(gw.z); g[5] = bf_hi(gw.z); g[6] = bf_lo(gw.w); g[7] = bf_hi(gw.w);
     }
+    float4 vl[NBT], vh[NBT];
+    if constexpr (MODE == ST_EMB) {
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {
+        if (b < p.nb) {
+          const uint4 w = ldnc16(p.embed + (size_t)misc->tok[b] * p.D.H + c * 8);
+          vl[b] = make_float4(bf_lo(w.x), bf_hi(w.x), bf_lo(w.y), bf_hi(w.y));
+          vh[b] = make_float4(bf_lo(w.z), bf_hi(w.z), bf_lo(w.w), bf_hi(w.w));
+        } else {
+          vl[b] = vh[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+    } else if constexpr (MODE == ST_ONE) {
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {  // issue every load, then validate
+        if (b < p.nb) {
+          vl[b] = ld_relaxed_f4(src + (size_t)b * ld + c * 8);
+          vh[b] = ld_relaxed_f4(src + (size_t)b * ld + c * 8 + 4);
+        } else {
+          vl[b] = vh[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      bool bad = false;
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) bad |= any_sent(vl[b]) | any_sent(vh[b]);
+      if (bad) {
+        const Chunk8<NBT> r = stage_one_slow<NBT>(p, src + c * 8, ld, ii, misc);
+#pragma unroll
+        for (int b = 0; b < NBT; ++b) { vl[b] = r.l[b]; vh[b] = r.h[b]; }
+      }
+    } else {
+      const size_t mbh = (size_t)p.D.max_batch * p.D.H;
+      const float* P0 = src + (p.off_p - p.off_x1);
+      const int nks = p.D.n_ks;
+#pragma unroll
+      for (int b = 0; b < NBT; ++b) {
+        vl[b] = vh[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (b >= p.nb) continue;
+        const float* xs = src + (size_t)b * p.D.H + c * 8;
+        float4 l0 = ld_relaxed_f4(xs), h0 = ld_relaxed_f4(xs + 4);
+        float4 pl[kMaxKS], ph[kMaxKS];
+#pragma unroll
+        for (int s = 0; s < kMaxKS; ++s)
+          if (s < nks) {
+            pl[s] = ld_relaxed_f4(P0 + s * mbh + (size_t)b * p.D.H + c * 8);
+            ph[s] = ld_relaxed_f4(P0 + s * mbh + (size_t)b * p.D.H + c * 8 + 4);
+          }
+        if (p.prof && ct == 0 && b == 0) {  // which source comes back last (profile only)
+          if (__float_as_uint(l0.x) == 0x7FC00001u) misc->slow_n += 0u;
+          misc->t_sum_x1 = (long long)globaltimer_ns();
+          if (__float_as_uint(pl[nks - 1].x) == 0x7FC00001u) misc->slow_n += 0u;
+          misc->t_sum_p = (long long)globaltimer_ns();
+        }
+        bool bad = any_sent(l0) | any_sent(h0);
+#pragma unroll
+        for (int s = 0; s < kMaxKS; ++s)
+          if (s < nks) bad |= any_sent(pl[s]) | any_sent(ph[s]);
+        if (bad) {  // rare: some element not yet visible; re-read the chunk element by element
+          const Chunk8<1> r = resid_chunk_slow(p, xs, P0, mbh, (size_t)b * p.D.H + c * 8, ii, misc);
+          l0 = r.l[0];
+          h0 = r.h[0];
+        } else {
+#pragma unroll
+          for (int s = 0; s < kMaxKS; ++s)
+            if (s < nks) {
+              l0.x += pl[s].x; l0.y += pl[s].y; l0.z += pl[s].z; l0.w += pl[s].w;
+              h0.x += ph[s].x; h0.y += ph[s].y; h0.z += ph[s].z; h0.w += ph[s].w;
+            }
+        }
+        vl[b] = l0;
+        vh[b] = h0;
+      }
+    }
+    if (p.prof && ct == 0 && c == 0) {  // the branch waits for the loaded value, then the clock is read
+      if (__float_as_uint(vl[0].x) == 0x7FC00001u) misc->slow_n += 0u;
+      misc->t_stage_loaded = (long long)globaltimer_ns();
+    }
 #pragma unroll
     for (int b = 0; b < NBT; ++b) {
-      float v[8];
-      if (b < p.nb) {
-        if (EMB) {
-          const uint4 w = ldnc16(p.embed + (size_t)misc->tok[b] * p.D.H + c * 8);
-          v[0] = bf_lo(w.x); v[1] = bf_hi(w.x); v[2] = bf_lo(w.y); v[3] = bf_hi(w.y);
-          v[4] = bf_lo(w.z); v[5] = bf_hi(w.z); v[6] = bf_lo(w.w); v[7] = bf_hi(w.w);
-          const int k0 = c * 8;
-          if (k0 + 8 > xlo && k0 < xhi) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-              if (k0 + e >= xlo && k0 + e < xhi) p.x[(size_t)b * p.D.H + k0 + e] = v[e];
-          }
-        } else {
-          const float4 a0 = ldcg4(src + (size_t)b * ld + c * 8), a1 = ldcg4(src + (size_t)b * ld + c * 8 + 4);
-          v[0] = a0.x; v[1] = a0.y; v[2] = a0.z; v[3] = a0.w;
-          v[4] = a1.x; v[5] = a1.y; v[6] = a1.z; v[7] = a1.w;
-        }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-      }
+      float v[8] = {vl[b].x, vl[b].y, vl[b].z, vl[b].w, vh[b].x, vh[b].y, vh[b].z, vh[b].w};
       if (NORM) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -502,6 +783,63 @@ __device__ __forceinline__ int rs_base(int n, int keep, int lane) {
   return idx;
 }
 
+// The residual entering layer `layer` at (lane b, row): the embedding for
+// layer 0, else the previous layer's x1 + P_0 + ... + P_{n_ks-1} (the order the
+// stage adds them in, so both see the same fp32 value).  The loads are issued
+// here; resid_finish validates and adds them once the caller needs the value.
+struct ResidIn {
+  float x, pp[kMaxKS];
+  const float* src;
+};
+__device__ __forceinline__ void resid_issue(const KParams& p, const Misc* misc, int layer, int b, int row,
+                                            ResidIn& r) {
+  if (layer == 0) {
+    r.src = nullptr;
+    r.x = __uint_as_float((uint32_t)p.embed[(size_t)misc->tok[b] * p.D.H + row] << 16);
+    return;
+  }
+  const float* prev = misc->actset + (size_t)(layer - 1) * p.layer_floats;
+  r.src = prev + p.off_x1 + (size_t)b * p.D.H + row;
+  r.x = ld_relaxed_f1(r.src);
+  const size_t mbh = (size_t)p.D.max_batch * p.D.H;
+#pragma unroll
+  for (int s = 0; s < kMaxKS; ++s)
+    if (s < p.D.n_ks) r.pp[s] = ld_relaxed_f1(prev + p.off_p + s * mbh + (size_t)b * p.D.H + row);
+}
+__device__ __noinline__ ResidIn resid_slow(const KParams& p, Misc* misc, ResidIn r, uint32_t ii) {
+  const size_t mbh = (size_t)p.D.max_batch * p.D.H;
+  const float* P0 = r.src + (p.off_p - p.off_x1);
+  Spin sp(p, misc);
+  do {
+    r.x = ld_relaxed_f1(r.src);
+#pragma unroll
+    for (int s = 0; s < kMaxKS; ++s)
+      if (s < p.D.n_ks) r.pp[s] = ld_relaxed_f1(P0 + s * mbh);
+    bool bad = is_sent(r.x);
+#pragma unroll
+    for (int s = 0; s < kMaxKS; ++s)
+      if (s < p.D.n_ks) bad |= is_sent(r.pp[s]);
+    if (!bad) return r;
+  } while (sp.again(p, ii, 10, misc));
+  r.x = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxKS; ++s) r.pp[s] = 0.f;
+  return r;
+}
+__device__ __forceinline__ float resid_finish(const KParams& p, Misc* misc, ResidIn& r, uint32_t ii) {
+  if (!r.src) return r.x;
+  bool bad = is_sent(r.x);
+#pragma unroll
+  for (int s = 0; s < kMaxKS; ++s)
+    if (s < p.D.n_ks) bad |= is_sent(r.pp[s]);
+  if (bad) r = resid_slow(p, misc, r, ii);
+  float x = r.x;
+#pragma unroll
+  for (int s = 0; s < kMaxKS; ++s)
+    if (s < p.D.n_ks) x += r.pp[s];
+  return x;
+}
+
 __device__ __forceinline__ bool lm_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
@@ -528,10 +866,11 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
   int besti[NBT];
 #pragma unroll
   for (int b = 0; b < NBT; ++b) { bestv[b] = -CUDART_INF_F; besti[b] = 0x7FFFFFFF; }
-  long long* prec = (p.prof && cw == 0)
-                        ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - p.sm_off[blockIdx.x])) * 16
+  long long* prec = p.prof
+                        ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - p.sm_off[blockIdx.x])) * kProfSlots
                         : nullptr;
-  long long c_wait = 0, c_pages = 0;
+  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;  // this layer's activation block
+  long long c_wait = 0, c_pages = 0, c_core = 0, c_epi = 0;
   // this step's logits (LM head only)
   float* lg = nullptr;
   if (OPK == OP_LM && p.logits) {
@@ -544,6 +883,15 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
   for (uint32_t k = cw; k < I.n_units; k += kConsumerWarps, rp.advance(kConsumerWarps, NP)) {
     const uint32_t u = I.u0 + k;
     const uint32_t slot = rp.slot;
+    ResidIn rin[OPK == OP_O ? NL : 1];
+    if constexpr (OPK == OP_O) {  // the residual rows this lane will write, loaded under the page wait
+      const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
+#pragma unroll
+      for (int m = 0; m < NL; ++m) {
+        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
+        if (writer && r < nr && b < p.nb) resid_issue(p, misc, I.layer, b, r0 + r, rin[m]);
+      }
+    }
     const long long tw = prec ? (long long)globaltimer_ns() : 0;
     bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
     if (prec) { c_wait += (long long)globaltimer_ns() - tw; c_pages += 1; }
@@ -556,9 +904,12 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
     for (int r = 0; r < RT; ++r)
 #pragma unroll
       for (int b = 0; b < NBT; ++b) acc[r][b] = make_float2(0.f, 0.f);
+    const long long tc = prec ? (long long)globaltimer_ns() : 0;
     mv_core<RT, NBT>(smem_u32(ring + (size_t)slot * kPageBytes), alo, ahi, nch, lane, acc);
     __syncwarp();
     if (lane == 0) mbar_arrive_cnt(&empty[slot], kConsumerWarps);
+    const long long te = prec ? (long long)globaltimer_ns() : 0;
+    if (prec) c_core += te - tc;
 
     float v[NV];
     if constexpr (PAIRED) {
@@ -594,15 +945,19 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
           r2 = v2 * cs.x + v1 * cs.y;
         }
         if (sec == 0) {
-          float* qq = p.q + (size_t)b * D.qdim + hh * D.d;
-          qq[i] = r1;
-          qq[i + half] = r2;
+          float* qq = lay + p.off_q + (size_t)b * D.qdim + hh * D.d;
+          st_relaxed_f32(qq + i, canon(r1));
+          st_relaxed_f32(qq + i + half, canon(r2));
         } else {
+          // the cache row serves later steps; this step's attention reads the fp32 copy
           const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
                                  (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
           uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
           cache[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
           cache[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
+          float* kv = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + (sec - 1) * D.kvdim + hh * D.d;
+          st_relaxed_f32(kv + i, canon(r1));
+          st_relaxed_f32(kv + i + half, canon(r2));
         }
       }
     } else if constexpr (OPK == OP_GU) {
@@ -612,14 +967,24 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         const int pi = vbase / 2 + m, r = pi / NBT, b = pi % NBT;
         if (!writer || r >= nr || b >= p.nb) continue;
         const float g = v[2 * m], up = v[2 * m + 1];
-        p.a[(size_t)b * D.F + r0 + r] = g / (1.0f + __expf(-g)) * up;
+        st_relaxed_f32(lay + p.off_a + (size_t)b * D.F + r0 + r, canon(g / (1.0f + __expf(-g)) * up));
       }
-    } else if constexpr (OPK == OP_O || OPK == OP_DOWN) {
+    } else if constexpr (OPK == OP_O) {  // x1 = residual + Wo . o
       const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
 #pragma unroll
       for (int m = 0; m < NL; ++m) {
         const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
-        if (writer && r < nr && b < p.nb) red_add_f32(p.x + (size_t)b * D.H + r0 + r, v[m]);
+        if (writer && r < nr && b < p.nb)
+          st_relaxed_f32(lay + p.off_x1 + (size_t)b * D.H + r0 + r,
+                         canon(resid_finish(p, misc, rin[m], ii) + v[m]));
+      }
+    } else if constexpr (OPK == OP_DOWN) {  // this K slice's partial of Wd . a
+      const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
+      float* P = lay + p.off_p + (size_t)I.arg * D.max_batch * D.H;
+#pragma unroll
+      for (int m = 0; m < NL; ++m) {
+        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
+        if (writer && r < nr && b < p.nb) st_relaxed_f32(P + (size_t)b * D.H + r0 + r, canon(v[m]));
       }
     } else if constexpr (OPK == OP_LM) {
       const int r0 = (int)u * RT, nr = min(RT, D.V - r0);
@@ -633,9 +998,20 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         if (writer && lg) lg[(size_t)b * D.V + r0 + r] = v[m];
       }
     }
+    if (prec) c_epi += (long long)globaltimer_ns() - te;
   }
 
-  if (prec && lane == 0) { prec[7] += c_wait; prec[8] += c_pages; }
+  if (prec && lane == 0) {  // summed over the warps
+    unsigned long long* pr = reinterpret_cast<unsigned long long*>(prec);
+    atomicAdd(pr + 7, (unsigned long long)c_wait);
+    atomicAdd(pr + 8, (unsigned long long)c_pages);
+    atomicAdd(pr + 14, (unsigned long long)c_core);
+    atomicAdd(pr + 15, (unsigned long long)c_epi);
+  }
+  if (p.prof && lane == 0) misc->warp_done[cw] = (long long)globaltimer_ns();  // profile only
+  // this warp's share is written: bump the hint counter (every warp, pages or not)
+  __syncwarp();
+  if (lane == 0 && I.sig != kNoCounter) red_relaxed_add(p.ctr + I.sig, 1u);
   if constexpr (OPK == OP_LM) {
     // combine the lanes' and warps' running argmax, publish this SM's, the last SM reduces
 #pragma unroll
@@ -715,6 +1091,7 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
   float* comb = act + REP * DH;
   const float scale = 1.0f / sqrtf((float)DH);
   const int myh = lane % REP;  // the query head of every score this lane computes
+  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;  // this layer's activation block
   uint32_t used = 0;
 
   for (uint32_t k = 0; k < I.n_units; ++k) {
@@ -724,24 +1101,42 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     if (s >= se) continue;  // uniform: this slice is not needed at this context length
     const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
     const int np_ = pe - pb;
-    // the warp owning this step's position (if this slice holds it) fetches its
-    // freshly written K/V row now, overlapping the q load
+    // the warp owning this step's position (if this slice holds it) fetches the
+    // fp32 K/V row the QKV instruction published, rounded as the cache holds it,
+    // overlapping the q load
     const int rcur_all = pos - (npg - 1) * PL;  // row of pos within the last page
     const bool own_cur = pe == npg && rcur_all / RPW == cw;
     uint32_t kcur[DH / 64], vcur[DH / 64];
     if (own_cur) {
-      const size_t base = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + g) *
-                              (size_t)(PL * DH) + (size_t)rcur_all * DH;
+      const float* kn = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + g * DH + lane * (DH / 32);
+      const float* vn = kn + D.kvdim;
+      float kf[DH / 32], vf[DH / 32];
+      if constexpr (DH == 64) {
+        float2 k2 = ld_relaxed_f2(kn), v2 = ld_relaxed_f2(vn);
+        ready(k2, p, kn, ii, misc);
+        ready(v2, p, vn, ii, misc);
+        kf[0] = k2.x; kf[1] = k2.y; vf[0] = v2.x; vf[1] = v2.y;
+      } else {
+        float4 k4 = ld_relaxed_f4(kn), v4 = ld_relaxed_f4(vn);
+        ready(k4, p, kn, ii, misc);
+        ready(v4, p, vn, ii, misc);
+        kf[0] = k4.x; kf[1] = k4.y; kf[2] = k4.z; kf[3] = k4.w;
+        vf[0] = v4.x; vf[1] = v4.y; vf[2] = v4.z; vf[3] = v4.w;
+      }
 #pragma unroll
       for (int e = 0; e < DH / 64; ++e) {
-        kcur[e] = __ldcg(reinterpret_cast<const unsigned int*>(p.kcache + base) + lane * (DH / 64) + e);
-        vcur[e] = __ldcg(reinterpret_cast<const unsigned int*>(p.vcache + base) + lane * (DH / 64) + e);
+        kcur[e] = KV16F ? (uint32_t)f2h(kf[2 * e]) | ((uint32_t)f2h(kf[2 * e + 1]) << 16)
+                        : (uint32_t)f2bf(kf[2 * e]) | ((uint32_t)f2bf(kf[2 * e + 1]) << 16);
+        vcur[e] = KV16F ? (uint32_t)f2h(vf[2 * e]) | ((uint32_t)f2h(vf[2 * e + 1]) << 16)
+                        : (uint32_t)f2bf(vf[2 * e]) | ((uint32_t)f2bf(vf[2 * e + 1]) << 16);
       }
     }
     for (int e = ct; e < REP * DC; e += 256) {
       const int h = e / DC, c = e % DC;
-      const float* src = p.q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
-      float4 a0 = ldcg4(src), a1 = ldcg4(src + 4);
+      const float* src = lay + p.off_q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
+      float4 a0 = ld_relaxed_f4(src), a1 = ld_relaxed_f4(src + 4);
+      ready(a0, p, src, ii, misc);
+      ready(a1, p, src + 4, ii, misc);
       a0.x *= scale; a0.y *= scale; a0.z *= scale; a0.w *= scale;
       a1.x *= scale; a1.y *= scale; a1.z *= scale; a1.w *= scale;
       qlo[h * DC + c] = a0;
@@ -884,10 +1279,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
             O += comb[(w * REP + h) * CS + i] * f;
           }
         }
-        p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
+        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
       }
       cbar();
-      if (ct == 0) red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+      if (ct == 0) red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
       used += (uint32_t)np_;
       cbar();
       continue;
@@ -931,12 +1326,12 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
             O += __ldcg(pp + (t * REP + h) * CS + i) * f;
           }
         }
-        p.o[(size_t)b * D.qdim + (g * REP + h) * DH + i] = O / L;
+        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
       }
       cbar();
       if (ct == 0) {
         p.ctr[ctr_part(D, I.layer, b, g)] = 0u;  // the next step's slices count from zero
-        red_release_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+        red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
       }
     }
     used += (uint32_t)np_;
@@ -987,59 +1382,76 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   uint32_t page_base = 0;
   const int half = D.d / 2;
   for (int t = 0; t < p.n_steps; ++t) {
-  // per-step constants: positions, RoPE (cos, sin) at each lane's position, and the
-  // KV page that position lives in
-  if (ct == 0) misc->step = t;
+  // step t begins once step t - 1 has written its ids everywhere (acquire): its
+  // tokens, every read of its activations and every write of its KV rows are done
+  if (ct == 0) {
+    misc->step = t;
+    misc->actset = p.acts + (size_t)((p.parity0 + t) & 1) * p.set_floats;
+    if (t > 0 && !wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, i0)) misc->stop = 1;
+  }
+  cbar();
+  if (misc->stop) break;
+  // per-step constants: positions, tokens, RoPE (cos, sin) at each lane's
+  // position, and the KV page that position lives in
   if (ct < p.nb) {
     misc->pos[ct] = p.pos[ct] + t;
     misc->cur_phys[ct] = p.page_table[p.slot[ct] * D.pages_per_seq + (p.pos[ct] + t) / D.PL];
+  }
+  if (ct < NBT) {
+    const int* step_tokens = (p.chain && t > 0) ? p.ids + (size_t)(t - 1) * p.ids_stride
+                                                : p.tokens + (size_t)(p.chain ? 0 : t) * p.nb;
+    int tk = ct < p.nb ? __ldcg(step_tokens + ct) : 0;  // may be written in this launch
+    if (tk < 0 || tk >= D.V) {
+      raise_error(p, E_BAD_TOKEN, i0, (uint32_t)tk, false);
+      tk = 0;
+    }
+    misc->tok[ct] = tk;
   }
   for (int e = ct; e < p.nb * half; e += 256) {
     const int b = e / half, i = e % half;
     misc->rope_cs[b][i] = p.rope[(size_t)(p.pos[b] + t) * half + i];
   }
-  const int* step_tokens = (p.chain && t > 0) ? p.ids + (size_t)(t - 1) * p.ids_stride
-                                              : p.tokens + (size_t)(p.chain ? 0 : t) * p.nb;
+  {  // refill this SM's share of the other activation set with the sentinel
+    uint4* other = reinterpret_cast<uint4*>(p.acts + (size_t)((p.parity0 + t + 1) & 1) * p.set_floats);
+    const long long n4 = p.set_floats / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
+    const long long lo = (long long)blockIdx.x * per, hi = min(n4, lo + per);
+    const uint4 sv = make_uint4(kSentinel, kSentinel, kSentinel, kSentinel);
+    for (long long e = lo + ct; e < hi; e += 256) st_relaxed_u4(other + e, sv);
+  }
   cbar();
+  bool stopped = false;  // set only where every warp reads misc->stop together
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1; ++ii) {
     const Instr In = ii + 1 < i1 ? p.instrs[ii + 1] : I;  // loaded while this one runs
-    long long* rec = (p.prof && ct == 0) ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * 16 : nullptr;
+    long long* rec = (p.prof && ct == 0) ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * kProfSlots : nullptr;
+    // The next instruction's RMSNorm gain is read once per step: pull it into L2
+    // now, so its staging does not start behind a DRAM miss.
+    if ((In.op == OP_QKV || In.op == OP_GU || In.op == OP_LM) && ct < 32 && ct * 64 < D.H)
+      prefetch_l2(static_cast<const uint16_t*>(In.ptr[3]) + ct * 64);
     if (rec) {
       rec[0] = (long long)I.op | ((long long)I.layer << 8) | ((long long)I.n_units << 24);
       rec[1] = (long long)globaltimer_ns();
     }
-    if (ct == 0) {
-      // counters only grow within a launch: step t waits for t + 1 steps' worth
-      bool ok = I.dep == kNoCounter || wait_counter(p, p.ctr + I.dep, I.dep_target * (uint32_t)(t + 1), ii);
-      // step t's first layer starts once step t - 1 wrote its ids (its input
-      // tokens, and the end of every read of the residual)
-      if (ok && t > 0 && I.op == OP_QKV && I.layer == 0)
-        ok = wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, ii);
-      if (!ok) misc->stop = 1;
+    if (ct == 0 && I.dep != kNoCounter) {
+      // hint: every warp of a matvec instruction bumps its counter, attention once
+      // per (lane, kv head); counters only grow within a launch
+      const uint32_t per = I.op == OP_O ? 1u : (uint32_t)kConsumerWarps;
+      if (!wait_hint(p, p.ctr + I.dep, I.dep_target * per * (uint32_t)(t + 1), ii)) misc->stop = 1;
     }
     cbar();
     if (rec) rec[2] = (long long)globaltimer_ns();
-    if (misc->stop) break;
+    if (misc->stop) { stopped = true; break; }
+    float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
     uint32_t used = I.n_units;  // one page per unit, except attention
     switch (I.op) {
       case OP_QKV: {
         const uint16_t* gain = static_cast<const uint16_t*>(I.ptr[3]);
-        if (I.layer == 0) {
-          if (ct < NBT) {
-            int tk = ct < p.nb ? __ldcg(step_tokens + ct) : 0;  // may be written in this launch
-            if (tk < 0 || tk >= D.V) {
-              raise_error(p, E_BAD_TOKEN, ii, (uint32_t)tk, false);
-              tk = 0;
-            }
-            misc->tok[ct] = tk;
-          }
-          cbar();
-          stage<NBT, true, true>(p, act, misc, nullptr, 0, D.H, gain, (int)I.aux0, (int)I.aux1);
-        } else {
-          stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, gain, 0, 0);
-        }
+        if (I.layer == 0)
+          stage<NBT, ST_EMB, true>(p, act, misc, nullptr, 0, D.H, gain, ii);
+        else
+          stage<NBT, ST_SUM, true>(p, act, misc, lay - p.layer_floats + p.off_x1, D.H, D.H, gain, ii);
+        if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_QKV, NBT>(2 * D.RP, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
       }
@@ -1048,33 +1460,52 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
                          : attn_dispatch<128>(p, I, page_base, ring, act, full, empty, misc, ii);
         break;
       case OP_O:
-        stage<NBT, false, false>(p, act, misc, p.o, D.qdim, D.qdim, nullptr, 0, 0);
+        stage<NBT, ST_ONE, false>(p, act, misc, lay + p.off_o, D.qdim, D.qdim, nullptr, ii);
+        if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_O, NBT>(D.Ro, p, I, page_base, ring, act, D.qdim, full, empty, misc, ii);
         break;
       case OP_GU:
-        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), 0, 0);
+        stage<NBT, ST_ONE, true>(p, act, misc, lay + p.off_x1, D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), ii);
+        if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_GU, NBT>(2 * D.Rgu, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
       case OP_DOWN:
-        stage<NBT, false, false>(p, act, misc, p.a + (size_t)I.arg * D.KS, D.F, D.KS, nullptr, 0, 0);
+        stage<NBT, ST_ONE, false>(p, act, misc, lay + p.off_a + (size_t)I.arg * D.KS, D.F, D.KS, nullptr, ii);
+        if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_DOWN, NBT>(D.Rdn, p, I, page_base, ring, act, D.KS, full, empty, misc, ii);
         break;
       case OP_LM:
-        stage<NBT, false, true>(p, act, misc, p.x, D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), 0, 0);
+        stage<NBT, ST_SUM, true>(p, act, misc, lay - p.layer_floats + p.off_x1, D.H, D.H,
+                                 static_cast<const uint16_t*>(I.ptr[3]), ii);
+        if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_LM, NBT>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
     }
     page_base += used;
-    if (rec) rec[3] = (long long)globaltimer_ns();
-    cbar();
-    if (misc->stop) break;
-    // the barrier orders every consumer thread's writes before thread 0's release,
-    // which is cumulative, so one release publishes the whole CTA's results
-    if (ct == 0 && I.sig != kNoCounter) red_release_add(p.ctr + I.sig, 1u);
+    // No barrier here: each warp bumped the hint counter after its own writes,
+    // and the next instruction's barrier keeps the activation buffer from being
+    // restaged while a warp still reads it.  Profiling adds one for its stamps.
+    if (p.prof) {
+      if (rec) rec[3] = (long long)globaltimer_ns();
+      cbar();
+      if (rec) {
+        long long last = 0;
+        for (int w = 0; w < kConsumerWarps; ++w) last = max(last, misc->warp_done[w]);
+        if (I.op != OP_ATTN) rec[12] = last;
+        rec[13] = rec[4] = (long long)globaltimer_ns();
+        if (I.op != OP_ATTN) { rec[18] = misc->t_stage_in; rec[19] = misc->t_stage_loaded; }
+        if (I.op == OP_LM || (I.op == OP_QKV && I.layer > 0)) { rec[20] = misc->t_sum_x1; rec[21] = misc->t_sum_p; }
+        rec[16] += misc->slow_n;
+        rec[17] += (long long)misc->slow_ns;
+        misc->slow_n = 0;
+        misc->slow_ns = 0;
+      }
+    }
     I = In;
-    if (rec) rec[4] = (long long)globaltimer_ns();
   }
-  if (misc->stop) break;
+  if (stopped) break;
+  // a stop raised later in this step is acted on after the next step's barrier,
+  // where every warp reads the flag at the same point
   }
 }
 
@@ -1084,6 +1515,9 @@ template <int NBT>
 __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_constant__ KParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   Misc* misc = reinterpret_cast<Misc*>(smem + p.misc_off);
+  static_assert(sizeof(KParams) % 4 == 0, "KParams copy");
+  for (int i = threadIdx.x; i < (int)(sizeof(KParams) / 4); i += kThreads)
+    reinterpret_cast<uint32_t*>(&misc->kp)[i] = reinterpret_cast<const uint32_t*>(&p)[i];
   // Ring protocol.  Page i (in this SM's stream order) goes to slot i % NP and
   // completes full barrier i % (2 NP), phase parity (i / (2 NP)) & 1; its slot is
   // released on empty barrier i % NP by 8 warp arrivals.  A consumer only waits on
@@ -1105,14 +1539,16 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     misc->last = 0;
     misc->issued = 0;
     misc->entry_abort = aborted(p) ? 1 : 0;
+    misc->slow_n = 0;
+    misc->slow_ns = 0;
   }
   __syncthreads();
   if (!misc->entry_abort) {
     const int warp = threadIdx.x >> 5;
     if (warp == 0) {
-      if (threadIdx.x == 0) producer(p, smem, full, empty, misc);
+      if (threadIdx.x == 0) producer(misc->kp, smem, full, empty, misc);
     } else if (warp <= kConsumerWarps) {
-      consumer<NBT>(p, smem, reinterpret_cast<float*>(smem + p.act_off), full, empty, misc);
+      consumer<NBT>(misc->kp, smem, reinterpret_cast<float*>(smem + p.act_off), full, empty, misc);
     }
   }
   __syncthreads();

@@ -26,9 +26,9 @@ namespace mk {
 enum Op : uint8_t {
   OP_QKV = 1,   // RMSNorm(x) -> rows of Wq|Wk|Wv -> RoPE -> q scratch / K,V cache
   OP_ATTN = 2,  // one slice of a (lane, kv head) over a range of KV pages -> partial; last merges
-  OP_O = 3,     // rows of Wo . o -> x += (red.add)
+  OP_O = 3,     // rows of Wo . o -> x1 = residual + Wo . o
   OP_GU = 4,    // RMSNorm(x) -> rows of Wgate and Wup -> a = silu(g) * u
-  OP_DOWN = 5,  // rows of Wdown over one K slice . a -> x += (red.add)
+  OP_DOWN = 5,  // rows of Wdown over one K slice . a -> that slice's partial of the residual
   OP_LM = 6,    // RMSNorm(x) -> rows of the LM head -> logits, running argmax; last reduces
 };
 
@@ -37,6 +37,8 @@ constexpr int kMaxNB = 8;              // lanes (sequences) per step
 constexpr int kConsumerWarps = 8;      // warps 1..8 compute; warp 0 loads the ring
 constexpr int kThreads = 32 * (1 + kConsumerWarps);
 constexpr int kActFloatsMax = 16384;   // max_batch * K of the staged activation
+constexpr int kMaxKS = 8;              // down-projection K slices (the residual sums them)
+constexpr int kProfSlots = 32;         // int64 fields of one profile record
 constexpr uint16_t kNoCounter = 0xFFFF;
 
 // counters of one layer
@@ -51,7 +53,7 @@ struct Instr {            // 64 bytes
   uint16_t dep;           // counter waited on before the instruction (kNoCounter: none)
   uint16_t sig;           // counter incremented once when the instruction is done
   uint32_t dep_target;    // value `dep` must reach in this step
-  uint32_t aux0, aux1;    // OP_QKV at layer 0: residual rows [aux0, aux1) this SM seeds
+  uint32_t aux0, aux1;    // reserved (zero)
   uint32_t pad;
   // device pointers resolved when the handle is created, so the kernel needs no
   // table lookup per instruction: [0..2] the weight matrices the producer

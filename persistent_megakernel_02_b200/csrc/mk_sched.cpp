@@ -67,7 +67,7 @@ std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, i
   }
   if (!n_ks) return "ffn cannot be split into K slices of at most max(hidden, qdim)";
   D.n_ks = n_ks; D.KS = ffn / n_ks;
-  if (n_ks > 255) return "too many down-projection K slices";
+  if (n_ks > kMaxKS) return "ffn needs more than 8 down-projection K slices";
   // rows per unit: as many as fit a page, but no more than keep every SM busy
   long long pairs = (long long)(n_heads + 2 * n_kv_heads) * (head_dim / 2);
   D.RP = std::min(page_rows(hidden) / 2, pow2_floor(pairs / n_sm));
@@ -170,17 +170,8 @@ Tape lower(const Dims& D, int n_sm, int nb) {
     uint16_t dep_qkv = l ? (uint16_t)ctr_layer(l - 1, C_DOWN) : kNoCounter;
     // RMSNorm + QKV + RoPE
     auto a = as.run(D.n_qkv, unit_bytes(D, OP_QKV, t.S), 0, n_sm);
-    std::vector<int> qkv_sms;
     for (int s = 0; s < n_sm; ++s)
-      if (!a[s].empty()) qkv_sms.push_back(s);
-    for (size_t k = 0; k < qkv_sms.size(); ++k) {
-      int s = qkv_sms[k];
-      Instr& I = emit(s, OP_QKV, l, a[s], dep_qkv, (uint16_t)ctr_layer(l, C_QKV), 0);
-      if (l == 0) {  // these SMs seed the residual with the embedding rows
-        I.aux0 = (uint32_t)((long long)D.H * k / qkv_sms.size());
-        I.aux1 = (uint32_t)((long long)D.H * (k + 1) / qkv_sms.size());
-      }
-    }
+      if (!a[s].empty()) emit(s, OP_QKV, l, a[s], dep_qkv, (uint16_t)ctr_layer(l, C_QKV), 0);
     // attention slices (lane, kv head, slice)
     {
       int n = nb * D.Hkv * t.S;

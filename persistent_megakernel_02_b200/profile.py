@@ -1,7 +1,7 @@
 """Summaries of the per-instruction timestamps the kernel records in profile mode.
 
 Create the handle with ``profile=1``; after a step, ``Megakernel.profile_records()``
-returns int64 [n_sm, stride, 8] records (see ``mk_profile_read`` in include/mk.h).
+returns int64 [n_sm, stride, 32] records (see ``mk_profile_read`` in include/mk.h).
 This module turns them into the time breakdown of one step: per op, how long
 SMs waited on counters, staged activations, computed, and when the last SM of
 each (layer, op) finished -- the critical path through the layer chain.
@@ -29,7 +29,11 @@ def flatten(rec: np.ndarray) -> list[dict]:
             rows.append(dict(sm=s, op=OPS.get(int(r[0]) & 0xFF, "?"), layer=int(r[0] >> 8) & 0xFFFF,
                              units=int(r[0] >> 24), t_start=int(r[1]), t_dep=int(r[2]),
                              t_done=int(r[3]), t_sig=int(r[4]), p_first=int(r[5]), p_last=int(r[6]),
-                             c_wait=int(r[7]), c_pages=int(r[8]), p_wait=int(r[9]), p_pages=int(r[10])))
+                             c_wait=int(r[7]), c_pages=int(r[8]), p_wait=int(r[9]), p_pages=int(r[10]),
+                             t_staged=int(r[11]), t_last_warp=int(r[12]), t_barrier=int(r[13]),
+                             c_core=int(r[14]), c_epi=int(r[15]), slow_n=int(r[16]), slow_ns=int(r[17]),
+                             t_stage_in=int(r[18]), t_stage_loaded=int(r[19]),
+                             t_sum_x1=int(r[20]), t_sum_p=int(r[21])))
     return rows
 
 
@@ -44,9 +48,26 @@ def summarize(rec: np.ndarray) -> dict:
     per_op = {}
     for r in rows:
         d = per_op.setdefault(r["op"], dict(n=0, wait=0, work=0, signal=0, c_wait=0, c_pages=0,
-                                            p_wait=0, p_pages=0))
+                                            p_wait=0, p_pages=0, stage=0, units=0, tail=0, n_mv=0,
+                                            bar=0, rel=0, c_core=0, c_epi=0, slow_n=0, slow_ns=0,
+                                            st_call=0, st_load=0, st_rest=0, n_sum=0, sum_x1=0, sum_p=0))
         d["n"] += 1
-        for k in ("c_wait", "c_pages", "p_wait", "p_pages"):
+        if r["t_staged"] and r["t_last_warp"]:
+            d["n_mv"] += 1
+            d["stage"] += r["t_staged"] - r["t_dep"]          # activation load (+ RMSNorm)
+            d["units"] += r["t_last_warp"] - r["t_staged"]    # pages, matvecs, epilogues
+            d["tail"] += r["t_sig"] - r["t_last_warp"]        # CTA barrier + release
+            d["bar"] += r["t_barrier"] - r["t_last_warp"]     # last warp -> barrier passed
+            d["rel"] += r["t_sig"] - r["t_barrier"]           # the release itself
+            if r["t_stage_in"] and r["t_stage_loaded"]:
+                d["st_call"] += r["t_stage_in"] - r["t_dep"]          # into the staging function
+                d["st_load"] += r["t_stage_loaded"] - r["t_stage_in"]  # activation loads back
+                d["st_rest"] += r["t_staged"] - r["t_stage_loaded"]    # norm, shared-memory stores
+            if r["t_sum_x1"] and r["t_stage_in"]:
+                d["n_sum"] += 1
+                d["sum_x1"] += r["t_sum_x1"] - r["t_stage_in"]     # residual x1 back
+                d["sum_p"] += r["t_sum_p"] - r["t_sum_x1"]         # then the last partial
+        for k in ("c_wait", "c_pages", "p_wait", "p_pages", "c_core", "c_epi", "slow_n", "slow_ns"):
             d[k] += r[k]
         d["wait"] += r["t_dep"] - r["t_start"]
         d["work"] += r["t_done"] - r["t_dep"]
@@ -54,8 +75,17 @@ def summarize(rec: np.ndarray) -> dict:
     for d in per_op.values():
         for k in ("wait", "work", "signal"):
             d[k + "_us_mean"] = d[k] / d["n"] / 1e3
+        for k in ("stage", "units", "tail", "bar", "rel", "st_call", "st_load", "st_rest"):
+            d[k + "_us_mean"] = d[k] / max(1, d["n_mv"]) / 1e3
         d["c_wait_us_per_page"] = d["c_wait"] / max(1, d["c_pages"]) / 1e3
         d["p_wait_us_per_page"] = d["p_wait"] / max(1, d["p_pages"]) / 1e3
+        d["c_core_us_per_page"] = d["c_core"] / max(1, d["c_pages"]) / 1e3
+        d["pages_per_instr_mean"] = d["c_pages"] / max(1, d["n_mv"])
+        d["sum_x1_us_mean"] = d["sum_x1"] / max(1, d["n_sum"]) / 1e3
+        d["sum_p_us_mean"] = d["sum_p"] / max(1, d["n_sum"]) / 1e3
+        d["slow_rereads_per_instr_mean"] = d["slow_n"] / d["n"]
+        d["slow_us_per_reread"] = d["slow_ns"] / max(1, d["slow_n"]) / 1e3
+        d["c_epi_us_per_page"] = d["c_epi"] / max(1, d["c_pages"]) / 1e3
     phases = {}
     for r in rows:
         key = (r["layer"], r["op"])
