@@ -29,8 +29,8 @@ struct mk_ctx {
   std::vector<DevTape> dtapes;
   const uint16_t* embed = nullptr;
   float* acts = nullptr;  // two sets of per-layer activation blocks (see KParams)
-  long long set_floats = 0, layer_floats = 0;
-  int off_q = 0, off_kvn = 0, off_o = 0, off_x1 = 0, off_a = 0, off_p = 0;
+  long long set_floats = 0, layer_floats = 0, acc_base = 0, acc_floats = 0;
+  int off_q = 0, off_kvn = 0, off_o = 0, off_x1 = 0, off_a = 0;
   unsigned long long steps_run = 0;  // decode steps launched (activation-set parity)
   float* part = nullptr;
   int2* lm_part = nullptr;
@@ -67,6 +67,17 @@ mk_status from_cuda(cudaError_t e) {
     mk_status _s = (expr);                         \
     if (_s != MK_OK) return _s;                    \
   } while (0)
+
+// Both activation sets to their empty state: float blocks hold the sentinel
+// (0xFFFFFFFF), accumulators zero.
+mk_status reset_acts(mk_ctx* h) {
+  for (int set = 0; set < 2; ++set) {
+    float* base = h->acts + (size_t)set * h->set_floats;
+    MK_TRY(from_cuda(cudaMemset(base, 0xFF, sizeof(float) * h->acc_base)));
+    MK_TRY(from_cuda(cudaMemset(base + h->acc_base, 0, sizeof(float) * (h->set_floats - h->acc_base))));
+  }
+  return MK_OK;
+}
 
 template <class T>
 mk_status dalloc(mk_ctx* h, T** p, size_t count) {
@@ -178,11 +189,12 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
     h->off_o = (int)off;   off += (long long)MB * D.qdim;
     h->off_x1 = (int)off;  off += (long long)MB * D.H;
     h->off_a = (int)off;   off += (long long)MB * D.F;
-    h->off_p = (int)off;   off += (long long)D.n_ks * MB * D.H;
     h->layer_floats = (off + 7) / 8 * 8;
-    h->set_floats = h->layer_floats * D.L;
+    h->acc_floats = 2LL * MB * D.H;  // 64-bit accumulators
+    h->acc_base = h->layer_floats * D.L;
+    h->set_floats = h->acc_base + h->acc_floats * D.L;
     MK_TRY(dalloc(h, &h->acts, (size_t)2 * h->set_floats));
-    MK_TRY(from_cuda(cudaMemset(h->acts, 0xFF, sizeof(float) * 2 * h->set_floats)));  // the sentinel
+    MK_TRY(reset_acts(h));
   }
   MK_TRY(dalloc(h, &h->part, (size_t)kMaxNB * D.Hkv * S1 * D.rep * (D.d + 2)));
   MK_TRY(dalloc(h, &h->lm_part, (size_t)h->n_sm * kMaxNB));
@@ -250,7 +262,9 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.set_floats = h->set_floats;
   p.layer_floats = h->layer_floats;
   p.off_q = h->off_q; p.off_kvn = h->off_kvn; p.off_o = h->off_o;
-  p.off_x1 = h->off_x1; p.off_a = h->off_a; p.off_p = h->off_p;
+  p.off_x1 = h->off_x1; p.off_a = h->off_a;
+  p.acc_base = h->acc_base;
+  p.acc_floats = h->acc_floats;
   p.parity0 = (int)(h->steps_run & 1);
   p.part = h->part; p.lm_part = h->lm_part;
   p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
@@ -541,7 +555,7 @@ extern "C" mk_status mk_clear_error(mk_handle h) {
   MK_TRY(from_cuda(cudaDeviceSynchronize()));
   MK_TRY(from_cuda(cudaMemset(h->err, 0, sizeof(ErrWord))));
   MK_TRY(from_cuda(cudaMemset(h->counters, 0, sizeof(uint32_t) * 2 * h->n_counters)));
-  // an aborted step may have left written elements behind: every set back to the sentinel
-  MK_TRY(from_cuda(cudaMemset(h->acts, 0xFF, sizeof(float) * 2 * h->set_floats)));
+  // an aborted step may have left written elements behind: every set back to its empty state
+  MK_TRY(reset_acts(h));
   return from_cuda(cudaDeviceSynchronize());
 }

@@ -136,6 +136,38 @@ __device__ __forceinline__ float2 ld_relaxed_f2(const float* p) {
   asm volatile("ld.relaxed.gpu.global.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
   return v;
 }
+// ---- the residual after a down projection: counted fixed-point accumulation ----
+// Element = sum of fixed-point terms (2^-32 units) shifted left by 4, plus one
+// per term in the low 4 bits: red.add of encoded terms is exact and
+// order-free, and a reader knows the element is complete once the count is
+// the number of terms, without any fence.  A term is clamped to +-2^22 so that
+// 16 terms cannot overflow.
+constexpr int kAccCountBits = 4;
+constexpr float kAccScale = 4294967296.0f;  // 2^32
+constexpr float kAccTermLimit = 4194304.0f;  // 2^22
+__device__ __forceinline__ unsigned long long acc_enc(float v) {
+  v = fminf(fmaxf(v, -kAccTermLimit), kAccTermLimit);  // NaN clamps too (to the lower limit)
+  return ((unsigned long long)__float2ll_rn(v * kAccScale) << kAccCountBits) + 1ull;
+}
+__device__ __forceinline__ uint32_t acc_count(unsigned long long a) { return (uint32_t)a & 15u; }
+__device__ __forceinline__ float acc_value(unsigned long long a) {
+  return __ll2float_rn((long long)a >> kAccCountBits) * (1.0f / kAccScale);
+}
+__device__ __forceinline__ void red_acc(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.L2::cache_hint.u64 [%0], %1, %2;" ::"l"(p), "l"(v),
+               "l"(l2_keep_policy())
+               : "memory");
+}
+__device__ __forceinline__ ulonglong2 ld_relaxed_u64x2(const unsigned long long* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p));
+  return v;
+}
 __device__ __forceinline__ float ld_relaxed_f1(const float* p) {
   float v;
   asm volatile("ld.relaxed.gpu.global.f32 %0, [%1];" : "=f"(v) : "l"(p));

@@ -79,19 +79,21 @@ struct KParams {
   int S;  // attention slices per (lane, kv head)
   // the embedding table (layer-0 inputs); all other weights are named by the instructions
   const uint16_t* embed;
-  // Activations: two sets (by decode-step parity) of L layer blocks of
-  // layer_floats floats.  Inside a block, with MB = max_batch lanes:
+  // Activations: two sets (by decode-step parity), each L layer blocks of
+  // layer_floats floats followed by L accumulators of acc_floats floats.  Inside
+  // a block, with MB = max_batch lanes:
   //   off_q   [MB][qdim]      rotated queries
   //   off_kvn [MB][2][kvdim]  this step's K and V rows (fp32, before caching)
   //   off_o   [MB][qdim]      attention output
   //   off_x1  [MB][H]         residual after the O projection
   //   off_a   [MB][F]         silu(gate) * up
-  //   off_p   [n_ks][MB][H]   down projection, one partial per K slice
-  // The residual after the down projection is x1 + P_0 + ... + P_{n_ks-1},
-  // summed in that order wherever it is read.
+  // and the accumulator of layer l, [MB][H] 64-bit counted fixed-point sums
+  // (acc_enc), holds the residual after its down projection: x1 plus every K
+  // slice's partial, 1 + n_ks terms.  Float blocks refill with the sentinel,
+  // accumulators with zero.
   float* acts;
-  long long set_floats, layer_floats;
-  int off_q, off_kvn, off_o, off_x1, off_a, off_p;
+  long long set_floats, layer_floats, acc_base, acc_floats;
+  int off_q, off_kvn, off_o, off_x1, off_a;
   int parity0;  // set of this launch's step 0
   float* part;  // attention partials [8][Hkv][S][rep][d + 2]
   int2* lm_part;  // [n_sm][8] best (value bits, index) per SM
@@ -136,11 +138,14 @@ struct Misc {
   int lmi[kConsumerWarps][kMaxNB];
   int tok[kMaxNB];
   long long warp_done[kConsumerWarps];  // profile mode: when each warp finished its units
+  long long warp_entry[kConsumerWarps];  // profile mode: when each warp entered its matvec
+  long long warp_first[kConsumerWarps];  // profile mode: when each warp had its first page
   int pos[kMaxNB];       // each lane's position in the current step
   int step;              // the current step of this launch
   int cur_phys[kMaxNB];  // physical KV page holding each lane's position this step
   float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
   float* actset;         // the activation set of the current step
+  uint32_t i0;           // this SM's first tape index (profile records)
   unsigned int slow_n;   // profile mode: group re-reads of unwritten activations
   unsigned long long slow_ns;  // and the time they took (summed over threads)
   long long t_stage_in, t_stage_loaded;  // profile mode: stage entry, thread 0's loads back
@@ -512,38 +517,32 @@ __device__ __noinline__ Chunk8<NBT> stage_one_slow(const KParams& p, const float
   for (int b = 0; b < NBT; ++b) r.l[b] = r.h[b] = make_float4(0.f, 0.f, 0.f, 0.f);
   return r;
 }
-// one 8-element chunk of x1 + P_0 + ... + P_{n_ks-1} (same order of additions)
-__device__ __noinline__ Chunk8<1> resid_chunk_slow(const KParams& p, const float* xs, const float* P0,
-                                                   size_t mbh, size_t off, uint32_t ii, Misc* misc) {
-  Chunk8<1> out;
+// one 8-element chunk of each lane's residual accumulator, until all 1 + n_ks terms are in
+template <int NBT>
+__device__ __noinline__ Chunk8<NBT> acc_chunk_slow(const KParams& p, const unsigned long long* src, int ld,
+                                                   uint32_t ii, Misc* misc) {
+  Chunk8<NBT> r;
+  const uint32_t want = 1u + (uint32_t)p.D.n_ks;
   Spin sp(p, misc);
   do {
-    float4 l = ld_relaxed_f4(xs), h = ld_relaxed_f4(xs + 4);
-    float4 pl[kMaxKS], ph[kMaxKS];
+    bool bad = false;
 #pragma unroll
-    for (int s = 0; s < kMaxKS; ++s)
-      if (s < p.D.n_ks) {
-        pl[s] = ld_relaxed_f4(P0 + s * mbh + off);
-        ph[s] = ld_relaxed_f4(P0 + s * mbh + off + 4);
-      }
-    bool bad = any_sent(l) | any_sent(h);
-#pragma unroll
-    for (int s = 0; s < kMaxKS; ++s)
-      if (s < p.D.n_ks) bad |= any_sent(pl[s]) | any_sent(ph[s]);
-    if (!bad) {
-#pragma unroll
-      for (int s = 0; s < kMaxKS; ++s)
-        if (s < p.D.n_ks) {
-          l.x += pl[s].x; l.y += pl[s].y; l.z += pl[s].z; l.w += pl[s].w;
-          h.x += ph[s].x; h.y += ph[s].y; h.z += ph[s].z; h.w += ph[s].w;
-        }
-      out.l[0] = l;
-      out.h[0] = h;
-      return out;
+    for (int b = 0; b < NBT; ++b) {
+      r.l[b] = r.h[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (b >= p.nb) continue;
+      const ulonglong2 e0 = ld_relaxed_u64x2(src + (size_t)b * ld), e1 = ld_relaxed_u64x2(src + (size_t)b * ld + 2);
+      const ulonglong2 e2 = ld_relaxed_u64x2(src + (size_t)b * ld + 4), e3 = ld_relaxed_u64x2(src + (size_t)b * ld + 6);
+      bad |= (acc_count(e0.x) != want) | (acc_count(e0.y) != want) | (acc_count(e1.x) != want) |
+             (acc_count(e1.y) != want) | (acc_count(e2.x) != want) | (acc_count(e2.y) != want) |
+             (acc_count(e3.x) != want) | (acc_count(e3.y) != want);
+      r.l[b] = make_float4(acc_value(e0.x), acc_value(e0.y), acc_value(e1.x), acc_value(e1.y));
+      r.h[b] = make_float4(acc_value(e2.x), acc_value(e2.y), acc_value(e3.x), acc_value(e3.y));
     }
+    if (!bad) return r;
   } while (sp.again(p, ii, 9, misc));
-  out.l[0] = out.h[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-  return out;
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) r.l[b] = r.h[b] = make_float4(0.f, 0.f, 0.f, 0.f);
+  return r;
 }
 
 // Stage NBT activation rows of length K into shared memory in the split layout
@@ -551,12 +550,12 @@ __device__ __noinline__ Chunk8<1> resid_chunk_slow(const KParams& p, const float
 // 8c+4..8c+7 at hi[b*nch + c]).  Sources (MODE):
 //   ST_EMB  the bf16 embedding rows of the lanes' tokens (layer 0);
 //   ST_ONE  one fp32 vector per lane at src + b * ld;
-//   ST_SUM  the residual after a down projection: x1 at src + b * H plus the
-//           layer's n_ks partials, added in slice order.
-// fp32 sources are this step's activations: every element is validated against
-// the sentinel (and re-read until written).  NORM applies RMSNorm with the bf16
-// gain.  Lanes >= nb are zero.
-enum { ST_EMB = 0, ST_ONE = 1, ST_SUM = 2 };
+//   ST_ACC  the residual after a down projection: the layer's accumulator at
+//           src (64-bit elements, lane stride ld).
+// The other sources are this step's activations: every element is validated
+// (sentinel, or the accumulator's term count) and re-read until written.  NORM
+// applies RMSNorm with the bf16 gain.  Lanes >= nb are zero.
+enum { ST_EMB = 0, ST_ONE = 1, ST_ACC = 2 };
 
 template <int NBT, int MODE, bool NORM>
 __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, const float* src, int ld,
@@ -606,47 +605,30 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
 #pragma unroll
         for (int b = 0; b < NBT; ++b) { vl[b] = r.l[b]; vh[b] = r.h[b]; }
       }
-    } else {
-      const size_t mbh = (size_t)p.D.max_batch * p.D.H;
-      const float* P0 = src + (p.off_p - p.off_x1);
-      const int nks = p.D.n_ks;
+    } else {  // ST_ACC: src is the accumulator array
+      const unsigned long long* A = reinterpret_cast<const unsigned long long*>(src) + c * 8;
+      const uint32_t want = 1u + (uint32_t)p.D.n_ks;
+      bool bad = false;
 #pragma unroll
       for (int b = 0; b < NBT; ++b) {
         vl[b] = vh[b] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (b >= p.nb) continue;
-        const float* xs = src + (size_t)b * p.D.H + c * 8;
-        float4 l0 = ld_relaxed_f4(xs), h0 = ld_relaxed_f4(xs + 4);
-        float4 pl[kMaxKS], ph[kMaxKS];
+        const ulonglong2 e0 = ld_relaxed_u64x2(A + (size_t)b * ld), e1 = ld_relaxed_u64x2(A + (size_t)b * ld + 2);
+        const ulonglong2 e2 = ld_relaxed_u64x2(A + (size_t)b * ld + 4), e3 = ld_relaxed_u64x2(A + (size_t)b * ld + 6);
+        bad |= (acc_count(e0.x) != want) | (acc_count(e0.y) != want) | (acc_count(e1.x) != want) |
+               (acc_count(e1.y) != want) | (acc_count(e2.x) != want) | (acc_count(e2.y) != want) |
+               (acc_count(e3.x) != want) | (acc_count(e3.y) != want);
+        vl[b] = make_float4(acc_value(e0.x), acc_value(e0.y), acc_value(e1.x), acc_value(e1.y));
+        vh[b] = make_float4(acc_value(e2.x), acc_value(e2.y), acc_value(e3.x), acc_value(e3.y));
+      }
+      if (p.prof && ct == 0) {  // when the accumulator came back (profile only)
+        misc->t_sum_x1 = (long long)globaltimer_ns() + (bad ? 1 : 0);
+        misc->t_sum_p = misc->t_sum_x1;
+      }
+      if (bad) {
+        const Chunk8<NBT> r = acc_chunk_slow<NBT>(p, A, ld, ii, misc);
 #pragma unroll
-        for (int s = 0; s < kMaxKS; ++s)
-          if (s < nks) {
-            pl[s] = ld_relaxed_f4(P0 + s * mbh + (size_t)b * p.D.H + c * 8);
-            ph[s] = ld_relaxed_f4(P0 + s * mbh + (size_t)b * p.D.H + c * 8 + 4);
-          }
-        if (p.prof && ct == 0 && b == 0) {  // which source comes back last (profile only)
-          if (__float_as_uint(l0.x) == 0x7FC00001u) misc->slow_n += 0u;
-          misc->t_sum_x1 = (long long)globaltimer_ns();
-          if (__float_as_uint(pl[nks - 1].x) == 0x7FC00001u) misc->slow_n += 0u;
-          misc->t_sum_p = (long long)globaltimer_ns();
-        }
-        bool bad = any_sent(l0) | any_sent(h0);
-#pragma unroll
-        for (int s = 0; s < kMaxKS; ++s)
-          if (s < nks) bad |= any_sent(pl[s]) | any_sent(ph[s]);
-        if (bad) {  // rare: some element not yet visible; re-read the chunk element by element
-          const Chunk8<1> r = resid_chunk_slow(p, xs, P0, mbh, (size_t)b * p.D.H + c * 8, ii, misc);
-          l0 = r.l[0];
-          h0 = r.h[0];
-        } else {
-#pragma unroll
-          for (int s = 0; s < kMaxKS; ++s)
-            if (s < nks) {
-              l0.x += pl[s].x; l0.y += pl[s].y; l0.z += pl[s].z; l0.w += pl[s].w;
-              h0.x += ph[s].x; h0.y += ph[s].y; h0.z += ph[s].z; h0.w += ph[s].w;
-            }
-        }
-        vl[b] = l0;
-        vh[b] = h0;
+        for (int b = 0; b < NBT; ++b) { vl[b] = r.l[b]; vh[b] = r.h[b]; }
       }
     }
     if (p.prof && ct == 0 && c == 0) {  // the branch waits for the loaded value, then the clock is read
@@ -675,26 +657,8 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
       for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
       if (lane == 0) misc->red[cw][b] = t;
     }
-    cbar();
-    float rinv[NBT];
-#pragma unroll
-    for (int b = 0; b < NBT; ++b) {
-      float t = 0.f;
-#pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) t += misc->red[w][b];
-      rinv[b] = 1.0f / sqrtf(t / (float)K + p.D.eps);
-    }
-    for (int c = ct; c < nch; c += 256) {
-#pragma unroll
-      for (int b = 0; b < NBT; ++b) {
-        float4 l4 = lo[b * nch + c], h4 = hi[b * nch + c];
-        const float r = rinv[b];
-        l4.x *= r; l4.y *= r; l4.z *= r; l4.w *= r;
-        h4.x *= r; h4.y *= r; h4.z *= r; h4.w *= r;
-        lo[b * nch + c] = l4;
-        hi[b * nch + c] = h4;
-      }
-    }
+    // the 1/rms scale is applied to the matvec outputs (norm_scales), which is
+    // the same linear map and saves a pass over the staged vector
   }
   cbar();
 }
@@ -784,92 +748,174 @@ __device__ __forceinline__ int rs_base(int n, int keep, int lane) {
 }
 
 // The residual entering layer `layer` at (lane b, row): the embedding for
-// layer 0, else the previous layer's x1 + P_0 + ... + P_{n_ks-1} (the order the
-// stage adds them in, so both see the same fp32 value).  The loads are issued
-// here; resid_finish validates and adds them once the caller needs the value.
+// layer 0, else the previous layer's accumulator.  The load is issued here;
+// resid_finish validates it (all 1 + n_ks terms in) once the value is needed.
 struct ResidIn {
-  float x, pp[kMaxKS];
-  const float* src;
+  unsigned long long acc;
+  const unsigned long long* src;  // null: layer 0, the value is in emb
+  float emb;
 };
+__device__ __forceinline__ const unsigned long long* acc_of(const KParams& p, const Misc* misc, int layer) {
+  return reinterpret_cast<const unsigned long long*>(misc->actset + p.acc_base + (size_t)layer * p.acc_floats);
+}
 __device__ __forceinline__ void resid_issue(const KParams& p, const Misc* misc, int layer, int b, int row,
                                             ResidIn& r) {
   if (layer == 0) {
     r.src = nullptr;
-    r.x = __uint_as_float((uint32_t)p.embed[(size_t)misc->tok[b] * p.D.H + row] << 16);
+    r.emb = __uint_as_float((uint32_t)p.embed[(size_t)misc->tok[b] * p.D.H + row] << 16);
     return;
   }
-  const float* prev = misc->actset + (size_t)(layer - 1) * p.layer_floats;
-  r.src = prev + p.off_x1 + (size_t)b * p.D.H + row;
-  r.x = ld_relaxed_f1(r.src);
-  const size_t mbh = (size_t)p.D.max_batch * p.D.H;
-#pragma unroll
-  for (int s = 0; s < kMaxKS; ++s)
-    if (s < p.D.n_ks) r.pp[s] = ld_relaxed_f1(prev + p.off_p + s * mbh + (size_t)b * p.D.H + row);
+  r.src = acc_of(p, misc, layer - 1) + (size_t)b * p.D.H + row;
+  r.acc = ld_relaxed_u64(r.src);
 }
-__device__ __noinline__ ResidIn resid_slow(const KParams& p, Misc* misc, ResidIn r, uint32_t ii) {
-  const size_t mbh = (size_t)p.D.max_batch * p.D.H;
-  const float* P0 = r.src + (p.off_p - p.off_x1);
+__device__ __noinline__ unsigned long long resid_slow(const KParams& p, Misc* misc, const unsigned long long* src,
+                                                      uint32_t ii) {
+  const uint32_t want = 1u + (uint32_t)p.D.n_ks;
   Spin sp(p, misc);
   do {
-    r.x = ld_relaxed_f1(r.src);
-#pragma unroll
-    for (int s = 0; s < kMaxKS; ++s)
-      if (s < p.D.n_ks) r.pp[s] = ld_relaxed_f1(P0 + s * mbh);
-    bool bad = is_sent(r.x);
-#pragma unroll
-    for (int s = 0; s < kMaxKS; ++s)
-      if (s < p.D.n_ks) bad |= is_sent(r.pp[s]);
-    if (!bad) return r;
+    const unsigned long long a = ld_relaxed_u64(src);
+    if (acc_count(a) == want) return a;
   } while (sp.again(p, ii, 10, misc));
-  r.x = 0.f;
-#pragma unroll
-  for (int s = 0; s < kMaxKS; ++s) r.pp[s] = 0.f;
-  return r;
+  return 0ull;
 }
 __device__ __forceinline__ float resid_finish(const KParams& p, Misc* misc, ResidIn& r, uint32_t ii) {
-  if (!r.src) return r.x;
-  bool bad = is_sent(r.x);
-#pragma unroll
-  for (int s = 0; s < kMaxKS; ++s)
-    if (s < p.D.n_ks) bad |= is_sent(r.pp[s]);
-  if (bad) r = resid_slow(p, misc, r, ii);
-  float x = r.x;
-#pragma unroll
-  for (int s = 0; s < kMaxKS; ++s)
-    if (s < p.D.n_ks) x += r.pp[s];
-  return x;
+  if (!r.src) return r.emb;
+  if (acc_count(r.acc) != 1u + (uint32_t)p.D.n_ks) r.acc = resid_slow(p, misc, r.src, ii);
+  return acc_value(r.acc);
 }
 
 __device__ __forceinline__ bool lm_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+// 1 / rms of each lane's staged vector (RMSNorm), from the per-warp sums of
+// squares the stage left in misc->red.
+template <int NBT>
+__device__ __forceinline__ void norm_scales(const KParams& p, const Misc* misc, int K, float (&rinv)[NBT]) {
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) {
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) t += misc->red[w][b];
+    rinv[b] = 1.0f / sqrtf(t / (float)K + p.D.eps);
+  }
+}
+template <int NBT>
+__device__ __forceinline__ float pick(const float (&v)[NBT], int b) {
+  float r = v[0];
+#pragma unroll
+  for (int i = 1; i < NBT; ++i)
+    if (i == b) r = v[i];
+  return r;
+}
+
+// End of the LM-head instruction: combine the lanes' and warps' running argmax,
+// publish this SM's best per lane; the last SM to arrive reduces all of them
+// into the greedy ids and releases the step counter.
+template <int NBT>
+struct LmBest {  // running argmax per lane (value, index); passed by value, so it stays in registers
+  float v[NBT];
+  int i[NBT];
+};
+template <int NBT>
+__device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBest<NBT> best) {
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) {
+    float bv = best.v[b];
+    int bi = best.i[b];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+      if (lm_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    if (lane == 0) { misc->lmv[cw][b] = bv; misc->lmi[cw][b] = bi; }
+  }
+  cbar();
+  if (ct < NBT) {
+    float bv = -CUDART_INF_F;
+    int bi = 0x7FFFFFFF;
+    for (int w = 0; w < kConsumerWarps; ++w)
+      if (lm_better(misc->lmv[w][ct], misc->lmi[w][ct], bv, bi)) { bv = misc->lmv[w][ct]; bi = misc->lmi[w][ct]; }
+    p.lm_part[blockIdx.x * kMaxNB + ct] = make_int2(__float_as_int(bv), bi);
+  }
+  cbar();
+  if (ct == 0) {
+    const uint32_t old = atom_acq_rel_add(p.ctr + ctr_lm(D), 1u);
+    misc->last = (old == gridDim.x - 1) && !misc->stop;
+  }
+  cbar();
+  if (misc->last) {
+    if (ct < p.nb) {
+      float bv = -CUDART_INF_F;
+      int bi = 0x7FFFFFFF;
+      for (int s = 0; s < (int)gridDim.x; ++s) {
+        const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
+        const float val = __int_as_float(e.x);
+        if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
+      }
+      p.ids[(size_t)misc->step * p.ids_stride + ct] = (bi >= 0 && bi < D.V) ? bi : 0;
+    }
+    cbar();
+    if (ct == 0) {
+      p.ctr[ctr_lm(D)] = 0u;                     // the next step's arrivals count from zero
+      red_release_add(p.ctr + ctr_step(D), 1u);  // this step's ids are written
+    }
+  }
+}
+
 // Warp-per-page matvec over this instruction's units, then the op's epilogue.
+// For QKV and GU the reduce-scatter keeps value pairs (rows j and j + RT/2 of a
+// unit, same lane) in one lane: a RoPE pair for QKV, (gate, up) for GU; the
+// other ops keep single values.
 template <int OPK, int RT, int NBT>
 __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t page_base,
                                       uint8_t* ring, const float* act, int K, uint64_t* full,
                                       uint64_t* empty, Misc* misc, uint32_t ii) {
   const Dims& D = p.D;
+  constexpr int op = OPK;
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const uint32_t NP = (uint32_t)p.ring_pages;
   const int nch = K >> 3;
   const uint32_t alo = smem_u32(act);
   const uint32_t ahi = alo + (uint32_t)(NBT * nch) * 16u;
-  constexpr bool PAIRED = (OPK == OP_QKV || OPK == OP_GU);
-  constexpr int P = PAIRED ? RT / 2 : RT;  // output rows of a unit
+  constexpr bool PL2 = OPK == OP_QKV || OPK == OP_GU;  // paired layout (RT >= 2 for these ops)
+  constexpr int P = PL2 ? RT / 2 : 1;  // rows between the two values of a pair
   constexpr int NV = RT * NBT;
-  constexpr int KEEP = PAIRED ? 2 : 1;
+  constexpr int KEEP = PL2 ? 2 : 1;
   constexpr int NL = rs_left(NV, KEEP);
   const int vbase = rs_base(NV, KEEP, lane);
   const bool writer = (lane & rs_dup_mask(NV, KEEP)) == 0;
-  float bestv[NBT];
-  int besti[NBT];
+  // value m of this lane after the reduction: unit row vrow[m], lane vlane[m]
+  int vrow[NL], vlane[NL];
 #pragma unroll
-  for (int b = 0; b < NBT; ++b) { bestv[b] = -CUDART_INF_F; besti[b] = 0x7FFFFFFF; }
-  long long* prec = p.prof
-                        ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - p.sm_off[blockIdx.x])) * kProfSlots
-                        : nullptr;
+  for (int m = 0; m < NL; ++m) {
+    if (PL2) {
+      const int pi = vbase / 2 + m / 2;
+      vrow[m] = pi / NBT + (m & 1) * P;
+      vlane[m] = pi % NBT;
+    } else {
+      vrow[m] = (vbase + m) / NBT;
+      vlane[m] = (vbase + m) % NBT;
+    }
+  }
+  LmBest<NBT> best;
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) { best.v[b] = -CUDART_INF_F; best.i[b] = 0x7FFFFFFF; }
+  long long* prec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - misc->i0)) * kProfSlots : nullptr;
+  if (p.prof && lane == 0) { misc->warp_entry[cw] = (long long)globaltimer_ns(); misc->warp_first[cw] = 0; }
   float* lay = misc->actset + (size_t)I.layer * p.layer_floats;  // this layer's activation block
+  // RMSNorm ops: the 1/rms scale of every value this lane holds after the reduction
+  constexpr bool normed = op == OP_QKV || op == OP_GU || op == OP_LM;
+  float osc[NL];
+  if constexpr (normed) {
+    float rinv[NBT];
+    norm_scales<NBT>(p, misc, K, rinv);
+#pragma unroll
+    for (int m = 0; m < NL; ++m) osc[m] = pick<NBT>(rinv, vlane[m]);
+  }
   long long c_wait = 0, c_pages = 0, c_core = 0, c_epi = 0;
   // this step's logits (LM head only)
   float* lg = nullptr;
@@ -877,6 +923,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
     if (!p.logits_last) lg = p.logits + (size_t)misc->step * p.nb * D.V;
     else if (misc->step == p.n_steps - 1) lg = p.logits;
   }
+  unsigned long long* accl = (OPK == OP_O || OPK == OP_DOWN) ? const_cast<unsigned long long*>(acc_of(p, misc, I.layer)) : nullptr;
 
   RingPos rp;
   rp.init(page_base + cw, NP);
@@ -887,14 +934,17 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
     if constexpr (OPK == OP_O) {  // the residual rows this lane will write, loaded under the page wait
       const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
 #pragma unroll
-      for (int m = 0; m < NL; ++m) {
-        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
-        if (writer && r < nr && b < p.nb) resid_issue(p, misc, I.layer, b, r0 + r, rin[m]);
-      }
+      for (int m = 0; m < NL; ++m)
+        if (writer && vrow[m] < nr && vlane[m] < p.nb) resid_issue(p, misc, I.layer, vlane[m], r0 + vrow[m], rin[m]);
     }
     const long long tw = prec ? (long long)globaltimer_ns() : 0;
     bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
-    if (prec) { c_wait += (long long)globaltimer_ns() - tw; c_pages += 1; }
+    if (prec) {
+      const long long now = (long long)globaltimer_ns();
+      c_wait += now - tw;
+      c_pages += 1;
+      if (lane == 0 && misc->warp_first[cw] == 0) misc->warp_first[cw] = now;
+    }
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) misc->stop = 1;
       break;
@@ -912,7 +962,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
     if (prec) c_core += te - tc;
 
     float v[NV];
-    if constexpr (PAIRED) {
+    if constexpr (PL2) {
 #pragma unroll
       for (int j = 0; j < P; ++j)
 #pragma unroll
@@ -926,75 +976,85 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
         for (int b = 0; b < NBT; ++b) v[r * NBT + b] = acc[r][b].x + acc[r][b].y;
     }
     warp_rs<NV, NV, KEEP, 16>(v, lane);
+    if constexpr (normed) {
+#pragma unroll
+      for (int m = 0; m < NL; ++m) v[m] *= osc[m];
+    }
 
     if constexpr (OPK == OP_QKV) {
-      const int half = D.d / 2;
-      const int P0 = (int)u * P, hg = P0 / half, i0 = P0 % half;
-      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
-      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+      if constexpr (PL2) {
+        const int half = D.d / 2;
+        const int P0 = (int)u * P, hg = P0 / half, i0 = P0 % half;
+        const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
+        const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
 #pragma unroll
-      for (int m = 0; m < NL / 2; ++m) {
-        const int pi = vbase / 2 + m, j = pi / NBT, b = pi % NBT;
-        if (!writer || b >= p.nb) continue;
-        const float v1 = v[2 * m], v2 = v[2 * m + 1];
-        const int i = i0 + j, pos = misc->pos[b];
-        float r1 = v1, r2 = v2;
-        if (sec < 2) {
-          const float2 cs = misc->rope_cs[b][i];
-          r1 = v1 * cs.x - v2 * cs.y;
-          r2 = v2 * cs.x + v1 * cs.y;
-        }
-        if (sec == 0) {
-          float* qq = lay + p.off_q + (size_t)b * D.qdim + hh * D.d;
-          st_relaxed_f32(qq + i, canon(r1));
-          st_relaxed_f32(qq + i + half, canon(r2));
-        } else {
-          // the cache row serves later steps; this step's attention reads the fp32 copy
-          const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
-                                 (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
-          uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
-          cache[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
-          cache[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
-          float* kv = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + (sec - 1) * D.kvdim + hh * D.d;
-          st_relaxed_f32(kv + i, canon(r1));
-          st_relaxed_f32(kv + i + half, canon(r2));
+        for (int m = 0; m < NL; m += 2) {
+          const int b = vlane[m];
+          if (!writer || b >= p.nb) continue;
+          const float v1 = v[m], v2 = v[m + 1];
+          const int i = i0 + vrow[m], pos = misc->pos[b];
+          float r1 = v1, r2 = v2;
+          if (sec < 2) {
+            const float2 cs = misc->rope_cs[b][i];
+            r1 = v1 * cs.x - v2 * cs.y;
+            r2 = v2 * cs.x + v1 * cs.y;
+          }
+          if (sec == 0) {
+            float* qq = lay + p.off_q + (size_t)b * D.qdim + hh * D.d;
+            st_relaxed_f32(qq + i, canon(r1));
+            st_relaxed_f32(qq + i + half, canon(r2));
+          } else {
+            // the cache row serves later steps; this step's attention reads the fp32 copy
+            const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
+                                   (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
+            uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
+            cache[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
+            cache[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
+            float* kv = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + (sec - 1) * D.kvdim + hh * D.d;
+            st_relaxed_f32(kv + i, canon(r1));
+            st_relaxed_f32(kv + i + half, canon(r2));
+          }
         }
       }
     } else if constexpr (OPK == OP_GU) {
-      const int r0 = (int)u * P, nr = min(P, D.F - r0);
+      if constexpr (PL2) {
+        const int r0 = (int)u * P, nr = min(P, D.F - r0);
 #pragma unroll
-      for (int m = 0; m < NL / 2; ++m) {
-        const int pi = vbase / 2 + m, r = pi / NBT, b = pi % NBT;
-        if (!writer || r >= nr || b >= p.nb) continue;
-        const float g = v[2 * m], up = v[2 * m + 1];
-        st_relaxed_f32(lay + p.off_a + (size_t)b * D.F + r0 + r, canon(g / (1.0f + __expf(-g)) * up));
+        for (int m = 0; m < NL; m += 2) {
+          const int r = vrow[m], b = vlane[m];
+          if (!writer || r >= nr || b >= p.nb) continue;
+          const float g = v[m], up = v[m + 1];
+          st_relaxed_f32(lay + p.off_a + (size_t)b * D.F + r0 + r, canon(g / (1.0f + __expf(-g)) * up));
+        }
       }
-    } else if constexpr (OPK == OP_O) {  // x1 = residual + Wo . o
+    } else if constexpr (OPK == OP_O) {  // x1 = residual + Wo . o, and x1 is the layer accumulator's first term
       const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
 #pragma unroll
       for (int m = 0; m < NL; ++m) {
-        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
-        if (writer && r < nr && b < p.nb)
-          st_relaxed_f32(lay + p.off_x1 + (size_t)b * D.H + r0 + r,
-                         canon(resid_finish(p, misc, rin[m], ii) + v[m]));
+        const int r = vrow[m], b = vlane[m];
+        if (writer && r < nr && b < p.nb) {
+          const float x1 = canon(resid_finish(p, misc, rin[m], ii) + v[m]);
+          st_relaxed_f32(lay + p.off_x1 + (size_t)b * D.H + r0 + r, x1);
+          red_acc(accl + (size_t)b * D.H + r0 + r, acc_enc(x1));
+        }
       }
-    } else if constexpr (OPK == OP_DOWN) {  // this K slice's partial of Wd . a
+    } else if constexpr (OPK == OP_DOWN) {  // this K slice's term of the layer's residual
       const int r0 = (int)u * RT, nr = min(RT, D.H - r0);
-      float* P = lay + p.off_p + (size_t)I.arg * D.max_batch * D.H;
 #pragma unroll
       for (int m = 0; m < NL; ++m) {
-        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
-        if (writer && r < nr && b < p.nb) st_relaxed_f32(P + (size_t)b * D.H + r0 + r, canon(v[m]));
+        const int r = vrow[m], b = vlane[m];
+        if (writer && r < nr && b < p.nb) red_acc(accl + (size_t)b * D.H + r0 + r, acc_enc(v[m]));
       }
-    } else if constexpr (OPK == OP_LM) {
+    } else {  // OP_LM
+      static_assert(OPK == OP_LM, "matvec op");
       const int r0 = (int)u * RT, nr = min(RT, D.V - r0);
 #pragma unroll
       for (int m = 0; m < NL; ++m) {
-        const int idx = vbase + m, r = idx / NBT, b = idx % NBT;
+        const int r = vrow[m], b = vlane[m];
         if (r >= nr || b >= p.nb) continue;
 #pragma unroll
         for (int bb = 0; bb < NBT; ++bb)
-          if (bb == b && lm_better(v[m], r0 + r, bestv[bb], besti[bb])) { bestv[bb] = v[m]; besti[bb] = r0 + r; }
+          if (bb == b && lm_better(v[m], r0 + r, best.v[bb], best.i[bb])) { best.v[bb] = v[m]; best.i[bb] = r0 + r; }
         if (writer && lg) lg[(size_t)b * D.V + r0 + r] = v[m];
       }
     }
@@ -1012,52 +1072,7 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
   // this warp's share is written: bump the hint counter (every warp, pages or not)
   __syncwarp();
   if (lane == 0 && I.sig != kNoCounter) red_relaxed_add(p.ctr + I.sig, 1u);
-  if constexpr (OPK == OP_LM) {
-    // combine the lanes' and warps' running argmax, publish this SM's, the last SM reduces
-#pragma unroll
-    for (int b = 0; b < NBT; ++b) {
-      float bv = bestv[b];
-      int bi = besti[b];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
-        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-        if (lm_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
-      if (lane == 0) { misc->lmv[cw][b] = bv; misc->lmi[cw][b] = bi; }
-    }
-    cbar();
-    if (ct < NBT) {
-      float bv = -CUDART_INF_F;
-      int bi = 0x7FFFFFFF;
-      for (int w = 0; w < kConsumerWarps; ++w)
-        if (lm_better(misc->lmv[w][ct], misc->lmi[w][ct], bv, bi)) { bv = misc->lmv[w][ct]; bi = misc->lmi[w][ct]; }
-      p.lm_part[blockIdx.x * kMaxNB + ct] = make_int2(__float_as_int(bv), bi);
-    }
-    cbar();
-    if (ct == 0) {
-      const uint32_t old = atom_acq_rel_add(p.ctr + ctr_lm(D), 1u);
-      misc->last = (old == gridDim.x - 1) && !misc->stop;
-    }
-    cbar();
-    if (misc->last) {
-      if (ct < p.nb) {
-        float bv = -CUDART_INF_F;
-        int bi = 0x7FFFFFFF;
-        for (int s = 0; s < (int)gridDim.x; ++s) {
-          const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
-          const float val = __int_as_float(e.x);
-          if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
-        }
-        p.ids[(size_t)misc->step * p.ids_stride + ct] = (bi >= 0 && bi < D.V) ? bi : 0;
-      }
-      cbar();
-      if (ct == 0) {
-        p.ctr[ctr_lm(D)] = 0u;                  // the next step's arrivals count from zero
-        red_release_add(p.ctr + ctr_step(D), 1u);  // this step's ids are written
-      }
-    }
-  }
+  if constexpr (OPK == OP_LM) lm_finish<NBT>(p, misc, best);
 }
 
 // ---------------------------------------------------------------- consumers: attention
@@ -1347,7 +1362,7 @@ __device__ __forceinline__ void mv_dispatch(int rt, const KParams& p, const Inst
                                             uint8_t* ring, const float* act, int K, uint64_t* full,
                                             uint64_t* empty, Misc* misc, uint32_t ii) {
   switch (rt) {
-    case 1: if constexpr (OPK != OP_QKV && OPK != OP_GU) mv_units<OPK, 1, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 1: if constexpr (OPK == OP_O || OPK == OP_DOWN || OPK == OP_LM) mv_units<OPK, 1, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
     case 2: mv_units<OPK, 2, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
     case 4: mv_units<OPK, 4, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
     case 8: mv_units<OPK, 8, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
@@ -1386,6 +1401,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   // tokens, every read of its activations and every write of its KV rows are done
   if (ct == 0) {
     misc->step = t;
+    misc->i0 = i0;
     misc->actset = p.acts + (size_t)((p.parity0 + t) & 1) * p.set_floats;
     if (t > 0 && !wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, i0)) misc->stop = 1;
   }
@@ -1411,12 +1427,12 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     const int b = e / half, i = e % half;
     misc->rope_cs[b][i] = p.rope[(size_t)(p.pos[b] + t) * half + i];
   }
-  {  // refill this SM's share of the other activation set with the sentinel
+  {  // refill this SM's share of the other activation set: sentinel, accumulators zero
     uint4* other = reinterpret_cast<uint4*>(p.acts + (size_t)((p.parity0 + t + 1) & 1) * p.set_floats);
-    const long long n4 = p.set_floats / 4, per = (n4 + gridDim.x - 1) / gridDim.x;
+    const long long n4 = p.set_floats / 4, per = (n4 + gridDim.x - 1) / gridDim.x, acc4 = p.acc_base / 4;
     const long long lo = (long long)blockIdx.x * per, hi = min(n4, lo + per);
-    const uint4 sv = make_uint4(kSentinel, kSentinel, kSentinel, kSentinel);
-    for (long long e = lo + ct; e < hi; e += 256) st_relaxed_u4(other + e, sv);
+    const uint4 sv = make_uint4(kSentinel, kSentinel, kSentinel, kSentinel), zv = make_uint4(0u, 0u, 0u, 0u);
+    for (long long e = lo + ct; e < hi; e += 256) st_relaxed_u4(other + e, e < acc4 ? sv : zv);
   }
   cbar();
   bool stopped = false;  // set only where every warp reads misc->stop together
@@ -1450,7 +1466,8 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         if (I.layer == 0)
           stage<NBT, ST_EMB, true>(p, act, misc, nullptr, 0, D.H, gain, ii);
         else
-          stage<NBT, ST_SUM, true>(p, act, misc, lay - p.layer_floats + p.off_x1, D.H, D.H, gain, ii);
+          stage<NBT, ST_ACC, true>(p, act, misc, reinterpret_cast<const float*>(acc_of(p, misc, I.layer - 1)),
+                                   D.H, D.H, gain, ii);
         if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_QKV, NBT>(2 * D.RP, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
@@ -1475,8 +1492,8 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         mv_dispatch<OP_DOWN, NBT>(D.Rdn, p, I, page_base, ring, act, D.KS, full, empty, misc, ii);
         break;
       case OP_LM:
-        stage<NBT, ST_SUM, true>(p, act, misc, lay - p.layer_floats + p.off_x1, D.H, D.H,
-                                 static_cast<const uint16_t*>(I.ptr[3]), ii);
+        stage<NBT, ST_ACC, true>(p, act, misc, reinterpret_cast<const float*>(acc_of(p, misc, D.L - 1)), D.H,
+                                 D.H, static_cast<const uint16_t*>(I.ptr[3]), ii);
         if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_LM, NBT>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
@@ -1495,6 +1512,16 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         rec[13] = rec[4] = (long long)globaltimer_ns();
         if (I.op != OP_ATTN) { rec[18] = misc->t_stage_in; rec[19] = misc->t_stage_loaded; }
         if (I.op == OP_LM || (I.op == OP_QKV && I.layer > 0)) { rec[20] = misc->t_sum_x1; rec[21] = misc->t_sum_p; }
+        if (I.op != OP_ATTN) {  // spread of the warps: entry, first page, done
+          long long e0 = LLONG_MAX, e1 = 0, f1 = 0, d0 = LLONG_MAX;
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            e0 = min(e0, misc->warp_entry[w]);
+            e1 = max(e1, misc->warp_entry[w]);
+            f1 = max(f1, misc->warp_first[w]);
+            if (misc->warp_first[w]) d0 = min(d0, misc->warp_done[w]);
+          }
+          rec[22] = e0; rec[23] = e1; rec[24] = f1; rec[25] = d0 == LLONG_MAX ? 0 : d0;
+        }
         rec[16] += misc->slow_n;
         rec[17] += (long long)misc->slow_ns;
         misc->slow_n = 0;

@@ -33,7 +33,8 @@ def flatten(rec: np.ndarray) -> list[dict]:
                              t_staged=int(r[11]), t_last_warp=int(r[12]), t_barrier=int(r[13]),
                              c_core=int(r[14]), c_epi=int(r[15]), slow_n=int(r[16]), slow_ns=int(r[17]),
                              t_stage_in=int(r[18]), t_stage_loaded=int(r[19]),
-                             t_sum_x1=int(r[20]), t_sum_p=int(r[21])))
+                             t_sum_x1=int(r[20]), t_sum_p=int(r[21]),
+                             w_entry0=int(r[22]), w_entry1=int(r[23]), w_first1=int(r[24]), w_done0=int(r[25])))
     return rows
 
 
@@ -50,7 +51,8 @@ def summarize(rec: np.ndarray) -> dict:
         d = per_op.setdefault(r["op"], dict(n=0, wait=0, work=0, signal=0, c_wait=0, c_pages=0,
                                             p_wait=0, p_pages=0, stage=0, units=0, tail=0, n_mv=0,
                                             bar=0, rel=0, c_core=0, c_epi=0, slow_n=0, slow_ns=0,
-                                            st_call=0, st_load=0, st_rest=0, n_sum=0, sum_x1=0, sum_p=0))
+                                            st_call=0, st_load=0, st_rest=0, n_sum=0, sum_x1=0, sum_p=0,
+                                            n_w=0, w_entry=0, w_entry_spread=0, w_first=0, w_done_first=0))
         d["n"] += 1
         if r["t_staged"] and r["t_last_warp"]:
             d["n_mv"] += 1
@@ -63,6 +65,12 @@ def summarize(rec: np.ndarray) -> dict:
                 d["st_call"] += r["t_stage_in"] - r["t_dep"]          # into the staging function
                 d["st_load"] += r["t_stage_loaded"] - r["t_stage_in"]  # activation loads back
                 d["st_rest"] += r["t_staged"] - r["t_stage_loaded"]    # norm, shared-memory stores
+            if r["w_entry0"] and r["w_done0"]:
+                d["n_w"] += 1
+                d["w_entry"] += r["w_entry0"] - r["t_staged"]          # staged -> first warp in its matvec
+                d["w_entry_spread"] += r["w_entry1"] - r["w_entry0"]   # first -> last warp in
+                d["w_first"] += r["w_first1"] - r["w_entry0"]          # -> last warp's first page ready
+                d["w_done_first"] += r["w_done0"] - r["w_entry0"]      # -> first warp done
             if r["t_sum_x1"] and r["t_stage_in"]:
                 d["n_sum"] += 1
                 d["sum_x1"] += r["t_sum_x1"] - r["t_stage_in"]     # residual x1 back
@@ -82,6 +90,8 @@ def summarize(rec: np.ndarray) -> dict:
         d["c_core_us_per_page"] = d["c_core"] / max(1, d["c_pages"]) / 1e3
         d["pages_per_instr_mean"] = d["c_pages"] / max(1, d["n_mv"])
         d["sum_x1_us_mean"] = d["sum_x1"] / max(1, d["n_sum"]) / 1e3
+        for k in ("w_entry", "w_entry_spread", "w_first", "w_done_first"):
+            d[k + "_us_mean"] = d[k] / max(1, d["n_w"]) / 1e3
         d["sum_p_us_mean"] = d["sum_p"] / max(1, d["n_sum"]) / 1e3
         d["slow_rereads_per_instr_mean"] = d["slow_n"] / d["n"]
         d["slow_us_per_reread"] = d["slow_ns"] / max(1, d["slow_n"]) / 1e3
