@@ -146,6 +146,7 @@ struct Misc {
   float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
   float* actset;         // the activation set of the current step
   uint32_t i0;           // this SM's first tape index (profile records)
+  uint32_t attn_extra;   // attention signals beyond one per (lane, kv head), summed over this launch's steps
   unsigned int slow_n;   // profile mode: group re-reads of unwritten activations
   unsigned long long slow_ns;  // and the time they took (summed over threads)
   long long t_stage_in, t_stage_loaded;  // profile mode: stage entry, thread 0's loads back
@@ -349,6 +350,37 @@ struct RingPos {
 // writes its output directly instead of through partials and a merge.
 __device__ __forceinline__ int attn_slices_used(int S, int npg) { return max(1, min(S, npg / 2)); }
 
+// What attention unit (lane, kv head, slice s) does at a context of npg pages.
+// Short contexts (at most kHeadSplitPages pages) with S >= rep split the group
+// by query head instead: slice s < rep takes query head s of the group over all
+// pages and writes it directly, so rep SMs share the group's latency and no
+// merge is needed (the pages are read rep times, from L2 after the first).
+// Longer contexts split the pages into se slices of all rep heads.
+constexpr int kHeadSplitPages = 4;
+struct AttnPlan {
+  bool active, single;  // single: one query head (head split)
+  int head, pb, pe, se;  // head: first query head within the group; pages [pb, pe)
+};
+__device__ __forceinline__ AttnPlan attn_plan(int S, int rep, int npg, int s) {
+  AttnPlan a;
+  if (rep > 1 && S >= rep && npg <= kHeadSplitPages) {
+    a.single = true;
+    a.active = s < rep;
+    a.head = s;
+    a.pb = 0;
+    a.pe = npg;
+    a.se = 1;
+  } else {
+    a.single = false;
+    a.se = attn_slices_used(S, npg);
+    a.active = s < a.se;
+    a.head = 0;
+    a.pb = (int)((long long)s * npg / a.se);
+    a.pe = (int)((long long)(s + 1) * npg / a.se);
+  }
+  return a;
+}
+
 // ---------------------------------------------------------------- producer
 
 __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr& I, uint32_t u,
@@ -437,9 +469,10 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
       for (uint32_t k = 0; k < I.n_units && ok; ++k) {
         int b, g, s;
         attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-        const int pos = p.pos[b] + t, npg = pos / D.PL + 1, se = attn_slices_used(p.S, npg);
-        if (s >= se) continue;
-        const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
+        const int pos = p.pos[b] + t, npg = pos / D.PL + 1;
+        const AttnPlan ap = attn_plan(p.S, D.rep, npg, s);
+        if (!ap.active) continue;
+        const int pb = ap.pb, pe = ap.pe;
         const int* pt = p.page_table + p.slot[b] * D.pages_per_seq;
         int phys_next = pb < pe ? pt[pb] : 0;
         for (int j = pb; j < pe; ++j) {
@@ -870,8 +903,12 @@ __device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBes
 // For QKV and GU the reduce-scatter keeps value pairs (rows j and j + RT/2 of a
 // unit, same lane) in one lane: a RoPE pair for QKV, (gate, up) for GU; the
 // other ops keep single values.
+// Inlined into the consumer for 1-2 lanes: a call spills and reloads the
+// caller's live registers for all 256 threads at every phase start (measured
+// ~0.25 us); with 4-8 lanes the inlined accumulators would not fit the
+// register budget, so those instantiations stay a call (mv_units_call).
 template <int OPK, int RT, int NBT>
-__device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t page_base,
+__device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint32_t page_base,
                                       uint8_t* ring, const float* act, int K, uint64_t* full,
                                       uint64_t* empty, Misc* misc, uint32_t ii) {
   const Dims& D = p.D;
@@ -1085,36 +1122,34 @@ __device__ __noinline__ void mv_units(const KParams& p, const Instr& I, uint32_t
 // query heads of the group.  After the slice the CTA combines the warps'
 // partials into the slice partial, and the last slice to finish (atomic
 // counter) merges all slices of the (lane, kv head) into o.
-template <int DH, int REP, bool KV16F>
-__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
-                                            uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
-                                            Misc* misc, uint32_t ii) {
+// One unit: query heads [hq0, hq0 + NH) of kv head g (NH = REP, or 1 in the head
+// split) over pages [pb, pe) of lane b's context (npg pages); se > 1 only with
+// NH = REP.  Returns false when the CTA stopped.
+template <int DH, int REP, int NH, bool KV16F>
+__device__ __forceinline__ bool attn_one(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+                                         float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii,
+                                         int b, int g, int hq0, int pb, int pe, int npg, int s, int se) {
   constexpr int DC = DH / 8;                 // 16-byte chunks per K/V row
   constexpr int PL = kPageBytes / (4 * DH);  // positions per KV page
   constexpr int RPW = PL / kConsumerWarps;   // positions of a page per warp
-  constexpr int PAIRS = RPW * REP;           // (position, head) scores per warp
+  constexpr int PAIRS = RPW * NH;            // (position, head) scores per warp
   constexpr int SPL = (PAIRS + 31) / 32;     // scores per lane
   constexpr int DPL = DH / 32;               // output dims per lane
   constexpr int CS = DH + 2;                 // partial record: o[DH], m, l
-  static_assert(32 % REP == 0, "REP must divide 32");
+  static_assert(32 % REP == 0 && 32 % NH == 0, "heads must divide 32");
   const Dims& D = p.D;
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const uint32_t NP = (uint32_t)p.ring_pages;
   float4* qlo = reinterpret_cast<float4*>(act);
-  float4* qhi = qlo + REP * DC;
+  float4* qhi = qlo + NH * DC;
   const uint32_t sqlo = smem_u32(qlo), sqhi = smem_u32(qhi);
-  float* comb = act + REP * DH;
+  float* comb = act + NH * DH;
   const float scale = 1.0f / sqrtf((float)DH);
-  const int myh = lane % REP;  // the query head of every score this lane computes
+  const int myh = lane % NH;  // the query head (of the unit's NH) of every score this lane computes
   float* lay = misc->actset + (size_t)I.layer * p.layer_floats;  // this layer's activation block
-  uint32_t used = 0;
-
-  for (uint32_t k = 0; k < I.n_units; ++k) {
-    int b, g, s;
-    attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
-    const int pos = misc->pos[b], npg = pos / PL + 1, se = attn_slices_used(p.S, npg);
-    if (s >= se) continue;  // uniform: this slice is not needed at this context length
-    const int pb = (int)((long long)s * npg / se), pe = (int)((long long)(s + 1) * npg / se);
+  const uint32_t used = 0;
+  {
+    const int pos = misc->pos[b];
     const int np_ = pe - pb;
     // the warp owning this step's position (if this slice holds it) fetches the
     // fp32 K/V row the QKV instruction published, rounded as the cache holds it,
@@ -1146,9 +1181,9 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
                         : (uint32_t)f2bf(vf[2 * e]) | ((uint32_t)f2bf(vf[2 * e + 1]) << 16);
       }
     }
-    for (int e = ct; e < REP * DC; e += 256) {
+    for (int e = ct; e < NH * DC; e += 256) {
       const int h = e / DC, c = e % DC;
-      const float* src = lay + p.off_q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
+      const float* src = lay + p.off_q + (size_t)b * D.qdim + (hq0 + h) * DH + c * 8;
       float4 a0 = ld_relaxed_f4(src), a1 = ld_relaxed_f4(src + 4);
       ready(a0, p, src, ii, misc);
       ready(a1, p, src + 4, ii, misc);
@@ -1159,9 +1194,9 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     }
     cbar();
 
-    float m[REP], l[REP], o[REP][DPL];
+    float m[NH], l[NH], o[NH][DPL];
 #pragma unroll
-    for (int h = 0; h < REP; ++h) {
+    for (int h = 0; h < NH; ++h) {
       m[h] = -CUDART_INF_F;
       l[h] = 0.f;
 #pragma unroll
@@ -1191,12 +1226,12 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         }
         __syncwarp();
       }
-      // scores: lane -> pair pi = lane + 32 t -> (position r0 + pi / REP, head pi % REP)
+      // scores: lane -> pair pi = lane + 32 t -> (position r0 + pi / NH, head pi % NH)
       float sc[SPL];
       const uint32_t kb = smem_u32(pg);
 #pragma unroll
       for (int t = 0; t < SPL; ++t) {
-        const int pi = lane + 32 * t, row = r0 + pi / REP;
+        const int pi = lane + 32 * t, row = r0 + pi / NH;
         float sv = -CUDART_INF_F;
         if (pi < PAIRS && row < cnt) {
           float2 a2 = make_float2(0.f, 0.f);
@@ -1215,15 +1250,15 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         }
         sc[t] = sv;
       }
-      // per-head max over the warp's positions (lanes with equal lane % REP share a head)
+      // per-head max over the warp's positions (lanes with equal lane % NH share a head)
       float mx = sc[0];
 #pragma unroll
       for (int t = 1; t < SPL; ++t) mx = fmaxf(mx, sc[t]);
 #pragma unroll
-      for (int off = REP; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+      for (int off = NH; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
       float mnew_mine = fmaxf(m[0], mx);
 #pragma unroll
-      for (int h = 1; h < REP; ++h)
+      for (int h = 1; h < NH; ++h)
         if (h == myh) mnew_mine = fmaxf(m[h], mx);
       float pr[SPL], ps = 0.f;
 #pragma unroll
@@ -1232,10 +1267,10 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         ps += pr[t];
       }
 #pragma unroll
-      for (int off = REP; off < 32; off <<= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
+      for (int off = NH; off < 32; off <<= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
       // fold into the running state of every head (lane h holds head h's values)
 #pragma unroll
-      for (int h = 0; h < REP; ++h) {
+      for (int h = 0; h < NH; ++h) {
         const float mh = __shfl_sync(0xFFFFFFFFu, mnew_mine, h);
         const float sh = __shfl_sync(0xFFFFFFFFu, ps, h);
         const float corr = mh > -CUDART_INF_F ? __expf(m[h] - mh) : 1.f;
@@ -1258,8 +1293,8 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
           vv[0] = kv_lo<KV16F>(w.x); vv[1] = kv_hi<KV16F>(w.x); vv[2] = kv_lo<KV16F>(w.y); vv[3] = kv_hi<KV16F>(w.y);
         }
 #pragma unroll
-        for (int h = 0; h < REP; ++h) {
-          const int pi = rr * REP + h;
+        for (int h = 0; h < NH; ++h) {
+          const int pi = rr * NH + h;
           const float ph = __shfl_sync(0xFFFFFFFFu, pr[pi / 32], pi % 32);
 #pragma unroll
           for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(ph, vv[e], o[h][e]);
@@ -1270,38 +1305,38 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
       if (lane == 0) mbar_arrive_cnt(&empty[slot], 1u);  // one of the 8 warps
     }
     // combine the warps' partials into this slice's partial
-    float* mine = comb + cw * REP * CS;
+    float* mine = comb + cw * NH * CS;
 #pragma unroll
-    for (int h = 0; h < REP; ++h) {
+    for (int h = 0; h < NH; ++h) {
 #pragma unroll
       for (int e = 0; e < DPL; ++e) mine[h * CS + lane * DPL + e] = o[h][e];
       if (lane == 0) { mine[h * CS + DH] = m[h]; mine[h * CS + DH + 1] = l[h]; }
     }
     cbar();
-    if (misc->stop) { cbar(); break; }
+    if (misc->stop) { cbar(); return false; }
     if (se == 1) {
-      // the only slice: normalise and write the output, then signal
-      for (int e = ct; e < REP * DH; e += 256) {
+      // the only slice of these heads: normalise and write the output, then signal
+      for (int e = ct; e < NH * DH; e += 256) {
         const int h = e / DH, i = e % DH;
         float M = -CUDART_INF_F;
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * REP + h) * CS + DH]);
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * NH + h) * CS + DH]);
         float L = 0.f, O = 0.f;
         for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = comb[(w * REP + h) * CS + DH];
+          const float mw = comb[(w * NH + h) * CS + DH];
           if (mw > -CUDART_INF_F) {
             const float f = __expf(mw - M);
-            L += comb[(w * REP + h) * CS + DH + 1] * f;
-            O += comb[(w * REP + h) * CS + i] * f;
+            L += comb[(w * NH + h) * CS + DH + 1] * f;
+            O += comb[(w * NH + h) * CS + i] * f;
           }
         }
-        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
+        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (hq0 + h) * DH + i, canon(O / L));
       }
       cbar();
       if (ct == 0) red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
-      used += (uint32_t)np_;
       cbar();
-      continue;
+      return true;
     }
+    if constexpr (NH == REP) {
     float* part = p.part + ((size_t)(b * D.Hkv + g) * p.S + s) * REP * CS;
     for (int e = ct; e < REP * DH; e += 256) {
       const int h = e / DH, i = e % DH;
@@ -1349,23 +1384,73 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
         red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
       }
     }
-    used += (uint32_t)np_;
     cbar();
+    }  // NH == REP
+  }
+  (void)used;
+  return true;
+}
+
+// Split-KV GQA decode attention for the units of this instruction (see
+// attn_plan): a slice covers a contiguous range of KV pages of one (lane, kv
+// head) and all its query heads, or, for short contexts, one query head over
+// all pages.  Every page is shared by the 8 warps, each taking PL/8 of its
+// positions: a lane scores one (position, query head) pair, then each warp folds
+// its positions into an online-softmax partial (running max m, sum l,
+// unnormalised o).  After the slice the CTA combines the warps' partials; a
+// slice that covers all pages writes o, otherwise the last slice to finish
+// (atomic counter) merges all slices of the (lane, kv head) into o.  Returns the
+// ring pages consumed.
+template <int DH, int REP, bool KV16F>
+__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
+                                            uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
+                                            Misc* misc, uint32_t ii) {
+  constexpr int PL = kPageBytes / (4 * DH);
+  const Dims& D = p.D;
+  uint32_t used = 0;
+  for (uint32_t k = 0; k < I.n_units; ++k) {
+    int b, g, s;
+    attn_unit(I.u0 + k, D.Hkv, p.S, &b, &g, &s);
+    const int npg = misc->pos[b] / PL + 1;
+    const AttnPlan ap = attn_plan(p.S, REP, npg, s);
+    if (!ap.active) continue;  // uniform: this slice is not needed at this context length
+    bool ok;
+    if (REP > 1 && ap.single)
+      ok = attn_one<DH, REP, 1, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g,
+                                       g * REP + ap.head, ap.pb, ap.pe, npg, s, 1);
+    else
+      ok = attn_one<DH, REP, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g,
+                                         g * REP, ap.pb, ap.pe, npg, s, ap.se);
+    if (!ok) break;
+    used += (uint32_t)(ap.pe - ap.pb);
   }
   return used;
 }
 
 // ---------------------------------------------------------------- consumers: ops
 
+template <int OPK, int RT, int NBT>
+__device__ __noinline__ void mv_units_call(const KParams& p, const Instr& I, uint32_t pb, uint8_t* ring,
+                                           const float* act, int K, uint64_t* full, uint64_t* empty, Misc* misc,
+                                           uint32_t ii) {
+  mv_units<OPK, RT, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii);
+}
+template <int OPK, int RT, int NBT>
+__device__ __forceinline__ void mv_run(const KParams& p, const Instr& I, uint32_t pb, uint8_t* ring,
+                                       const float* act, int K, uint64_t* full, uint64_t* empty, Misc* misc,
+                                       uint32_t ii) {
+  if constexpr (NBT <= 2) mv_units<OPK, RT, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii);
+  else mv_units_call<OPK, RT, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii);
+}
 template <int OPK, int NBT>
 __device__ __forceinline__ void mv_dispatch(int rt, const KParams& p, const Instr& I, uint32_t pb,
                                             uint8_t* ring, const float* act, int K, uint64_t* full,
                                             uint64_t* empty, Misc* misc, uint32_t ii) {
   switch (rt) {
-    case 1: if constexpr (OPK == OP_O || OPK == OP_DOWN || OPK == OP_LM) mv_units<OPK, 1, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
-    case 2: mv_units<OPK, 2, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
-    case 4: mv_units<OPK, 4, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
-    case 8: mv_units<OPK, 8, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 1: if constexpr (OPK == OP_O || OPK == OP_DOWN || OPK == OP_LM) mv_run<OPK, 1, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 2: mv_run<OPK, 2, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 4: mv_run<OPK, 4, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
+    case 8: mv_run<OPK, 8, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii); break;
   }
 }
 
@@ -1404,6 +1489,11 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     misc->i0 = i0;
     misc->actset = p.acts + (size_t)((p.parity0 + t) & 1) * p.set_floats;
     if (t > 0 && !wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, i0)) misc->stop = 1;
+    // a (lane, kv head) split by query head signals once per head (attn_plan)
+    uint32_t extra = 0;
+    for (int b = 0; b < p.nb; ++b)
+      if (attn_plan(p.S, D.rep, (p.pos[b] + t) / D.PL + 1, 0).single) extra += (uint32_t)(D.Hkv * (D.rep - 1));
+    misc->attn_extra += extra;
   }
   cbar();
   if (misc->stop) break;
@@ -1453,7 +1543,8 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
       // hint: every warp of a matvec instruction bumps its counter, attention once
       // per (lane, kv head); counters only grow within a launch
       const uint32_t per = I.op == OP_O ? 1u : (uint32_t)kConsumerWarps;
-      if (!wait_hint(p, p.ctr + I.dep, I.dep_target * per * (uint32_t)(t + 1), ii)) misc->stop = 1;
+      const uint32_t extra = I.op == OP_O ? misc->attn_extra : 0u;
+      if (!wait_hint(p, p.ctr + I.dep, I.dep_target * per * (uint32_t)(t + 1) + extra, ii)) misc->stop = 1;
     }
     cbar();
     if (rec) rec[2] = (long long)globaltimer_ns();
@@ -1568,6 +1659,7 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     misc->entry_abort = aborted(p) ? 1 : 0;
     misc->slow_n = 0;
     misc->slow_ns = 0;
+    misc->attn_extra = 0;
   }
   __syncthreads();
   if (!misc->entry_abort) {
