@@ -1391,6 +1391,168 @@ __device__ __forceinline__ bool attn_one(const KParams& p, const Instr& I, uint3
   return true;
 }
 
+// Short-context attention of one query head (the head split of attn_plan):
+// every position of lane b's context (npg <= kHeadSplitPages pages, at most 256
+// positions) is scored at once, one position per thread, then a block-wide
+// softmax, then P.V with one thread per (pair of output dims, run of 32
+// positions within one page).  The
+// pages of the unit are all resident in the ring (npg <= 4 <= ring pages).
+template <int DH, bool KV16F>
+__device__ __forceinline__ bool attn_flat(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+                                          float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii,
+                                          int b, int g, int hq, int npg) {
+  constexpr int PL = kPageBytes / (4 * DH);  // positions per KV page
+  constexpr int DC = DH / 8;                 // 16-byte chunks per K row
+  constexpr int WPR = DH / 2;                       // 32-bit words (dim pairs) per V row
+  constexpr int NCH = kConsumerWarps * 32 / WPR;   // runs of positions in P.V
+  constexpr int RUN = kHeadSplitPages * PL / NCH;  // positions per run
+  static_assert(kHeadSplitPages * PL <= kConsumerWarps * 32, "one position per thread");
+  static_assert(PL % RUN == 0, "a run stays within one page");
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
+  const uint32_t NP = (uint32_t)p.ring_pages;
+  float* qs = act;            // [DH] query, scaled by 1/sqrt(d)
+  float* ps = qs + DH;        // [256] unnormalised probabilities
+  float* wred = ps + 256;     // [2][8] per-warp maxima, sums
+  float* part = wred + 16;    // [NCH][DH] partial outputs (NCH * DH = 512)
+  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
+  const int pos = misc->pos[b], cnt = pos + 1;
+  // ring slots of the unit's pages
+  uint32_t slot[kHeadSplitPages];
+  {
+    RingPos rp;
+    rp.init(page_base, NP);
+#pragma unroll
+    for (int j = 0; j < kHeadSplitPages; ++j, rp.advance(1, NP)) slot[j] = rp.slot;
+  }
+  // the query, and this step's K/V row patched into the last page (rounded as the
+  // cache holds it; the page's bulk copy stops short of that row)
+  if (ct < DH / 4) {
+    const float* src = lay + p.off_q + (size_t)b * D.qdim + hq * DH + ct * 4;
+    float4 v = ld_relaxed_f4(src);
+    ready(v, p, src, ii, misc);
+    const float sc = 1.0f / sqrtf((float)DH);
+    reinterpret_cast<float4*>(qs)[ct] = make_float4(v.x * sc, v.y * sc, v.z * sc, v.w * sc);
+  }
+  const int rcur = pos - (npg - 1) * PL;
+  uint8_t* lastpg = ring + (size_t)slot[npg - 1 < 0 ? 0 : npg - 1] * kPageBytes;
+  const bool patcher = ct >= 32 && ct < 32 + DH / 2;  // warp 1 (and 2 for DH = 128)
+  if (patcher) {
+    const int e = ct - 32;  // element pair (2e, 2e + 1)
+    const float* kn = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + g * DH + 2 * e;
+    float2 k2 = ld_relaxed_f2(kn), v2 = ld_relaxed_f2(kn + D.kvdim);
+    ready(k2, p, kn, ii, misc);
+    ready(v2, p, kn + D.kvdim, ii, misc);
+    const uint32_t kw = KV16F ? (uint32_t)f2h(k2.x) | ((uint32_t)f2h(k2.y) << 16)
+                              : (uint32_t)f2bf(k2.x) | ((uint32_t)f2bf(k2.y) << 16);
+    const uint32_t vw = KV16F ? (uint32_t)f2h(v2.x) | ((uint32_t)f2h(v2.y) << 16)
+                              : (uint32_t)f2bf(v2.x) | ((uint32_t)f2bf(v2.y) << 16);
+    reinterpret_cast<uint32_t*>(lastpg + rcur * DH * 2)[e] = kw;
+    reinterpret_cast<uint32_t*>(lastpg + PL * DH * 2 + rcur * DH * 2)[e] = vw;
+  }
+  // every warp waits for all pages (each warp releases each page once, below)
+  bool ok = true;
+  {
+    RingPos rp;
+    rp.init(page_base, NP);
+    for (int j = 0; j < npg && ok; ++j, rp.advance(1, NP)) ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+  }
+  if (!__all_sync(0xFFFFFFFFu, ok) && lane == 0) misc->stop = 1;
+  cbar();
+  if (misc->stop) { cbar(); return false; }
+  // scores: thread t -> position t
+  float sv = -CUDART_INF_F;
+  if (ct < cnt) {
+    const int j = ct / PL, row = ct % PL;
+    uint32_t sl = slot[0];
+#pragma unroll
+    for (int jj = 1; jj < kHeadSplitPages; ++jj)
+      if (jj == j) sl = slot[jj];
+    const uint32_t krow = smem_u32(ring + (size_t)sl * kPageBytes) + (uint32_t)(row * DH * 2);
+    const uint32_t qa = smem_u32(qs);
+    float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int cc = 0; cc < DC; ++cc) {
+      const int c = (cc + lane) & (DC - 1);  // lanes of a phase hit distinct banks
+      const uint4 kw = lds128(krow + (uint32_t)(c * 16));
+      const float4 q0 = lds128f(qa + (uint32_t)(c * 32)), q1 = lds128f(qa + (uint32_t)(c * 32 + 16));
+      a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.x), kv_hi<KV16F>(kw.x)), make_float2(q0.x, q0.y), a2);
+      a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.y), kv_hi<KV16F>(kw.y)), make_float2(q0.z, q0.w), a2);
+      a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.z), kv_hi<KV16F>(kw.z)), make_float2(q1.x, q1.y), a2);
+      a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.w), kv_hi<KV16F>(kw.w)), make_float2(q1.z, q1.w), a2);
+    }
+    sv = a2.x + a2.y;
+  }
+  // block max, then probabilities and their sum
+  float mx = sv;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if (lane == 0) wred[cw] = mx;
+  cbar();
+  float M = wred[0];
+#pragma unroll
+  for (int w = 1; w < kConsumerWarps; ++w) M = fmaxf(M, wred[w]);
+  const float e = ct < cnt ? __expf(sv - M) : 0.f;
+  ps[ct] = e;
+  float sum = e;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+  if (lane == 0) wred[8 + cw] = sum;
+  cbar();
+  // P.V: thread (word wd = dims 2wd, 2wd + 1; run ch) sums positions [ch * RUN, ch * RUN + RUN)
+  {
+    const int wd = ct % WPR, ch = ct / WPR;
+    const int t0 = ch * RUN, t1 = min(cnt, t0 + RUN);
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+    if (t0 < t1) {
+      const int j = t0 / PL;
+      uint32_t sl = slot[0];
+#pragma unroll
+      for (int jj = 1; jj < kHeadSplitPages; ++jj)
+        if (jj == j) sl = slot[jj];
+      const uint32_t vb = smem_u32(ring + (size_t)sl * kPageBytes + PL * DH * 2) +
+                          (uint32_t)((t0 % PL) * DH * 2 + wd * 4);
+      const float* pp = ps + t0;
+      const int n = t1 - t0;
+      int t = 0;
+#pragma unroll 4
+      for (; t + 2 <= n; t += 2) {
+        const uint32_t w0 = lds32(vb + (uint32_t)(t * DH * 2)), w1 = lds32(vb + (uint32_t)((t + 1) * DH * 2));
+        const float p0 = pp[t], p1 = pp[t + 1];
+        a0 = fmaf(p0, kv_lo<KV16F>(w0), a0);
+        a1 = fmaf(p0, kv_hi<KV16F>(w0), a1);
+        b0 = fmaf(p1, kv_lo<KV16F>(w1), b0);
+        b1 = fmaf(p1, kv_hi<KV16F>(w1), b1);
+      }
+      if (t < n) {
+        const uint32_t w0 = lds32(vb + (uint32_t)(t * DH * 2));
+        a0 = fmaf(pp[t], kv_lo<KV16F>(w0), a0);
+        a1 = fmaf(pp[t], kv_hi<KV16F>(w0), a1);
+      }
+    }
+    part[ch * DH + 2 * wd] = a0 + b0;
+    part[ch * DH + 2 * wd + 1] = a1 + b1;
+  }
+  // every read of the pages is done: release them (the patch first, to the async proxy)
+  if (patcher) fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0)
+    for (int j = 0; j < npg; ++j) mbar_arrive_cnt(&empty[slot[j]], 1u);
+  cbar();
+  if (ct < DH) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) L += wred[8 + w];
+    float O = 0.f;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) O += part[c * DH + ct];
+    st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + hq * DH + ct, canon(O / L));
+  }
+  cbar();
+  if (ct == 0) red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+  return true;
+}
+
 // Split-KV GQA decode attention for the units of this instruction (see
 // attn_plan): a slice covers a contiguous range of KV pages of one (lane, kv
 // head) and all its query heads, or, for short contexts, one query head over
@@ -1416,8 +1578,8 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     if (!ap.active) continue;  // uniform: this slice is not needed at this context length
     bool ok;
     if (REP > 1 && ap.single)
-      ok = attn_one<DH, REP, 1, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g,
-                                       g * REP + ap.head, ap.pb, ap.pe, npg, s, 1);
+      ok = attn_flat<DH, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, g * REP + ap.head,
+                                npg);
     else
       ok = attn_one<DH, REP, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g,
                                          g * REP, ap.pb, ap.pe, npg, s, ap.se);

@@ -316,6 +316,8 @@ SmemLayout smem_layout(const Dims& D, int nb_max, int max_dyn_smem, int want_pag
   int act = nb_max * std::max(std::max(D.H, D.qdim), D.KS) * 4;
   // attention scratch: q (rep x d) and the per-warp partials (rep x (d + 2))
   int attn = D.rep * D.d * 4 + kConsumerWarps * D.rep * (D.d + 2) * 4;
+  // single-head short-context attention: q, 256 probabilities, 16 reductions, 512 partials
+  attn = std::max(attn, (D.d + 256 + 16 + 512) * 4);
   s.act_bytes = (std::max(act, attn) + 1023) / 1024 * 1024;
   int misc = 8192;  // mbarriers (128 full + 64 empty), reduction scratch, step constants
   // Prefer a ring that fits the 196 KiB shared-memory carveout: the larger L1
