@@ -56,7 +56,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -111,8 +111,9 @@ def kernel_src_hash() -> str:
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on this
-    workload with the current kernel sources; otherwise None."""
+    """DRAM bytes per decode step from the committed ncu summary (a capture of one
+    single-step launch of the kernel), if it was taken on this workload with the
+    current kernel sources; otherwise None."""
     p = os.path.join(ROOT, "profiles", f"mk_decode_kernel_{workload}_traffic.txt")
     if not os.path.exists(p):
         return None
@@ -124,7 +125,7 @@ def recorded_traffic(workload: str):
                 kv[k.strip()] = v.strip()
     if kv.get("kernel_src_sha256_16") != kernel_src_hash():
         return None
-    return float(kv["dram_bytes_per_launch"])
+    return float(kv["dram_bytes_per_step"])
 
 
 def _dist():
@@ -223,7 +224,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=25.0)
     ap.add_argument("--traffic-bytes", type=float, default=None,
-                    help="DRAM bytes per launch from an ncu capture of this kernel (optional)")
+                    help="DRAM bytes per decode step from an ncu capture of this kernel (optional)")
     args = ap.parse_args()
     from synth import configs
 
