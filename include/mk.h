@@ -256,6 +256,30 @@ mk_status mk_greedy_head_noalloc(const float* hidden_dev, int32_t nb, int32_t hi
                                  const void* final_norm, const void* lm_head, int32_t vocab,
                                  float rms_eps, float* logits_dev, int32_t* ids_dev, void* stream);
 
+/* The two engines a decode step's matvecs can run on, measured apart.
+ *
+ * The Hazy megakernel article (section "Megakernel: a deep-fusion design from
+ * scratch") says tensor cores win again on Blackwell.  This call runs the
+ * streaming batched matvec the decode kernel is made of,
+ *     Y[b][r] = sum_k W[r][k] * X[b][k],  b < nb,  r < rows,
+ * on one engine, so the claim can be checked per batch size:
+ *   engine 0  CUDA cores (packed FP32 FMA over bulk-copied pages of whole rows;
+ *             the decode kernel's engine); requires K == 2048, rows % 4 == 0;
+ *   engine 1  tcgen05 tensor cores: TMA tiles of 128 rows x 64, MMA M = 128,
+ *             N = 16 with X split into bf16 high and low parts (fp32-level
+ *             accuracy), fp32 accumulators in tensor memory; requires K % 64 == 0,
+ *             K <= 4096, rows % 128 == 0.
+ *   W  device bf16 [rows][K] row-major, 16-byte aligned (caller-owned)
+ *   X  device fp32 [nb][K], 16-byte aligned;   Y  device fp32 [nb][rows]
+ *   nb 1..8;  n_sm: CTAs at most (0: one per SM);  wait_limit_ms: bound of every
+ *   wait in the kernel (0: 1000).
+ * Asynchronous on `stream`; MK_ERR_UNSUPPORTED for shapes outside the limits,
+ * without launching.  mk_matvec_engine_status synchronises `stream` and returns
+ * MK_ERR_TIMEOUT if a wait of the last launch ran out. */
+mk_status mk_matvec_engine(int32_t engine, const void* W, int32_t rows, int32_t K, const float* X,
+                           int32_t nb, float* Y, int32_t n_sm, int32_t wait_limit_ms, void* stream);
+mk_status mk_matvec_engine_status(void* stream);
+
 /* Library version string (static storage). */
 const char* mk_version(void);
 

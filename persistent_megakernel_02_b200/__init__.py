@@ -112,6 +112,10 @@ _SIGS = {
                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
                                               ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                               ctypes.c_void_p]),
+    "mk_matvec_engine": (ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_void_p]),
+    "mk_matvec_engine_status": (ctypes.c_int, [ctypes.c_void_p]),
     "mk_version": (ctypes.c_char_p, []),
 }
 
@@ -173,6 +177,23 @@ def greedy_head_noalloc(hidden, final_norm, lm_head, rms_eps, ids, logits=None, 
                                         None if logits is None else logits.data_ptr(),
                                         ids.data_ptr(), _stream_handle(stream)),
            "mk_greedy_head_noalloc")
+
+
+ENGINES = {"cuda_cores": 0, "tcgen05": 1}
+
+
+def matvec_engine(engine, W, X, Y, n_sm: int = 0, wait_limit_ms: int = 0, stream=None):
+    """Y[b, r] = sum_k W[r, k] * X[b, k] on one engine (``mk_matvec_engine``):
+    "cuda_cores" or "tcgen05".  W bf16 [rows, K], X float32 [nb, K], Y float32
+    [nb, rows], all CUDA tensors.  Asynchronous; ``matvec_engine_status`` waits."""
+    rows, K = W.shape
+    nb = X.shape[0]
+    _check(lib().mk_matvec_engine(ENGINES[engine], W.data_ptr(), rows, K, X.data_ptr(), nb, Y.data_ptr(),
+                                  n_sm, wait_limit_ms, _stream_handle(stream)), "mk_matvec_engine")
+
+
+def matvec_engine_status(stream=None):
+    _check(lib().mk_matvec_engine_status(_stream_handle(stream)), "mk_matvec_engine")
 
 
 def _i32_array(values):

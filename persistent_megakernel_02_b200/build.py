@@ -15,8 +15,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmk.so")
-SOURCES = ["mk_api.cu", "mk_sched.cpp", "mk_noalloc.cu"]
-DEPS = ["mk_kernel.cuh", "mk_device.cuh", "mk_plan.h"]
+SOURCES = ["mk_api.cu", "mk_sched.cpp", "mk_noalloc.cu", "mk_engines.cu"]
+DEPS = ["mk_kernel.cuh", "mk_device.cuh", "mk_matvec.cuh", "mk_plan.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
