@@ -19,6 +19,7 @@ struct mk_ctx {
   mk_config cfg{};
   Dims D{};
   int dev = 0, n_sm = 0, nbt = 1;
+  int spec = 0;  // kernel specialisation (mk_kernel.cuh, Spec)
   unsigned long long wait_limit_ns = 1000000000ull;
   SmemLayout sm{};
   std::vector<Tape> tapes;  // index nb - 1
@@ -164,6 +165,19 @@ void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w) {
   }
 }
 
+template <int SPEC>
+const void* kernel_for_spec(int nbt) {
+  switch (nbt) {
+    case 1: return (const void*)mk_decode_kernel<1, SPEC>;
+    case 2: return (const void*)mk_decode_kernel<2, SPEC>;
+    case 4: return (const void*)mk_decode_kernel<4, SPEC>;
+    default: return (const void*)mk_decode_kernel<8, SPEC>;
+  }
+}
+const void* kernel_for(int nbt, int spec) {
+  return spec == 1 ? kernel_for_spec<1>(nbt) : spec == 2 ? kernel_for_spec<2>(nbt) : kernel_for_spec<0>(nbt);
+}
+
 mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   const Dims& D = h->D;
   // tapes, one per active batch size
@@ -226,25 +240,20 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   h->sm = smem_layout(D, h->nbt, max_dyn, want_pages);
   if (h->sm.ring_pages < kConsumerWarps) return MK_ERR_UNSUPPORTED;
   if (h->sm.ring_pages > 64) return MK_ERR_UNSUPPORTED;
-  const void* kfn[4] = {(const void*)mk_decode_kernel<1>, (const void*)mk_decode_kernel<2>,
-                        (const void*)mk_decode_kernel<4>, (const void*)mk_decode_kernel<8>};
-  for (auto k : kfn)
-    MK_TRY(from_cuda(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, h->sm.total)));
+  // the specialised kernel when every unit has the same row count and the attention one known form
+  const int rq = 2 * D.RP, ro = D.Ro, rg = 2 * D.Rgu, rd = D.Rdn, rl = D.Rlm;
+  if (rq == 4 && ro == 4 && rg == 4 && rd == 4 && rl == 4 && D.d == 64 && D.rep == 4 && !D.kv_fp16) h->spec = 1;
+  else if (rq == 2 && ro == 2 && rg == 2 && rd == 2 && rl == 2 && D.d == 128 && D.rep == 4 && D.kv_fp16) h->spec = 2;
+  for (int nbt : {1, 2, 4, 8})
+    MK_TRY(from_cuda(cudaFuncSetAttribute(kernel_for(nbt, h->spec), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          h->sm.total)));
   int blocks = 0;
-  MK_TRY(from_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, mk_decode_kernel<8>, kThreads,
+  MK_TRY(from_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kernel_for(8, h->spec), kThreads,
                                                                   h->sm.total)));
   if (blocks < 1) return MK_ERR_UNSUPPORTED;
   return from_cuda(cudaDeviceSynchronize());
 }
 
-const void* kernel_for(int nbt) {
-  switch (nbt) {
-    case 1: return (const void*)mk_decode_kernel<1>;
-    case 2: return (const void*)mk_decode_kernel<2>;
-    case 4: return (const void*)mk_decode_kernel<4>;
-    default: return (const void*)mk_decode_kernel<8>;
-  }
-}
 
 // One launch of n_steps decode steps (see KParams for the token / ids / logits modes).
 mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, const int* slot,
@@ -296,7 +305,7 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.D = D;
   void* args[] = {&p};
   const int nbt = lanes_template(nb);
-  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(nbt), dim3(h->n_sm), dim3(kThreads), args,
+  cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(nbt, h->spec), dim3(h->n_sm), dim3(kThreads), args,
                                               (size_t)h->sm.total, st);
   h->step++;
   if (e == cudaSuccess) h->steps_run += (unsigned long long)n_steps;
