@@ -1464,9 +1464,9 @@ __device__ __forceinline__ bool attn_flat(const KParams& p, const Instr& I, uint
 // (atomic counter) merges all slices of the (lane, kv head) into o.  Returns the
 // ring pages consumed.
 template <int DH, int REP, bool KV16F>
-__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base,
-                                            uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
-                                            Misc* misc, uint32_t ii) {
+__device__ __forceinline__ uint32_t attn_units_body(const KParams& p, const Instr& I, uint32_t page_base,
+                                                    uint8_t* ring, float* act, uint64_t* full, uint64_t* empty,
+                                                    Misc* misc, uint32_t ii) {
   constexpr int PL = kPageBytes / (4 * DH);
   const Dims& D = p.D;
   uint32_t used = 0;
@@ -1487,6 +1487,11 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
     used += (uint32_t)(ap.pe - ap.pb);
   }
   return used;
+}
+template <int DH, int REP, bool KV16F>
+__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+                                            float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii) {
+  return attn_units_body<DH, REP, KV16F>(p, I, page_base, ring, act, full, empty, misc, ii);
 }
 
 // ---------------------------------------------------------------- consumers: ops
@@ -1641,7 +1646,10 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         break;
       }
       case OP_ATTN:
-        if constexpr (SPEC != 0)
+        if constexpr (SPEC != 0 && NBT <= 2)  // inlined in the specialised kernels (no call spills)
+          used = attn_units_body<Spec<SPEC>::dh, Spec<SPEC>::rep, Spec<SPEC>::kv16>(p, I, page_base, ring, act,
+                                                                                    full, empty, misc, ii);
+        else if constexpr (SPEC != 0)
           used = attn_units<Spec<SPEC>::dh, Spec<SPEC>::rep, Spec<SPEC>::kv16>(p, I, page_base, ring, act, full,
                                                                                empty, misc, ii);
         else
