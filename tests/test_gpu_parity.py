@@ -183,6 +183,31 @@ def test_multi_step_launch_matches_single_steps_and_oracle():
             assert got[t] == want[t], (b, t)
 
 
+def test_multi_step_launch_across_the_attention_mode_threshold():
+    """Contexts of at most 4 KV pages use single-head attention units, longer ones
+    split the pages over slices and merge; one multi-step launch over positions
+    250..261 changes mode at 256 from one step to the next.  Its logits match the
+    oracle at every step."""
+    cfg = configs.model_config("tiny", max_batch=1, max_seq=280)
+    w = H.gpu_weights(cfg)
+    prompt = synth.prompt_tokens(cfg, 0, 250).tolist()
+    teacher = synth.teacher_tokens(cfg, 0, 12).numpy()
+    n, V = 12, cfg["vocab"]
+    mk = _mk(cfg, w)
+    mk.prefill(0, prompt)  # itself crosses 64-position pages, not the threshold
+    tok = torch.tensor([int(teacher[0])], dtype=torch.int32, device="cuda")
+    ids = torch.empty((n, 1), dtype=torch.int32, device="cuda")
+    lg = torch.empty((n, 1, V), dtype=torch.float32, device="cuda")
+    mk.decode_steps(tok, [250], n, ids, lg)  # positions 250..261: 4 pages of 64 end at 255
+    mk.sync()
+    mk.close()
+    orc = H.oracle_for(cfg, w)
+    greedy = [int(teacher[0])] + ids[:, 0].tolist()
+    _, w_steps = H.oracle_teacher_forced(orc, np.array(prompt), np.array(greedy[:n]), n)
+    for t in range(n):
+        H.compare_logits(lg[t, 0].cpu().numpy(), w_steps[t], f"step {t} (position {250 + t})")
+
+
 def test_zero_layers_greedy_is_identity_tiny():
     cfg = configs.model_config("tiny")
     w = H.gpu_weights(cfg, zero_layers=True)
