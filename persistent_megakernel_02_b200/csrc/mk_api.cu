@@ -20,6 +20,7 @@ struct mk_ctx {
   Dims D{};
   int dev = 0, n_sm = 0, nbt = 1;
   int spec = 0;  // kernel specialisation (mk_kernel.cuh, Spec)
+  int hints = 0;  // KParams::hints (the fault-injection hook works through a hint wait)
   unsigned long long wait_limit_ns = 1000000000ull;
   SmemLayout sm{};
   std::vector<Tape> tapes;  // index nb - 1
@@ -275,6 +276,7 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.acc_base = h->acc_base;
   p.acc_floats = h->acc_floats;
   p.parity0 = (int)(h->steps_run & 1);
+  p.hints = h->hints;
   p.part = h->part; p.lm_part = h->lm_part;
   p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
   const int par = (int)(h->step & 1);
@@ -394,6 +396,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
     s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * kProfSlots);
   }
   if (s == MK_OK && o.debug_fault == 1) {
+    h->hints = 1;
     // test hook: one wait (the first layer-0 O projection of SM 0's tape for every
     // batch size) gets a target one above what its counter can reach
     for (size_t k = 0; k < h->tapes.size(); ++k) {
