@@ -60,6 +60,11 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # nvidia-smi takes a while to start: begin timing once it samples
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
+            self.lines.clear()
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -70,6 +75,9 @@ class ClockSampler:
 
     def __exit__(self, *a):
         if self.proc:
+            t0 = time.time()  # a short timed region: wait for at least two samples
+            while len(self.lines) < 2 and time.time() - t0 < 0.5:
+                time.sleep(0.01)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)

@@ -20,7 +20,10 @@ struct mk_ctx {
   Dims D{};
   int dev = 0, n_sm = 0, nbt = 1;
   int spec = 0;  // kernel specialisation (mk_kernel.cuh, Spec)
-  int hints = 0;  // KParams::hints (the fault-injection hook works through a hint wait)
+  // KParams::hints: every op reads its inputs directly (measured faster than waiting on
+  // the hint counters, also for the O projection's long wait on attention).  The
+  // fault-injection hook works through hint waits, so it turns all of them on.
+  int hints = 0;
   unsigned long long wait_limit_ns = 1000000000ull;
   SmemLayout sm{};
   std::vector<Tape> tapes;  // index nb - 1
@@ -396,7 +399,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
     s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * kProfSlots);
   }
   if (s == MK_OK && o.debug_fault == 1) {
-    h->hints = 1;
+    h->hints = 0xFE;
     // test hook: one wait (the first layer-0 O projection of SM 0's tape for every
     // batch size) gets a target one above what its counter can reach
     for (size_t k = 0; k < h->tapes.size(); ++k) {

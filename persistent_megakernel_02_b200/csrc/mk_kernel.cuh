@@ -96,8 +96,9 @@ struct KParams {
   long long set_floats, layer_floats, acc_base, acc_floats;
   int off_q, off_kvn, off_o, off_x1, off_a;
   int parity0;  // set of this launch's step 0
-  int hints;    // 1: wait on each op's hint counter before reading its inputs; 0: read and
-                // validate the inputs directly (they carry their own readiness)
+  int hints;    // bit op set: instructions of that op wait on their hint counter before
+                // reading their inputs; clear: they read and validate the inputs at once
+                // (the inputs carry their own readiness)
   float* part;  // attention partials [8][Hkv][S][rep][d + 2]
   int2* lm_part;  // [n_sm][8] best (value bits, index) per SM
   uint16_t* kcache;
@@ -291,7 +292,7 @@ struct Spin {
         return false;
       }
     }
-    if (it > 4) __nanosleep(64);
+    if (it > 64) __nanosleep(32);
     return true;
   }
 };
@@ -1623,7 +1624,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
       rec[0] = (long long)I.op | ((long long)I.layer << 8) | ((long long)I.n_units << 24);
       rec[1] = (long long)globaltimer_ns();
     }
-    if (ct == 0 && I.dep != kNoCounter && p.hints) {
+    if (ct == 0 && I.dep != kNoCounter && ((p.hints >> I.op) & 1)) {
       // hint: every warp of a matvec instruction bumps its counter, attention once
       // per (lane, kv head); counters only grow within a launch
       const uint32_t per = I.op == OP_O ? 1u : (uint32_t)kConsumerWarps;
