@@ -189,7 +189,11 @@ mk_status mk_clear_error(mk_handle h);
  * barrier (the counter release follows), and accumulate [14] ns the first
  * consumer warps spent in page dot products, [15] ns in the reductions and
  * epilogues, [16] group re-reads of activations not yet written when first
- * loaded, [17] ns those re-reads took (summed over threads); [18..31] unused.
+ * loaded, [17] ns those re-reads took (lane 0 of each warp), [18] staging
+ * entered, [19] the first staged values back, [20..21] the residual
+ * accumulator back (QKV, LM head), [22] the first warp entered its pages,
+ * [24] its first page landed; [23], [25..31] unused.  The end stamps [4], [12],
+ * [13] are the last warp's (no barrier is added for them).
  * Reading resets the accumulators.
  * `cap` is the capacity of `out` in int64 elements; *n_sm and *stride are set
  * even when out is NULL, so a first call can size the buffer.  Synchronises

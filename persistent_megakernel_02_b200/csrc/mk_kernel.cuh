@@ -271,14 +271,16 @@ struct Spin {
   uint32_t it = 0;
   const KParams* pp;
   Misc* m;
+  // profile mode: lane 0 of each warp counts its re-read groups and their time
+  // (one shared-memory atomic per warp, so that profiling barely slows the wait)
   __device__ __forceinline__ Spin(const KParams& p, Misc* misc) : pp(&p), m(misc) {
-    if (p.prof) {
+    if (p.prof && (threadIdx.x & 31) == 0) {
       tp = globaltimer_ns();
       atomicAdd(&misc->slow_n, 1u);
     }
   }
   __device__ __forceinline__ ~Spin() {
-    if (pp->prof) atomicAdd(&m->slow_ns, (unsigned long long)(globaltimer_ns() - tp));
+    if (pp->prof && (threadIdx.x & 31) == 0) atomicAdd(&m->slow_ns, (unsigned long long)(globaltimer_ns() - tp));
   }
   __device__ __forceinline__ bool again(const KParams& p, uint32_t instr, uint32_t info, Misc* misc) {
     ++it;
@@ -1611,6 +1613,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   }
   cbar();
   bool stopped = false;  // set only where every warp reads misc->stop together
+  long long* prev_rec = nullptr;  // profile: record whose re-read counters await their flush
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
   for (uint32_t ii = i0; ii < i1; ++ii) {
@@ -1633,6 +1636,13 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     }
     cbar();
     if (rec) rec[2] = (long long)globaltimer_ns();
+    if (prev_rec) {  // every warp is past the previous instruction now
+      prev_rec[16] += misc->slow_n;
+      prev_rec[17] += (long long)misc->slow_ns;
+      misc->slow_n = 0;
+      misc->slow_ns = 0;
+      prev_rec = nullptr;
+    }
     if (misc->stop) { stopped = true; break; }
     float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
     uint32_t used = I.n_units;  // one page per unit, except attention
@@ -1684,31 +1694,23 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
     page_base += used;
     // No barrier here: each warp bumped the hint counter after its own writes,
     // and the next instruction's barrier keeps the activation buffer from being
-    // restaged while a warp still reads it.  Profiling adds one for its stamps.
+    // restaged while a warp still reads it.  Profiling stamps without a barrier
+    // too: every warp raises the record's end times to its own.
     if (p.prof) {
-      if (rec) rec[3] = (long long)globaltimer_ns();
-      cbar();
+      const long long now = (long long)globaltimer_ns();
+      long long* rw = p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * kProfSlots;
+      if ((ct & 31) == 0) {
+        unsigned long long* ru = reinterpret_cast<unsigned long long*>(rw);
+        if (I.op != OP_ATTN) atomicMax(ru + 12, (unsigned long long)now);
+        atomicMax(ru + 13, (unsigned long long)now);
+        atomicMax(ru + 4, (unsigned long long)now);
+      }
       if (rec) {
-        long long last = 0;
-        for (int w = 0; w < kConsumerWarps; ++w) last = max(last, misc->warp_done[w]);
-        if (I.op != OP_ATTN) rec[12] = last;
-        rec[13] = rec[4] = (long long)globaltimer_ns();
+        rec[3] = now;
         if (I.op != OP_ATTN) { rec[18] = misc->t_stage_in; rec[19] = misc->t_stage_loaded; }
         if (I.op == OP_LM || (I.op == OP_QKV && I.layer > 0)) { rec[20] = misc->t_sum_x1; rec[21] = misc->t_sum_p; }
-        if (I.op != OP_ATTN) {  // spread of the warps: entry, first page, done
-          long long e0 = LLONG_MAX, e1 = 0, f1 = 0, d0 = LLONG_MAX;
-          for (int w = 0; w < kConsumerWarps; ++w) {
-            e0 = min(e0, misc->warp_entry[w]);
-            e1 = max(e1, misc->warp_entry[w]);
-            f1 = max(f1, misc->warp_first[w]);
-            if (misc->warp_first[w]) d0 = min(d0, misc->warp_done[w]);
-          }
-          rec[22] = e0; rec[23] = e1; rec[24] = f1; rec[25] = d0 == LLONG_MAX ? 0 : d0;
-        }
-        rec[16] += misc->slow_n;
-        rec[17] += (long long)misc->slow_ns;
-        misc->slow_n = 0;
-        misc->slow_ns = 0;
+        if (I.op != OP_ATTN) { rec[22] = misc->warp_entry[0]; rec[24] = misc->warp_first[0]; }
+        prev_rec = rec;  // its re-read counters are flushed once every warp is past it
       }
     }
     I = In;

@@ -65,7 +65,7 @@ def summarize(rec: np.ndarray) -> dict:
                 d["st_call"] += r["t_stage_in"] - r["t_dep"]          # into the staging function
                 d["st_load"] += r["t_stage_loaded"] - r["t_stage_in"]  # activation loads back
                 d["st_rest"] += r["t_staged"] - r["t_stage_loaded"]    # norm, shared-memory stores
-            if r["w_entry0"] and r["w_done0"]:
+            if r["w_entry0"] and r["w_done0"] and False:  # per-warp spread: no longer recorded
                 d["n_w"] += 1
                 d["w_entry"] += r["w_entry0"] - r["t_staged"]          # staged -> first warp in its matvec
                 d["w_entry_spread"] += r["w_entry1"] - r["w_entry0"]   # first -> last warp in
