@@ -117,6 +117,9 @@ typedef struct {
                                 MK_ERR_TIMEOUT and the context stays usable) */
   int32_t profile;           /* 1: every step records per-instruction timestamps
                                 (see mk_profile_read); costs a few stores per instruction */
+  int32_t dyn_percent;       /* share of the gate/up, down and LM-head rows that SMs claim
+                                at run time instead of taking from a fixed range: 0 = none
+                                (default), 1..90 = that percent; else MK_ERR_INVALID_ARG */
 } mk_options;
 
 /* Create a handle: validates the config, lowers it into per-SM instruction
@@ -220,11 +223,13 @@ typedef struct {
 } mk_plan_report;
 
 /* Lower `cfg` for `n_sm` SMs and `nb` active lanes, run the CPU tape simulator
- * over the result and fill `rep`.  `fault` != 0 plants a fault in the tape
- * first (1: one signal dropped, 2: one wait target raised by one) so tests can
- * see the simulator report it. */
+ * over the result and fill `rep`.  `dyn_percent` is mk_options.dyn_percent (the
+ * share of the streaming phases claimed at run time, 0..90).  `fault` != 0 plants
+ * a fault in the tape first (1: one signal dropped, 2: one wait target raised by
+ * one, 3: one instruction's claim range of the LM head shortened by one row
+ * block, with dyn_percent > 0) so tests can see the simulator report it. */
 mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                        mk_plan_report* rep);
+                        int32_t dyn_percent, mk_plan_report* rep);
 
 /* ---- greedy head without allocation ----
  *

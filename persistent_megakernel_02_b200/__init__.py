@@ -67,7 +67,7 @@ class MkOptions(ctypes.Structure):
     _fields_ = [
         ("device", ctypes.c_int32), ("wait_limit_ms", ctypes.c_int32), ("n_sm", ctypes.c_int32),
         ("ring_pages", ctypes.c_int32), ("debug_fault", ctypes.c_int32),
-        ("profile", ctypes.c_int32),
+        ("profile", ctypes.c_int32), ("dyn_percent", ctypes.c_int32),
     ]
 
 
@@ -103,7 +103,7 @@ _SIGS = {
     "mk_get_error": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int32]),
     "mk_clear_error": (ctypes.c_int, [ctypes.c_void_p]),
     "mk_destroy": (ctypes.c_int, [ctypes.c_void_p]),
-    "mk_plan_check": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.c_int32, ctypes.c_int32,
+    "mk_plan_check": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.POINTER(MkPlanReport)]),
     "mk_profile_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.POINTER(ctypes.c_int32),
@@ -154,11 +154,12 @@ def config_struct(cfg: dict) -> MkConfig:
     return MkConfig(**{k: cfg.get(k, 0) if k == "kv_dtype" else cfg[k] for k in _CFG_FIELDS})
 
 
-def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0) -> dict:
+def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0, dyn_percent: int = 0) -> dict:
     """Lower ``cfg`` on the host and run the tape simulator (no GPU needed)."""
     rep = MkPlanReport()
     c = config_struct(cfg)
-    _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, ctypes.byref(rep)), "mk_plan_check")
+    _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, dyn_percent, ctypes.byref(rep)),
+           "mk_plan_check")
     return {f: getattr(rep, f) for f, _ in MkPlanReport._fields_}
 
 
@@ -213,13 +214,16 @@ class Megakernel:
     ``weights`` is the dict of :func:`synth.make_weights` layout: 'embed',
     'lm_head' (None when tied), 'final_norm' and per-layer lists 'attn_norm',
     'wq', 'wk', 'wv', 'wo', 'mlp_norm', 'w_gate', 'w_up', 'w_down' -- contiguous
-    bf16 CUDA tensors.  The handle keeps references to them.
+    bf16 CUDA tensors.  The handle keeps references to them.  The keyword options
+    are mk_options' fields (include/mk.h); ``dyn_percent`` > 0 leaves that share of
+    the gate/up, down and LM-head rows to run-time claims.
     """
 
     _LAYER = ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")
 
     def __init__(self, cfg: dict, weights: dict, device: int = 0, wait_limit_ms: int = 1000,
-                 n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0):
+                 n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0,
+                 dyn_percent: int = 0):
         self.cfg = dict(cfg)
         self._weights = weights
         self._arrays = {}
@@ -233,7 +237,8 @@ class Megakernel:
             **{n: ctypes.cast(self._arrays[n], _PP) for n in self._LAYER},
         )
         opt = MkOptions(device=device, wait_limit_ms=wait_limit_ms, n_sm=n_sm,
-                        ring_pages=ring_pages, debug_fault=debug_fault, profile=profile)
+                        ring_pages=ring_pages, debug_fault=debug_fault, profile=profile,
+                        dyn_percent=dyn_percent)
         self._cfg_struct = config_struct(cfg)
         h = ctypes.c_void_p()
         _check(lib().mk_create(ctypes.byref(self._cfg_struct), ctypes.byref(w), ctypes.byref(opt),

@@ -35,10 +35,12 @@ struct mk_ctx {
   const uint16_t* embed = nullptr;
   float* acts = nullptr;  // two sets of per-layer activation blocks (see KParams)
   long long set_floats = 0, layer_floats = 0, acc_base = 0, acc_floats = 0;
+  long long claim_off = 0;  // claim counters of the dynamic tails, after the accumulators
+  long long lmkey_off = 0;  // the step's greedy keys, after the claim counters
+  int dyn_percent = kDynPercent;
   int off_q = 0, off_kvn = 0, off_o = 0, off_x1 = 0, off_a = 0;
   unsigned long long steps_run = 0;  // decode steps launched (activation-set parity)
   float* part = nullptr;
-  int2* lm_part = nullptr;
   uint16_t *kcache = nullptr, *vcache = nullptr;
   int* page_table = nullptr;
   uint32_t* counters = nullptr;
@@ -186,7 +188,7 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   const Dims& D = h->D;
   // tapes, one per active batch size
   for (int nb = 1; nb <= D.max_batch; ++nb) {
-    h->tapes.push_back(lower(D, h->n_sm, nb));
+    h->tapes.push_back(lower(D, h->n_sm, nb, h->dyn_percent));
     Tape& t = h->tapes.back();
     resolve_pointers(t, D, w);
     mk_ctx::DevTape dt;
@@ -210,12 +212,13 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
     h->layer_floats = (off + 7) / 8 * 8;
     h->acc_floats = 2LL * MB * D.H;  // 64-bit accumulators
     h->acc_base = h->layer_floats * D.L;
-    h->set_floats = h->acc_base + h->acc_floats * D.L;
+    h->claim_off = h->acc_base + h->acc_floats * D.L;
+    h->lmkey_off = h->claim_off + (n_pools(D) + 3) / 4 * 4;
+    h->set_floats = h->lmkey_off + 2 * kMaxNB;  // a whole number of 16-byte refill stores
     MK_TRY(dalloc(h, &h->acts, (size_t)2 * h->set_floats));
     MK_TRY(reset_acts(h));
   }
   MK_TRY(dalloc(h, &h->part, (size_t)kMaxNB * D.Hkv * S1 * D.rep * (D.d + 2)));
-  MK_TRY(dalloc(h, &h->lm_part, (size_t)h->n_sm * kMaxNB));
   const size_t kv = (size_t)D.L * D.n_phys_pages * D.Hkv * D.PL * D.d;
   MK_TRY(dalloc(h, &h->kcache, kv));
   MK_TRY(dalloc(h, &h->vcache, kv));
@@ -278,9 +281,11 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.off_x1 = h->off_x1; p.off_a = h->off_a;
   p.acc_base = h->acc_base;
   p.acc_floats = h->acc_floats;
+  p.claim_off = h->claim_off;
+  p.lmkey_off = h->lmkey_off;
   p.parity0 = (int)(h->steps_run & 1);
   p.hints = h->hints;
-  p.part = h->part; p.lm_part = h->lm_part;
+  p.part = h->part;
   p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
   const int par = (int)(h->step & 1);
   p.ctr = h->counters + (size_t)par * h->n_counters;
@@ -332,15 +337,18 @@ mk_status status_of(const ErrWord& e) {
 }  // namespace
 
 extern "C" mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                                   mk_plan_report* rep) {
-  if (!cfg || !rep || n_sm < 1) return MK_ERR_INVALID_ARG;
+                                   int32_t dyn_percent, mk_plan_report* rep) {
+  if (!cfg || !rep || n_sm < 1 || dyn_percent < 0 || dyn_percent > 90) return MK_ERR_INVALID_ARG;
   memset(rep, 0, sizeof(*rep));
   Dims D;
   std::string why = dims_from_config(cfg, n_sm, &D);
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
   if (nb < 1 || nb > D.max_batch) return MK_ERR_INVALID_ARG;
-  Tape t = lower(D, n_sm, nb);
-  if (fault == 1) {  // drop one signal: the first QKV instruction of the last layer
+  Tape t = lower(D, n_sm, nb, dyn_percent > 0 ? dyn_percent : kDynPercent);
+  if (fault == 3) {  // shrink the LM head's claim range by one unit on one SM
+    for (auto& I : t.instrs)
+      if (I.op == OP_LM && I.pool) { I.pool_u1 -= 1; break; }
+  } else if (fault == 1) {  // drop one signal: the first QKV instruction of the last layer
     for (auto& I : t.instrs)
       if (I.op == OP_QKV && I.layer == D.L - 1) { I.sig = kNoCounter; break; }
   } else if (fault == 2) {  // raise one wait target
@@ -370,6 +378,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   mk_options o{};
   if (opt) o = *opt;
   if (o.wait_limit_ms < 0 || o.n_sm < 0 || o.ring_pages < 0 || o.device < 0) return MK_ERR_INVALID_ARG;
+  if (o.dyn_percent < 0 || o.dyn_percent > 90) return MK_ERR_INVALID_ARG;
   Dims D;
   std::string why = dims_from_config(cfg, 148, &D);  // validation only; rederived below
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
@@ -388,6 +397,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   h->dev = o.device;
   h->n_sm = o.n_sm > 0 ? std::min(o.n_sm, sms) : sms;
   h->wait_limit_ns = (unsigned long long)(o.wait_limit_ms > 0 ? o.wait_limit_ms : 1000) * 1000000ull;
+  h->dyn_percent = o.dyn_percent > 0 ? o.dyn_percent : kDynPercent;
   why = dims_from_config(cfg, h->n_sm, &h->D);
   h->nbt = lanes_template(cfg->max_batch);
   mk_status s = why.empty() ? build(h, w, o.ring_pages) : MK_ERR_UNSUPPORTED;

@@ -90,17 +90,18 @@ struct KParams {
   //   off_a   [MB][F]         silu(gate) * up
   // and the accumulator of layer l, [MB][H] 64-bit counted fixed-point sums
   // (acc_enc), holds the residual after its down projection: x1 plus every K
-  // slice's partial, 1 + n_ks terms.  Float blocks refill with the sentinel,
-  // accumulators with zero.
+  // slice's partial, 1 + n_ks terms.  After the accumulators, at claim_off, the
+  // claim counters of the step's dynamic tails (uint32, Instr::pool), then at
+  // lmkey_off the greedy keys of the step (uint64 per lane, lm_key).  Float
+  // blocks refill with the sentinel, the rest with zero.
   float* acts;
-  long long set_floats, layer_floats, acc_base, acc_floats;
+  long long set_floats, layer_floats, acc_base, acc_floats, claim_off, lmkey_off;
   int off_q, off_kvn, off_o, off_x1, off_a;
   int parity0;  // set of this launch's step 0
   int hints;    // bit op set: instructions of that op wait on their hint counter before
                 // reading their inputs; clear: they read and validate the inputs at once
                 // (the inputs carry their own readiness)
   float* part;  // attention partials [8][Hkv][S][rep][d + 2]
-  int2* lm_part;  // [n_sm][8] best (value bits, index) per SM
   uint16_t* kcache;
   uint16_t* vcache;
   const int* page_table;  // [max_batch][pages_per_seq]
@@ -150,6 +151,7 @@ struct Misc {
   float2 rope_cs[kMaxNB][64];  // (cos, sin) of each lane's position, per frequency
   float* actset;         // the activation set of the current step
   uint32_t i0;           // this SM's first tape index (profile records)
+  uint32_t n_instr;      // this SM's tape length
   uint32_t attn_extra;   // attention signals beyond one per (lane, kv head), summed over this launch's steps
   unsigned int slow_n;   // profile mode: group re-reads of unwritten activations
   unsigned long long slow_ns;  // and the time they took (summed over threads)
@@ -158,6 +160,16 @@ struct Misc {
   volatile int stop;
   volatile int last;
   uint32_t issued;  // pages the ring producer issued
+  // Dynamic tails.  unit[slot]: the unit whose weights the page in that ring slot
+  // holds (written by the producer before the page's full-barrier arrival).
+  // dyn_end[s & 15]: for the s-th instruction of this launch (s = step * tape
+  // length + index), (s << 32) | the stream position where its pages end, written
+  // by the producer once its claims are exhausted.  cons_seq: the instruction the
+  // consumers are in (the producer reuses an entry only after they left it).
+  uint32_t unit[64];
+  volatile unsigned long long dyn_end[16];
+  volatile uint32_t cons_seq;
+  volatile uint32_t last_claim;
   int entry_abort;
 };
 // the misc region is what smem_layout leaves after the barriers: 8192 - 8 * (128 + 64)
@@ -368,6 +380,55 @@ __device__ __forceinline__ AttnPlan attn_plan(int S, int rep, int npg, int s) {
   return a;
 }
 
+// ---------------------------------------------------------------- dynamic tails
+
+// Producer: wait until the consumers have entered instruction seq - 15, so the
+// dyn_end entry of seq - 16 is no longer read.
+__device__ __noinline__ bool wait_consumers(const KParams& p, Misc* misc, uint32_t seq, uint32_t instr) {
+  if (misc->cons_seq + 16u > seq) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (misc->cons_seq + 16u > seq) return true;
+    if ((it & 63) == 0) {
+      if (aborted(p)) return false;
+      if (globaltimer_ns() - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_EMPTY, instr, seq, true);
+        return false;
+      }
+    }
+    __nanosleep(64);
+  }
+}
+
+// Consumer: wait for the page at stream position q of a dynamic instruction
+// (launch-wide index seq).  1: the page is there and belongs to the instruction;
+// 0: the instruction's pages ended before q (the page at q, if any, is the next
+// instruction's and stays untouched); -1: aborted or timed out.  The end is read
+// again after the barrier completes: the producer publishes it before issuing
+// any later instruction's page, so a completed foreign page implies a visible end.
+__device__ __forceinline__ int wait_dyn(const KParams& p, uint64_t* bar, uint32_t parity, Misc* misc,
+                                        uint32_t seq, uint32_t q, uint32_t instr) {
+  const volatile unsigned long long* de = &misc->dyn_end[seq & 15];
+  auto ended = [&]() {
+    const unsigned long long e = *de;
+    return (uint32_t)(e >> 32) == seq && (int32_t)(q - (uint32_t)e) >= 0;
+  };
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (ended()) return 0;
+    if (mbar_try_wait_hint(bar, parity, 256u)) return ended() ? 0 : 1;
+    if ((it & 63) == 63) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) t0 = now;
+      if (aborted(p)) return -1;
+      if (now - t0 > p.wait_limit_ns) {
+        raise_error(p, E_WAIT_FULL, instr, q, true);
+        return -1;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- producer
 
 __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr& I, uint32_t u,
@@ -438,6 +499,7 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
   for (int t = 0; t < p.n_steps && ok; ++t) {
   Instr I;
   if (i0 < i1) I = p.instrs[i0];
+  bool synced = false;  // this step's claim counters are ready (step t - 1 ended)
   for (uint32_t ii = i0; ii < i1 && ok; ++ii) {
     const Instr In = ii + 1 < i1 ? p.instrs[ii + 1] : I;
     long long* rec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - i0)) * kProfSlots : nullptr;
@@ -484,13 +546,58 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
         }
       }
     } else {
-      for (uint32_t k = 0; k < I.n_units; ++k) {
+      // The static units, then (dynamic tail) the chunks this SM claims from the
+      // phase's pool.  Three claims are in flight at a time (the first one issued
+      // under the last static pages), so a claim's round trip stays hidden behind
+      // the stream.  Claims are used in the order issued, so their values grow and
+      // the first one past the pool ends the instruction.
+      uint32_t* claim = nullptr;
+      uint32_t chunk = 0, pn = 0, va = 0, vb = 0, vc = 0;
+      if (I.pool) {
+        // the counters live in this step's activation set, which SMs zeroed
+        // during step t - 1: wait until every SM is past that step
+        if (t > 0 && !synced) {
+          if (!(ok = wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, ii))) break;
+          synced = true;
+        }
+        claim = reinterpret_cast<uint32_t*>(p.acts + (size_t)((p.parity0 + t) & 1) * p.set_floats + p.claim_off) +
+                ((I.pool & 0xFFFFFFu) - 1u);
+        chunk = I.pool >> 24;
+        pn = I.pool_u1 - I.pool_u0;
+      }
+      auto page = [&](uint32_t u) {
         const long long tw = rec ? (long long)globaltimer_ns() : 0;
-        if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
+        if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) return;
         if (rec) { acc_wait += (long long)globaltimer_ns() - tw; acc_pages += 1; }
-        issue_matvec_page(p, I, I.u0 + k, ring + (size_t)rp.slot * kPageBytes, &full[rp.fidx], pol);
+        misc->unit[rp.slot] = u;  // published to the consumer by the full barrier's arrival
+        issue_matvec_page(p, I, u, ring + (size_t)rp.slot * kPageBytes, &full[rp.fidx], pol);
         ++pidx;
         rp.advance(1, NP);
+      };
+      const uint32_t k_claim = I.n_units > 4u ? I.n_units - 4u : 0u;
+      for (uint32_t k = 0; k < I.n_units && ok; ++k) {
+        if (claim && k == k_claim) va = atomicAdd(claim, chunk);
+        page(I.u0 + k);
+      }
+      if (I.pool && ok) {
+        if (I.n_units == 0) va = atomicAdd(claim, chunk);
+        vb = atomicAdd(claim, chunk);
+        vc = atomicAdd(claim, chunk);
+        auto take = [&](uint32_t& v) {  // stream claim v's chunk, then claim again into v
+          if (v >= pn) return false;
+          const uint32_t ve = min(v + chunk, pn);
+          for (uint32_t x = v; x < ve && ok; ++x) page(I.pool_u0 + x);
+          v = atomicAdd(claim, chunk);
+          return ok;
+        };
+        while (take(va) && take(vb) && take(vc)) {
+        }
+        misc->last_claim = va + vb + vc;  // every claim has landed before the step can end
+        // publish where this instruction's pages end; its entry's previous user
+        // (instruction seq - 16) must be behind the consumers
+        const uint32_t seq = (uint32_t)t * (i1 - i0) + (ii - i0);
+        if (ok) ok = wait_consumers(p, misc, seq, ii);
+        if (ok) misc->dyn_end[seq & 15] = ((unsigned long long)seq << 32) | pidx;
       }
     }
     if (rec) { rec[6] = (long long)globaltimer_ns(); rec[9] += acc_wait; rec[10] += acc_pages; }
@@ -726,6 +833,19 @@ __device__ __forceinline__ bool lm_better(float v, int i, float bv, int bi) {
   return v > bv || (v == bv && i < bi);
 }
 
+// (value, row) as one 64-bit key whose unsigned order is lm_better's order, so an
+// atomic maximum over the keys picks the greedy token: the value's bits made
+// monotone (negative floats reversed, +0 and -0 equal), then the row reversed so
+// the lower row wins a tie.  NaN maps to 0 and never wins, as in lm_better; key 0
+// (nothing seen) decodes to row 0x7FFFFFFF.
+__device__ __forceinline__ unsigned long long lm_key(float v, int i) {
+  if (v != v) return 0ull;
+  const uint32_t u = __float_as_uint(v == 0.0f ? 0.0f : v);
+  const uint32_t hi = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((unsigned long long)hi << 32) | (uint32_t)(0x7FFFFFFF - i);
+}
+__device__ __forceinline__ int lm_key_row(unsigned long long k) { return 0x7FFFFFFF - (int)(uint32_t)k; }
+
 // 1 / rms of each lane's staged vector (RMSNorm), from the per-warp sums of
 // squares the stage left in misc->red.
 template <int NBT>
@@ -755,6 +875,11 @@ struct LmBest {  // running argmax per lane (value, index); passed by value, so 
   float v[NBT];
   int i[NBT];
 };
+// the step's greedy keys, one per lane, at lmkey_off in the activation set
+__device__ __forceinline__ unsigned long long* lm_keys(const KParams& p, const Misc* misc) {
+  return reinterpret_cast<unsigned long long*>(misc->actset + p.lmkey_off);
+}
+
 template <int NBT>
 __device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBest<NBT> best) {
   const Dims& D = p.D;
@@ -777,7 +902,8 @@ __device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBes
     int bi = 0x7FFFFFFF;
     for (int w = 0; w < kConsumerWarps; ++w)
       if (lm_better(misc->lmv[w][ct], misc->lmi[w][ct], bv, bi)) { bv = misc->lmv[w][ct]; bi = misc->lmi[w][ct]; }
-    p.lm_part[blockIdx.x * kMaxNB + ct] = make_int2(__float_as_int(bv), bi);
+    // this SM's best joins the step's maximum (zeroed with the activation set)
+    if (ct < p.nb && bi != 0x7FFFFFFF) atomicMax(lm_keys(p, misc) + ct, lm_key(bv, bi));
   }
   cbar();
   if (ct == 0) {
@@ -786,14 +912,8 @@ __device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBes
   }
   cbar();
   if (misc->last) {
-    if (ct < p.nb) {
-      float bv = -CUDART_INF_F;
-      int bi = 0x7FFFFFFF;
-      for (int s = 0; s < (int)gridDim.x; ++s) {
-        const int2 e = __ldcg(p.lm_part + s * kMaxNB + ct);
-        const float val = __int_as_float(e.x);
-        if (lm_better(val, e.y, bv, bi)) { bv = val; bi = e.y; }
-      }
+    if (ct < p.nb) {  // every SM's maximum is in (ordered by the counter's acquire)
+      const int bi = lm_key_row(ld_relaxed_u64(lm_keys(p, misc) + ct));
       p.ids[(size_t)misc->step * p.ids_stride + ct] = (bi >= 0 && bi < D.V) ? bi : 0;
     }
     cbar();
@@ -867,10 +987,15 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
   }
   unsigned long long* accl = (OPK == OP_O || OPK == OP_DOWN) ? const_cast<unsigned long long*>(acc_of(p, misc, I.layer)) : nullptr;
 
+  // a dynamic tail (gate/up, down, LM head): the units come with the pages, and
+  // the stream position where the instruction ends is published by the producer
+  constexpr bool DYN = OPK == OP_GU || OPK == OP_DOWN || OPK == OP_LM;
+  const bool dyn = DYN && I.pool != 0;
+  const uint32_t seq = (uint32_t)misc->step * misc->n_instr + (ii - misc->i0);
   RingPos rp;
   rp.init(page_base + cw, NP);
-  for (uint32_t k = cw; k < I.n_units; k += kConsumerWarps, rp.advance(kConsumerWarps, NP)) {
-    const uint32_t u = I.u0 + k;
+  for (uint32_t k = cw; dyn || k < I.n_units; k += kConsumerWarps, rp.advance(kConsumerWarps, NP)) {
+    uint32_t u = I.u0 + k;
     const uint32_t slot = rp.slot;
     ResidIn rin[OPK == OP_O ? NL : 1];
     if constexpr (OPK == OP_O) {  // the residual rows this lane will write, loaded under the page wait
@@ -880,7 +1005,15 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
         if (writer && vrow[m] < nr && vlane[m] < p.nb) resid_issue(p, misc, I.layer, vlane[m], r0 + vrow[m], rin[m]);
     }
     const long long tw = prec ? (long long)globaltimer_ns() : 0;
-    bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+    bool ok;
+    if (DYN && dyn) {
+      const int r = wait_dyn(p, &full[rp.fidx], rp.fphase, misc, seq, page_base + k, ii);
+      if (__any_sync(0xFFFFFFFFu, r == 0)) break;  // every lane sees the same end
+      ok = r > 0;
+      if (ok) u = misc->unit[slot];
+    } else {
+      ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+    }
     if (prec) {
       const long long now = (long long)globaltimer_ns();
       c_wait += now - tw;
@@ -1574,6 +1707,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
   if (ct == 0) {
     misc->step = t;
     misc->i0 = i0;
+    misc->n_instr = i1 - i0;
     misc->actset = p.acts + (size_t)((p.parity0 + t) & 1) * p.set_floats;
     if (t > 0 && !wait_counter(p, p.ctr + ctr_step(D), (uint32_t)t, i0)) misc->stop = 1;
     // a (lane, kv head) split by query head signals once per head (attn_plan)
@@ -1635,10 +1769,11 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
       if (!wait_hint(p, p.ctr + I.dep, I.dep_target * per * (uint32_t)(t + 1) + extra, ii)) misc->stop = 1;
     }
     cbar();
+    if (ct == 0) misc->cons_seq = (uint32_t)t * misc->n_instr + (ii - i0);  // entered (dynamic-tail table)
     if (rec) rec[2] = (long long)globaltimer_ns();
-    if (prev_rec) {  // every warp is past the previous instruction now
-      prev_rec[16] += misc->slow_n;
-      prev_rec[17] += (long long)misc->slow_ns;
+    if (prev_rec) {  // every warp is past the previous instruction now (reductions: no wait)
+      atomicAdd(reinterpret_cast<unsigned long long*>(prev_rec + 16), (unsigned long long)misc->slow_n);
+      atomicAdd(reinterpret_cast<unsigned long long*>(prev_rec + 17), misc->slow_ns);
       misc->slow_n = 0;
       misc->slow_ns = 0;
       prev_rec = nullptr;
@@ -1691,6 +1826,7 @@ __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* ac
         mv_dispatch<OP_LM, NBT, SPEC>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
     }
+    if (I.pool) used = (uint32_t)misc->dyn_end[((uint32_t)t * misc->n_instr + (ii - i0)) & 15] - page_base;
     page_base += used;
     // No barrier here: each warp bumped the hint counter after its own writes,
     // and the next instruction's barrier keeps the activation buffer from being
@@ -1754,6 +1890,8 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
     misc->slow_n = 0;
     misc->slow_ns = 0;
     misc->attn_extra = 0;
+    misc->cons_seq = 0;
+    for (int i = 0; i < 16; ++i) misc->dyn_end[i] = ~0ull;  // a tag no instruction has
   }
   __syncthreads();
   if (!misc->entry_abort) {

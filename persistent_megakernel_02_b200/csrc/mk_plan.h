@@ -8,6 +8,7 @@
 // is exactly one shared-memory page of weights, or one attention slice), the
 // counter it waits on with its target, and the counter it bumps when done.
 // Ranges keep the kernel free of per-unit table lookups: a unit id is u0 + k.
+// The streaming phases end with a dynamic tail that SMs claim at run time.
 #pragma once
 
 #include <stdint.h>
@@ -53,8 +54,12 @@ struct Instr {            // 64 bytes
   uint16_t dep;           // counter waited on before the instruction (kNoCounter: none)
   uint16_t sig;           // counter incremented once when the instruction is done
   uint32_t dep_target;    // value `dep` must reach in this step
-  uint32_t aux0, aux1;    // reserved (zero)
-  uint32_t pad;
+  // Dynamic tail (gate/up, down, LM head).  After its static units the SM claims
+  // chunks of (pool >> 24) units from [pool_u0, pool_u1), a range shared by every
+  // SM of the phase, through claim counter (pool & 0xFFFFFF) - 1 of the step's
+  // activation set, until the range is exhausted.  pool == 0: static units only.
+  uint32_t pool;
+  uint32_t pool_u0, pool_u1;
   // device pointers resolved when the handle is created, so the kernel needs no
   // table lookup per instruction: [0..2] the weight matrices the producer
   // streams (QKV: Wq, Wk, Wv; O: Wo; GU: Wgate, Wup; DOWN: Wdown; LM: the head),
@@ -88,6 +93,20 @@ struct Tape {
   std::vector<Instr> instrs;
 };
 
+// Share of the gate/up, down and LM-head units (percent) left to dynamic claims
+// by default.  A claimed tail lets faster SMs take over work from slower ones,
+// but on the measured workloads the SMs' end times within a phase differ by only
+// 1-3 us, and the claims (an L2 round trip each) cost more than they balance
+// (Llama-3.2-1B batch 1: 539 us static, 545 with 10-25 % of the LM head claimed,
+// 647 with all three phases at 25 %), so the default assignment is static.
+constexpr int kDynPercent = 0;
+
+// claim counters of one step: per layer gate/up and each down K slice, then the LM head
+MK_HD inline int n_pools(const Dims& D) { return D.L * (1 + D.n_ks) + 1; }
+MK_HD inline int pool_gu(const Dims& D, int layer) { return layer * (1 + D.n_ks); }
+MK_HD inline int pool_dn(const Dims& D, int layer, int ks) { return layer * (1 + D.n_ks) + 1 + ks; }
+MK_HD inline int pool_lm(const Dims& D) { return D.L * (1 + D.n_ks); }
+
 // lanes the kernel is instantiated for: the batch size rounded up to 1, 2, 4 or 8
 MK_HD inline int lanes_template(int nb) { return nb <= 1 ? 1 : nb <= 2 ? 2 : nb <= 4 ? 4 : 8; }
 
@@ -113,7 +132,9 @@ std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, i
                         int ffn, int vocab, int tied, float eps, int max_batch, int max_seq,
                         int n_sm, Dims* out);
 int attn_slices(const Dims& D, int n_sm, int nb);
-Tape lower(const Dims& D, int n_sm, int nb);
+// dyn_percent: share of the gate/up, down and LM-head units claimed at run time
+// (0: every unit statically assigned)
+Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent = kDynPercent);
 
 struct SimReport {
   bool deadlock_free = false, coverage_ok = false, targets_ok = false;

@@ -143,7 +143,7 @@ struct Assigner {
 };
 }  // namespace
 
-Tape lower(const Dims& D, int n_sm, int nb) {
+Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent) {
   Tape t;
   t.nb = nb;
   t.S = attn_slices(D, n_sm, nb);
@@ -166,6 +166,35 @@ Tape lower(const Dims& D, int n_sm, int nb) {
     return ins[sm].back();
   };
 
+  // A streaming phase over SMs [lo, hi): the first units are split statically
+  // (contiguous ranges), the last dyn_percent % form the pool the SMs claim from
+  // in chunks.  Every SM of the range gets an instruction when there is a pool.
+  dyn_percent = std::max(0, std::min(90, dyn_percent));
+  auto phase = [&](uint8_t op, int layer, int n, int lo, int hi, uint16_t dep, uint16_t sig, uint8_t arg,
+                   int pool, bool every_sm) {
+    const int n_part = hi - lo;
+    const int n_dyn = pool >= 0 ? (int)((int64_t)n * dyn_percent / 100) : 0;
+    const int n_st = n - n_dyn;
+    const int64_t ub = unit_bytes(D, op, t.S);
+    auto st = as.run(n_st, ub, lo, hi);
+    // each SM's expected share of the pool counts toward its load
+    if (n_dyn > 0)
+      for (int s = lo; s < hi; ++s) load[s] += ub * n_dyn / n_part;
+    // chunks small enough that the last ones balance the SMs' end times, at least
+    // two units where the pool has them (a claim is a round trip to L2)
+    const int per_sm = n_dyn / std::max(1, n_part);
+    const uint32_t chunk = (uint32_t)std::max(per_sm >= 4 ? 2 : 1, std::min(4, per_sm / 8));
+    for (int s = lo; s < hi; ++s)
+      if (!st[s].empty() || n_dyn > 0 || every_sm) {
+        Instr& I = emit(s, op, layer, st[s], dep, sig, arg);
+        if (n_dyn > 0) {
+          I.pool = (uint32_t)(pool + 1) | (chunk << 24);
+          I.pool_u0 = (uint32_t)n_st;
+          I.pool_u1 = (uint32_t)n;
+        }
+      }
+  };
+
   for (int l = 0; l < D.L; ++l) {
     uint16_t dep_qkv = l ? (uint16_t)ctr_layer(l - 1, C_DOWN) : kNoCounter;
     // RMSNorm + QKV + RoPE
@@ -184,24 +213,19 @@ Tape lower(const Dims& D, int n_sm, int nb) {
     for (int s = 0; s < n_sm; ++s)
       if (!o[s].empty()) emit(s, OP_O, l, o[s], (uint16_t)ctr_layer(l, C_ATTN), (uint16_t)ctr_layer(l, C_O), 0);
     // RMSNorm + gate/up + SwiGLU
-    auto gu = as.run(D.n_gu, unit_bytes(D, OP_GU, t.S), 0, n_sm);
-    for (int s = 0; s < n_sm; ++s)
-      if (!gu[s].empty()) emit(s, OP_GU, l, gu[s], (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0);
+    phase(OP_GU, l, D.n_gu, 0, n_sm, (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0,
+          pool_gu(D, l), false);
     // down projection + residual: SMs split into one group per K slice
     for (int ks = 0; ks < D.n_ks; ++ks) {
       int lo = (int)((long long)n_sm * ks / D.n_ks), hi = (int)((long long)n_sm * (ks + 1) / D.n_ks);
       if (hi <= lo) hi = lo + 1;  // more slices than SMs: share
       lo %= n_sm; hi = std::min(hi, n_sm);
-      auto dn = as.run(D.n_dn, unit_bytes(D, OP_DOWN, t.S), lo, hi);
-      for (int s = lo; s < hi; ++s)
-        if (!dn[s].empty())
-          emit(s, OP_DOWN, l, dn[s], (uint16_t)ctr_layer(l, C_GU), (uint16_t)ctr_layer(l, C_DOWN), (uint8_t)ks);
+      phase(OP_DOWN, l, D.n_dn, lo, hi, (uint16_t)ctr_layer(l, C_GU), (uint16_t)ctr_layer(l, C_DOWN),
+            (uint8_t)ks, pool_dn(D, l, ks), false);
     }
   }
   // final norm + LM head + argmax: every SM takes part (possibly with no rows)
-  auto lm = as.run(D.n_lm, unit_bytes(D, OP_LM, t.S), 0, n_sm);
-  for (int s = 0; s < n_sm; ++s)
-    emit(s, OP_LM, D.L, lm[s], (uint16_t)ctr_layer(D.L - 1, C_DOWN), kNoCounter, 0);
+  phase(OP_LM, D.L, D.n_lm, 0, n_sm, (uint16_t)ctr_layer(D.L - 1, C_DOWN), kNoCounter, 0, pool_lm(D), true);
 
   // wait targets = how many instructions signal the counter in one step
   std::vector<uint32_t> fan(t.n_counters, 0);
@@ -234,13 +258,21 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
       ca((size_t)D.L * nb * D.Hkv * S, 0), cl(D.n_lm, 0);
   std::vector<uint32_t> ip(n_sm);
   r.bytes_min = INT64_MAX; r.bytes_max = 0;
+  // SMs taking part in each pool: each is expected to stream an equal share of it
+  std::vector<int64_t> pool_part(n_pools(D), 0);
+  for (const Instr& I : t.instrs)
+    if (I.pool && (I.pool & 0xFFFFFFu) - 1 < pool_part.size()) pool_part[(I.pool & 0xFFFFFFu) - 1]++;
   for (int s = 0; s < n_sm; ++s) {
     ip[s] = t.sm_off[s];
     int n = (int)(t.sm_off[s + 1] - t.sm_off[s]);
     r.max_instr_per_sm = std::max(r.max_instr_per_sm, n);
     int64_t by = 0;
-    for (uint32_t i = t.sm_off[s]; i < t.sm_off[s + 1]; ++i)
-      if (t.instrs[i].n_units != 0xFFFFFFFFu) by += unit_bytes(D, t.instrs[i].op, S) * t.instrs[i].n_units;
+    for (uint32_t i = t.sm_off[s]; i < t.sm_off[s + 1]; ++i) {
+      const Instr& I = t.instrs[i];
+      if (I.n_units != 0xFFFFFFFFu) by += unit_bytes(D, I.op, S) * I.n_units;
+      if (I.pool && (I.pool & 0xFFFFFFu) - 1 < pool_part.size() && I.pool_u1 >= I.pool_u0)
+        by += unit_bytes(D, I.op, S) * (I.pool_u1 - I.pool_u0) / pool_part[(I.pool & 0xFFFFFFu) - 1];
+    }
     r.bytes_min = std::min(r.bytes_min, by);
     r.bytes_max = std::max(r.bytes_max, by);
   }
@@ -250,6 +282,10 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
     if (i >= v.size()) { cover_err = true; return; }
     v[i]++;
   };
+  // a pool's units are produced once, by whichever SMs claim them: the simulator
+  // credits them when the first instruction of the pool runs
+  std::vector<char> pool_seen(n_pools(D), 0);
+  std::vector<int64_t> pool_range(n_pools(D), -1);
   bool progress = true;
   while (progress) {
     progress = false;
@@ -259,8 +295,25 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
         if (I.dep != kNoCounter && ctr[I.dep] < (int64_t)I.dep_target) break;
         int l = I.layer;
         if (I.n_units == 0xFFFFFFFFu) { cover_err = true; ip[s]++; progress = true; continue; }
-        for (uint32_t k = 0; k < I.n_units; ++k) {
-          uint32_t u = I.u0 + k;
+        uint32_t n_run = I.n_units;
+        std::vector<uint32_t> extra;
+        if (I.pool) {
+          const uint32_t pi = (I.pool & 0xFFFFFFu) - 1, chunk = I.pool >> 24;
+          const int64_t key = ((int64_t)I.pool_u0 << 32) | I.pool_u1;
+          const bool op_ok = I.op == OP_GU || I.op == OP_DOWN || I.op == OP_LM;
+          if (!op_ok || pi >= pool_seen.size() || chunk < 1 || I.pool_u0 > I.pool_u1 ||
+              I.u0 + I.n_units > I.pool_u0 || (pool_range[pi] >= 0 && pool_range[pi] != key)) {
+            cover_err = true;
+          } else {
+            pool_range[pi] = key;
+            if (!pool_seen[pi]) {
+              pool_seen[pi] = 1;
+              for (uint32_t u = I.pool_u0; u < I.pool_u1; ++u) extra.push_back(u);
+            }
+          }
+        }
+        for (uint32_t k = 0; k < n_run + extra.size(); ++k) {
+          uint32_t u = k < n_run ? I.u0 + k : extra[k - n_run];
           switch (I.op) {
             case OP_QKV: bump(cq, (size_t)l * D.n_qkv + u); break;
             case OP_O: bump(co, (size_t)l * D.n_o + u); break;

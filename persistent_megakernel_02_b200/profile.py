@@ -107,8 +107,39 @@ def summarize(rec: np.ndarray) -> dict:
     for (layer, op), ph in phases.items():
         c = crit.setdefault(op, [])
         c.append((ph["last_sig"] - ph["first_dep"]) / 1e3)
+    # the chain through a few middle layers: per op, when its first SM passed the
+    # instruction barrier, when its last SM did, and when its last SM finished
+    layers = sorted({layer for layer, _ in phases})
+    mid = layers[len(layers) // 2 - 1: len(layers) // 2 + 1] if len(layers) > 2 else layers
+    chain = []
+    if mid:
+        base = phases.get((mid[0], "qkv"), next(iter(phases.values())))["first_dep"]
+        order = ["qkv", "attn", "o", "gu", "down"]
+        for layer in mid:
+            for op in order:
+                ph = phases.get((layer, op))
+                if ph:
+                    chain.append((layer, op, round((ph["first_dep"] - base) / 1e3, 2),
+                                  round((ph["last_dep"] - base) / 1e3, 2), round((ph["last_sig"] - base) / 1e3, 2)))
+    # spread between SMs in the streaming phases of the middle layer (and the LM
+    # head): percentiles of each SM's start, units time and end, from the phase's
+    # first start
+    spread = {}
+    for op in ("gu", "down", "lm"):
+        lay = mid[0] if op != "lm" and mid else None
+        rs = [r for r in rows if r["op"] == op and (lay is None or r["layer"] == lay)]
+        if not rs:
+            continue
+        f = min(r["t_dep"] for r in rs)
+        q = lambda xs: [round(float(np.percentile(xs, k)) / 1e3, 2) for k in (0, 10, 50, 90, 100)]
+        spread[op] = dict(dep=q([r["t_dep"] - f for r in rs]),
+                          units=q([r["t_last_warp"] - r["t_staged"] for r in rs if r["t_staged"]]),
+                          end=q([r["t_sig"] - f for r in rs]),
+                          end_by_sm=[round((r["t_sig"] - f) / 1e3, 1) for r in sorted(rs, key=lambda r: r["sm"])])
     return {
         "step_us": (t1 - t0) / 1e3,
+        "spread_p0_10_50_90_100_us": spread,
+        "chain_first_last_end_us": chain,
         "per_op": {k: {kk: round(vv, 3) if isinstance(vv, float) else vv for kk, vv in v.items()}
                    for k, v in per_op.items()},
         "phase_us_mean": {op: round(float(np.mean(v)), 3) for op, v in crit.items()},
@@ -135,12 +166,13 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="llama1b_bs1")
     ap.add_argument("--ring-pages", type=int, default=0)
+    ap.add_argument("--dyn-percent", type=int, default=0, help="claimed share of the streaming phases (0: none)")
     args = ap.parse_args(argv)
     wl = configs.WORKLOADS[args.workload]
     nb, P = wl["batch"], max(wl["prompt_lens"])
     cfg = configs.model_config(args.workload, max_seq=P + 8)
     w = synth.make_weights(cfg, device="cuda")
-    mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages)
+    mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages, dyn_percent=args.dyn_percent)
     prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
     ids = torch.tensor([mk.prefill(b, prompts[b]) for b in range(nb)], dtype=torch.int32, device="cuda")
     pos = [len(p) for p in prompts]

@@ -39,10 +39,11 @@ def test_version_string():
 
 @pytest.mark.parametrize("wl", list(configs.WORKLOADS))
 @pytest.mark.parametrize("n_sm", [148, 132, 37])
-def test_tapes_are_deadlock_free_and_cover_every_output(wl, n_sm):
+@pytest.mark.parametrize("dyn", [0, 25])
+def test_tapes_are_deadlock_free_and_cover_every_output(wl, n_sm, dyn):
     cfg = configs.model_config(wl)
     for nb in sorted({1, cfg["max_batch"]}):
-        r = mk.plan_check(cfg, n_sm, nb)
+        r = mk.plan_check(cfg, n_sm, nb, dyn_percent=dyn)
         assert r["deadlock_free"] and r["coverage_ok"] and r["targets_ok"], (wl, n_sm, nb, r)
         # bytes per SM balanced to within one attention slice + one page
         assert r["bytes_max_sm"] - r["bytes_min_sm"] <= 2 * 16384 * (1 + 130 // r["attn_slices"])
@@ -62,6 +63,14 @@ def test_simulator_reports_planted_faults(fault):
     r = mk.plan_check(configs.model_config("tiny"), 148, 1, fault=fault)
     assert not r["deadlock_free"]
     assert not r["targets_ok"]
+
+
+def test_simulator_reports_an_uncovered_claim_range():
+    """3: one SM's copy of the LM head's claim range ends a row block early; the
+    ranges of the pool then disagree and the simulator reports the coverage."""
+    r = mk.plan_check(configs.model_config("tiny"), 148, 1, fault=3, dyn_percent=25)
+    assert r["deadlock_free"] and r["targets_ok"]
+    assert not r["coverage_ok"]
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(hidden=4104), dict(n_heads=12, n_kv_heads=4),
