@@ -124,7 +124,11 @@ typedef struct {
 
 /* Create a handle: validates the config, lowers it into per-SM instruction
  * tapes (one set per active batch size 1..max_batch), allocates the KV cache
- * (bf16, pages of 16 KiB per layer and kv head) and scratch, zeroes them.
+ * (bf16, pages of 16 KiB per layer and kv head) and scratch, zeroes them, and
+ * copies the QKV, gate/up and down matrices into device buffers of its own in
+ * the order the kernel streams them (each 16 KiB page one contiguous block; the
+ * handle then holds a second copy of those matrices, e.g. 1.8 GB for the
+ * Llama-3.2-1B shape).
  * Returns MK_ERR_INVALID_ARG / MK_ERR_UNSUPPORTED before touching the GPU when
  * the config or pointers are bad. */
 mk_status mk_create(const mk_config* cfg, const mk_weights* w, const mk_options* opt,

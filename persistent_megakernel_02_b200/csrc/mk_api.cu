@@ -43,6 +43,9 @@ struct mk_ctx {
   float* part = nullptr;
   uint16_t *kcache = nullptr, *vcache = nullptr;
   int* page_table = nullptr;
+  // the layer matrices in page order (pack_weights): every unit's page is one
+  // contiguous 16 KiB block, so the producer moves it with a single bulk copy
+  uint16_t *pk_qkv = nullptr, *pk_gu = nullptr, *pk_dn = nullptr;
   uint32_t* counters = nullptr;
   int n_counters = 0;
   ErrWord* err = nullptr;
@@ -154,17 +157,92 @@ mk_status check_weights(const mk_config* c, const mk_weights* w) {
   return MK_OK;
 }
 
+// Packed-layer sizes (elements per layer).
+size_t pk_qkv_elems(const Dims& D) { return (size_t)D.n_qkv * 2 * D.RP * D.H; }
+size_t pk_gu_elems(const Dims& D) { return (size_t)D.n_gu * 2 * D.Rgu * D.H; }
+size_t pk_dn_elems(const Dims& D) { return (size_t)D.n_ks * D.H * D.KS; }
+
+// Copies row r (row_u4 16-byte words) from src[r], or zeros where src[r] is null,
+// to dst + r * row_u4.
+__global__ void pack_rows_kernel(const uint4* const* src, uint4* dst, long long n_rows, int row_u4) {
+  const long long n = n_rows * row_u4;
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const long long r = e / row_u4;
+    const uint4* s = src[r];
+    dst[e] = s ? s[e - r * row_u4] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+mk_status pack_rows(const std::vector<const void*>& rows, void* dst, int row_bytes) {
+  const uint4** d_src = nullptr;
+  MK_TRY(from_cuda(cudaMalloc(&d_src, rows.size() * sizeof(void*))));
+  cudaError_t e = cudaMemcpy(d_src, rows.data(), rows.size() * sizeof(void*), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) {
+    pack_rows_kernel<<<1184, 256>>>(d_src, static_cast<uint4*>(dst), (long long)rows.size(), row_bytes / 16);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(d_src);
+  return from_cuda(e);
+}
+
+// Lay the layer matrices out in the order the producer streams them, one unit
+// after another, each unit one contiguous page:
+//   QKV   unit u: the RP rows of its RoPE first halves, then the RP second halves
+//   GU    unit u: Rgu rows of W_gate, then the same Rgu rows of W_up (rows past
+//         ffn in a ragged last unit are zero)
+//   DOWN  K slice ks, rows r: W_down[r][ks*KS .. ks*KS + KS), slices one after
+//         another, so the Rdn rows of a unit are adjacent
+// A page made of several strided pieces streamed measurably slower than one
+// contiguous block (Llama-3.2-1B batch 1: 538 vs 463 us per step).
+mk_status pack_weights(mk_ctx* h, const mk_weights* w) {
+  const Dims& D = h->D;
+  const int half = D.d / 2;
+  MK_TRY(dalloc(h, &h->pk_qkv, pk_qkv_elems(D) * D.L));
+  MK_TRY(dalloc(h, &h->pk_gu, pk_gu_elems(D) * D.L));
+  MK_TRY(dalloc(h, &h->pk_dn, pk_dn_elems(D) * D.L));
+  const size_t rowH = (size_t)D.H;
+  std::vector<const void*> rows;
+  for (int l = 0; l < D.L; ++l)
+    for (int u = 0; u < D.n_qkv; ++u) {
+      const int P0 = u * D.RP, hg = P0 / half, i0 = P0 % half;
+      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
+      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
+      const uint16_t* m = static_cast<const uint16_t*>(sec == 0 ? w->wq[l] : sec == 1 ? w->wk[l] : w->wv[l]);
+      for (int hf = 0; hf < 2; ++hf)
+        for (int j = 0; j < D.RP; ++j) rows.push_back(m + ((size_t)hh * D.d + i0 + hf * half + j) * rowH);
+    }
+  MK_TRY(pack_rows(rows, h->pk_qkv, D.H * 2));
+  rows.clear();
+  for (int l = 0; l < D.L; ++l)
+    for (int u = 0; u < D.n_gu; ++u)
+      for (int m = 0; m < 2; ++m)
+        for (int j = 0; j < D.Rgu; ++j) {
+          const int r = u * D.Rgu + j;
+          const uint16_t* src = static_cast<const uint16_t*>(m == 0 ? w->w_gate[l] : w->w_up[l]);
+          rows.push_back(r < D.F ? src + (size_t)r * rowH : nullptr);
+        }
+  MK_TRY(pack_rows(rows, h->pk_gu, D.H * 2));
+  rows.clear();
+  for (int l = 0; l < D.L; ++l)
+    for (int ks = 0; ks < D.n_ks; ++ks)
+      for (int r = 0; r < D.H; ++r)
+        rows.push_back(static_cast<const uint16_t*>(w->w_down[l]) + (size_t)r * D.F + (size_t)ks * D.KS);
+  MK_TRY(pack_rows(rows, h->pk_dn, D.KS * 2));
+  return MK_OK;
+}
+
 // Resolve the device pointers each instruction streams from (see Instr::ptr).
-void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w) {
+void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w, const mk_ctx* h) {
   const void* lm = D.tied ? w->embed : w->lm_head;
   for (Instr& I : t.instrs) {
     const int l = I.layer;
     I.ptr[0] = I.ptr[1] = I.ptr[2] = I.ptr[3] = nullptr;
     switch (I.op) {
-      case OP_QKV: I.ptr[0] = w->wq[l]; I.ptr[1] = w->wk[l]; I.ptr[2] = w->wv[l]; I.ptr[3] = w->attn_norm[l]; break;
+      case OP_QKV: I.ptr[0] = h->pk_qkv + pk_qkv_elems(D) * l; I.ptr[3] = w->attn_norm[l]; break;
       case OP_O: I.ptr[0] = w->wo[l]; break;
-      case OP_GU: I.ptr[0] = w->w_gate[l]; I.ptr[1] = w->w_up[l]; I.ptr[3] = w->mlp_norm[l]; break;
-      case OP_DOWN: I.ptr[0] = w->w_down[l]; break;
+      case OP_GU: I.ptr[0] = h->pk_gu + pk_gu_elems(D) * l; I.ptr[3] = w->mlp_norm[l]; break;
+      case OP_DOWN: I.ptr[0] = h->pk_dn + pk_dn_elems(D) * l; break;
       case OP_LM: I.ptr[0] = lm; I.ptr[3] = w->final_norm; break;
       default: break;
     }
@@ -186,11 +264,12 @@ const void* kernel_for(int nbt, int spec) {
 
 mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   const Dims& D = h->D;
+  MK_TRY(pack_weights(h, w));
   // tapes, one per active batch size
   for (int nb = 1; nb <= D.max_batch; ++nb) {
     h->tapes.push_back(lower(D, h->n_sm, nb, h->dyn_percent));
     Tape& t = h->tapes.back();
-    resolve_pointers(t, D, w);
+    resolve_pointers(t, D, w, h);
     mk_ctx::DevTape dt;
     MK_TRY(dalloc(h, &dt.instrs, t.instrs.size()));
     MK_TRY(dalloc(h, &dt.sm_off, t.sm_off.size()));

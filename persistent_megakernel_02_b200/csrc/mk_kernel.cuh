@@ -435,17 +435,10 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
                                                   uint8_t* dst, uint64_t* bar, uint64_t pol) {
   const Dims& D = p.D;
   switch (I.op) {
-    case OP_QKV: {
-      const int half = D.d / 2;
-      const int P0 = (int)u * D.RP, hg = P0 / half, i0 = P0 % half;
-      const int sec = hg < D.Hq ? 0 : (hg < D.Hq + D.Hkv ? 1 : 2);
-      const int hh = sec == 0 ? hg : (sec == 1 ? hg - D.Hq : hg - D.Hq - D.Hkv);
-      const uint16_t* w = static_cast<const uint16_t*>(I.ptr[sec]);
-      const size_t r0 = (size_t)hh * D.d + i0;
-      const uint32_t bytes = (uint32_t)D.RP * D.H * 2;
-      mbar_arrive_expect_tx(bar, 2 * bytes);
-      bulk_g2s(dst, w + r0 * D.H, bytes, bar, pol);
-      bulk_g2s(dst + bytes, w + (r0 + half) * D.H, bytes, bar, pol);
+    case OP_QKV: {  // packed: the unit's RP first-half rows, then its RP second-half rows
+      const uint32_t bytes = (uint32_t)(2 * D.RP) * D.H * 2;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)u * (2 * D.RP) * D.H, bytes, bar, pol);
       break;
     }
     case OP_O: {
@@ -455,21 +448,18 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
       bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)r0 * D.qdim, bytes, bar, pol);
       break;
     }
-    case OP_GU: {
-      const int r0 = (int)u * D.Rgu, nr = min(D.Rgu, D.F - r0);
-      const uint32_t bytes = (uint32_t)nr * D.H * 2;
-      mbar_arrive_expect_tx(bar, 2 * bytes);
-      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)r0 * D.H, bytes, bar, pol);
-      bulk_g2s(dst + (size_t)D.Rgu * D.H * 2, static_cast<const uint16_t*>(I.ptr[1]) + (size_t)r0 * D.H,
-               bytes, bar, pol);
+    case OP_GU: {  // packed: Rgu gate rows, then the same Rgu up rows (zero past ffn)
+      const uint32_t bytes = (uint32_t)(2 * D.Rgu) * D.H * 2;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, static_cast<const uint16_t*>(I.ptr[0]) + (size_t)u * (2 * D.Rgu) * D.H, bytes, bar, pol);
       break;
     }
-    case OP_DOWN: {
+    case OP_DOWN: {  // packed K-slice major: the unit's rows of slice I.arg are adjacent
       const int r0 = (int)u * D.Rdn, nr = min(D.Rdn, D.H - r0);
-      const uint32_t rb = (uint32_t)D.KS * 2;
-      const uint16_t* w = static_cast<const uint16_t*>(I.ptr[0]) + (size_t)I.arg * D.KS;
-      mbar_arrive_expect_tx(bar, nr * rb);
-      for (int r = 0; r < nr; ++r) bulk_g2s(dst + r * rb, w + (size_t)(r0 + r) * D.F, rb, bar, pol);
+      const uint32_t bytes = (uint32_t)nr * D.KS * 2;
+      const uint16_t* w = static_cast<const uint16_t*>(I.ptr[0]) + ((size_t)I.arg * D.H + r0) * D.KS;
+      mbar_arrive_expect_tx(bar, bytes);
+      bulk_g2s(dst, w, bytes, bar, pol);
       break;
     }
     case OP_LM: {

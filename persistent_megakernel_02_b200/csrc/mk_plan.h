@@ -61,9 +61,10 @@ struct Instr {            // 64 bytes
   uint32_t pool;
   uint32_t pool_u0, pool_u1;
   // device pointers resolved when the handle is created, so the kernel needs no
-  // table lookup per instruction: [0..2] the weight matrices the producer
-  // streams (QKV: Wq, Wk, Wv; O: Wo; GU: Wgate, Wup; DOWN: Wdown; LM: the head),
-  // [3] the bf16 RMSNorm gain the consumers stage with (QKV, GU, LM)
+  // table lookup per instruction: [0] the weights the producer streams (QKV, GU,
+  // DOWN: the layer's packed matrix, every unit one contiguous page; O: Wo; LM:
+  // the head), [1..2] unused, [3] the bf16 RMSNorm gain the consumers stage with
+  // (QKV, GU, LM)
   const void* ptr[4];
 };
 static_assert(sizeof(Instr) == 64, "Instr layout");

@@ -167,10 +167,13 @@ def main(argv=None):
     ap.add_argument("--workload", default="llama1b_bs1")
     ap.add_argument("--ring-pages", type=int, default=0)
     ap.add_argument("--dyn-percent", type=int, default=0, help="claimed share of the streaming phases (0: none)")
+    ap.add_argument("--max-seq-extra", type=int, default=181,
+                    help="max_seq = prompt + this (181: bench.py's default sizing, which sets the "
+                         "attention slices per kv head)")
     args = ap.parse_args(argv)
     wl = configs.WORKLOADS[args.workload]
     nb, P = wl["batch"], max(wl["prompt_lens"])
-    cfg = configs.model_config(args.workload, max_seq=P + 8)
+    cfg = configs.model_config(args.workload, max_seq=P + max(8, args.max_seq_extra))
     w = synth.make_weights(cfg, device="cuda")
     mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages, dyn_percent=args.dyn_percent)
     prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
