@@ -41,7 +41,7 @@ struct mk_ctx {
   int off_q = 0, off_kvn = 0, off_o = 0, off_x1 = 0, off_a = 0;
   unsigned long long steps_run = 0;  // decode steps launched (activation-set parity)
   float* part = nullptr;
-  uint16_t *kcache = nullptr, *vcache = nullptr;
+  uint16_t* kv = nullptr;  // [layer][physical page][kv head][K, V][PL][d]
   int* page_table = nullptr;
   // the layer matrices in page order (pack_weights): every unit's page is one
   // contiguous 16 KiB block, so the producer moves it with a single bulk copy
@@ -299,8 +299,7 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   }
   MK_TRY(dalloc(h, &h->part, (size_t)kMaxNB * D.Hkv * S1 * D.rep * (D.d + 2)));
   const size_t kv = (size_t)D.L * D.n_phys_pages * D.Hkv * D.PL * D.d;
-  MK_TRY(dalloc(h, &h->kcache, kv));
-  MK_TRY(dalloc(h, &h->vcache, kv));
+  MK_TRY(dalloc(h, &h->kv, 2 * kv));
   std::vector<int> pt((size_t)D.max_batch * D.pages_per_seq);
   for (size_t i = 0; i < pt.size(); ++i) pt[i] = (int)i;  // slot s owns pages s*pps .. s*pps+pps-1
   MK_TRY(dalloc(h, &h->page_table, pt.size()));
@@ -365,7 +364,7 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   p.parity0 = (int)(h->steps_run & 1);
   p.hints = h->hints;
   p.part = h->part;
-  p.kcache = h->kcache; p.vcache = h->vcache; p.page_table = h->page_table;
+  p.kv = h->kv; p.page_table = h->page_table;
   const int par = (int)(h->step & 1);
   p.ctr = h->counters + (size_t)par * h->n_counters;
   p.ctr_next = h->counters + (size_t)(1 - par) * h->n_counters;

@@ -102,8 +102,9 @@ struct KParams {
                 // reading their inputs; clear: they read and validate the inputs at once
                 // (the inputs carry their own readiness)
   float* part;  // attention partials [8][Hkv][S][rep][d + 2]
-  uint16_t* kcache;
-  uint16_t* vcache;
+  // KV cache [layer][physical page][kv head][K, V][PL][d]: a page's K and V are
+  // one contiguous 16 KiB block
+  uint16_t* kv;
   const int* page_table;  // [max_batch][pages_per_seq]
   uint32_t* ctr;          // counters of this step
   uint32_t* ctr_next;     // counters of the next step (zeroed here)
@@ -522,12 +523,18 @@ __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t*
           const int n_old = min(D.PL, pos - j * D.PL);
           uint64_t* fb = &full[rp.fidx];
           if (n_old > 0) {
-            const size_t base = (((size_t)I.layer * D.n_phys_pages + phys) * D.Hkv + g) * (size_t)(D.PL * D.d);
-            const uint32_t bytes = (uint32_t)n_old * D.d * 2;
+            const size_t kvp = (size_t)D.PL * D.d;  // elements of one page's K (or V)
+            const uint16_t* src = p.kv + (((size_t)I.layer * D.n_phys_pages + phys) * D.Hkv + g) * 2 * kvp;
             uint8_t* dst = ring + (size_t)rp.slot * kPageBytes;
-            mbar_arrive_expect_tx(fb, 2 * bytes);
-            bulk_g2s(dst, p.kcache + base, bytes, fb, pol);
-            bulk_g2s(dst + (size_t)D.PL * D.d * 2, p.vcache + base, bytes, fb, pol);
+            if (n_old == D.PL) {  // a full page: K and V in one copy
+              mbar_arrive_expect_tx(fb, (uint32_t)(4 * kvp));
+              bulk_g2s(dst, src, (uint32_t)(4 * kvp), fb, pol);
+            } else {  // the written positions of K, then of V
+              const uint32_t bytes = (uint32_t)n_old * D.d * 2;
+              mbar_arrive_expect_tx(fb, 2 * bytes);
+              bulk_g2s(dst, src, bytes, fb, pol);
+              bulk_g2s(dst + 2 * kvp, src + kvp, bytes, fb, pol);
+            }
           } else {
             mbar_arrive(fb);
           }
@@ -1070,11 +1077,10 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
             st_relaxed_f32(qq + i + half, canon(r2));
           } else {
             // the cache row serves later steps; this step's attention reads the fp32 copy
-            const size_t idx = (((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) *
-                                   (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
-            uint16_t* cache = sec == 1 ? p.kcache : p.vcache;
-            cache[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
-            cache[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
+            const size_t idx = ((((size_t)I.layer * D.n_phys_pages + misc->cur_phys[b]) * D.Hkv + hh) * 2 +
+                                (sec - 1)) * (size_t)(D.PL * D.d) + (size_t)(pos % D.PL) * D.d + i;
+            p.kv[idx] = D.kv_fp16 ? f2h(r1) : f2bf(r1);
+            p.kv[idx + half] = D.kv_fp16 ? f2h(r2) : f2bf(r2);
             float* kv = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + (sec - 1) * D.kvdim + hh * D.d;
             st_relaxed_f32(kv + i, canon(r1));
             st_relaxed_f32(kv + i + half, canon(r2));

@@ -373,10 +373,18 @@ SmemLayout smem_layout(const Dims& D, int nb_max, int max_dyn_smem, int want_pag
   attn = std::max(attn, (D.d + 256 + 16 + 512) * 4);
   s.act_bytes = (std::max(act, attn) + 1023) / 1024 * 1024;
   int misc = 8192;  // mbarriers (128 full + 64 empty), reduction scratch, step constants
-  // Prefer a ring that fits the 196 KiB shared-memory carveout: the larger L1
-  // left beside it measured faster than a deeper ring in the 228 KiB carveout.
+  // Ring depth against L1: for a model streamed from HBM (weights larger than
+  // L2) with a small activation region (10 KiB: one lane of a 2048-wide model, or
+  // its attention scratch) the deepest ring that fits measured fastest
+  // (Llama-3.2-1B batch 1: 13 pages 462 us, 11 pages 469; 8192-token context 738
+  // vs 747).  Otherwise a ring fitted to the 196 KiB carveout, which leaves a
+  // larger L1, measured faster (batch 4, 32 KiB: 974 vs 998 us; 8B batch 1,
+  // 19 KiB: 3309 vs 3373; an L2-resident 256-wide model: 44 vs 62).
+  const int64_t layer_w = 2LL * D.H * (D.qdim + 2 * D.kvdim) + 2LL * D.qdim * D.H + 6LL * D.H * D.F;
+  const int64_t weights = layer_w * D.L + 2LL * D.V * D.H;
+  const bool deep = s.act_bytes <= 12 * 1024 && weights > (128LL << 20);
   const int kCarveout196 = 196 * 1024 - 1024;  // minus the per-CTA reserved KiB
-  int cap = std::min(max_dyn_smem, kCarveout196);
+  int cap = deep ? max_dyn_smem : std::min(max_dyn_smem, kCarveout196);
   int np = std::min(64, (cap - s.act_bytes - misc) / kPageBytes);
   if (np < kConsumerWarps) np = std::min(64, (max_dyn_smem - s.act_bytes - misc) / kPageBytes);
   // the ring protocol needs at least one page per consumer warp
