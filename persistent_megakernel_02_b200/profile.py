@@ -65,12 +65,10 @@ def summarize(rec: np.ndarray) -> dict:
                 d["st_call"] += r["t_stage_in"] - r["t_dep"]          # into the staging function
                 d["st_load"] += r["t_stage_loaded"] - r["t_stage_in"]  # activation loads back
                 d["st_rest"] += r["t_staged"] - r["t_stage_loaded"]    # norm, shared-memory stores
-            if r["w_entry0"] and r["w_done0"] and False:  # per-warp spread: no longer recorded
+            if r["w_entry0"] and r["w_first1"]:  # warp 0 of the consumers
                 d["n_w"] += 1
-                d["w_entry"] += r["w_entry0"] - r["t_staged"]          # staged -> first warp in its matvec
-                d["w_entry_spread"] += r["w_entry1"] - r["w_entry0"]   # first -> last warp in
-                d["w_first"] += r["w_first1"] - r["w_entry0"]          # -> last warp's first page ready
-                d["w_done_first"] += r["w_done0"] - r["w_entry0"]      # -> first warp done
+                d["w_entry"] += r["w_entry0"] - r["t_staged"]          # staged -> warp 0 in its matvec
+                d["w_first"] += r["w_first1"] - r["w_entry0"]          # -> its first page ready
             if r["t_sum_x1"] and r["t_stage_in"]:
                 d["n_sum"] += 1
                 d["sum_x1"] += r["t_sum_x1"] - r["t_stage_in"]     # residual x1 back
