@@ -50,6 +50,18 @@ def test_tapes_are_deadlock_free_and_cover_every_output(wl, n_sm, dyn):
         assert r["ring_pages"] >= 8
 
 
+def test_ring_depth_follows_the_measured_rule():
+    """The deepest ring that fits (228 KiB carveout) only for HBM-streamed shapes with
+    a small activation region (the 1B shape at batch 1); the 196 KiB carveout for
+    the rest (batch 4 and 8, the 8B shape, an L2-resident model)."""
+    want = {"llama1b_bs1": 13, "llama1b_long": 13, "llama1b_bs4": 9, "llama1b_bs8": 9,
+            "llama8b_bs1": 10, "tiny": 11}
+    for wl, pages in want.items():
+        r = mk.plan_check(configs.model_config(wl), 148, 1)
+        assert r["ring_pages"] == pages, (wl, r["ring_pages"])
+        assert r["smem_bytes"] <= 232448
+
+
 def test_ragged_shapes_lower_cleanly():
     cfg = configs.model_config("tiny", vocab=4099, ffn=1000, max_batch=3, max_seq=77)
     for nb in (1, 2, 3):
