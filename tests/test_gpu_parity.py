@@ -216,6 +216,37 @@ def test_dynamic_tails_give_the_static_logits_bit_for_bit():
     np.testing.assert_array_equal(runs[0][2], runs[1][2])
 
 
+def test_greedy_ties_take_the_lowest_row_across_sms():
+    """Exact ties in the LM head: with every row identical all logits are equal and
+    the greedy id is row 0; with the first half of the rows negated, the winner is
+    row 0 or the first row of the second half (whichever half has the larger
+    logit), rows that other SMs stream."""
+    cfg = configs.model_config("tiny", tied=0, max_seq=32)
+    w = H.gpu_weights(cfg)
+    V = cfg["vocab"]
+    row = w["lm_head"][17].clone()
+    w["lm_head"][:] = row
+    prompt = synth.prompt_tokens(cfg, 0, 6).tolist()
+    lg = torch.empty(V, dtype=torch.float32, device="cuda")
+    mk = _mk(cfg, w)
+    first = mk.prefill(0, prompt, logits_last=lg)
+    mk.sync()
+    mk.close()
+    vals = lg.cpu().numpy()
+    assert np.all(vals == vals[0]), "identical rows must give identical logits"
+    assert first == 0
+    m = V // 2 + 3
+    w["lm_head"][:m] = -row
+    mk = _mk(cfg, w)
+    first = mk.prefill(0, prompt, logits_last=lg)
+    mk.sync()
+    mk.close()
+    vals = lg.cpu().numpy()
+    want = m if vals[m] > vals[0] else 0
+    assert vals[0] != vals[m]
+    assert first == want, (first, want, vals[0], vals[m])
+
+
 def test_multi_step_launch_across_the_attention_mode_threshold():
     """Contexts of at most 4 KV pages use single-head attention units, longer ones
     split the pages over slices and merge; one multi-step launch over positions
