@@ -146,6 +146,42 @@ def summarize(rec: np.ndarray) -> dict:
     }
 
 
+def markdown(s: dict, bench_us: float | None = None) -> str:
+    """The summary of one profiled step as the tables of a text report: per-op
+    means, the chain through the middle layers, the per-SM spread."""
+    po, ph = s["per_op"], s["phase_us_mean"]
+    out = []
+    note = f" (bench without stamps: {bench_us:.1f} us)" if bench_us else ""
+    out.append(f"Step in profile mode: {s['step_us']:.1f} us{note}.")
+    out.append("")
+    out.append("| op | window | barrier wait | stage | entry | first page | pages | dot/page | "
+               "epilogue/page | page wait/page | slot wait/page | pages/SM |")
+    out.append("|---|---|---|---|---|---|---|---|---|---|---|---|")
+    for op in ("qkv", "attn", "o", "gu", "down", "lm"):
+        if op not in po:
+            continue
+        d = po[op]
+        if op == "attn":
+            out.append(f"| attn | {ph.get('attn', 0):.2f} | {d['wait_us_mean']:.2f} | - | - | - | "
+                       f"{d['work_us_mean']:.2f} (work) | - | - | - | - | - |")
+            continue
+        out.append(f"| {op} | {ph.get(op, 0):.2f} | {d['wait_us_mean']:.2f} | {d['stage_us_mean']:.2f} | "
+                   f"{d['w_entry_us_mean']:.2f} | {d['w_first_us_mean']:.2f} | {d['units_us_mean']:.2f} | "
+                   f"{d['c_core_us_per_page']:.2f} | {d['c_epi_us_per_page']:.2f} | "
+                   f"{d['c_wait_us_per_page']:.2f} | {d['p_wait_us_per_page']:.2f} | "
+                   f"{d['pages_per_instr_mean']:.2f} |")
+    out.append("")
+    out.append("| layer | op | first start | last start | last end |")
+    out.append("|---|---|---|---|---|")
+    for layer, op, a, b, c in s["chain_first_last_end_us"]:
+        out.append(f"| {layer} | {op} | {a} | {b} | {c} |")
+    out.append("")
+    sp = s["spread_p0_10_50_90_100_us"]
+    out.append("Spread between SMs (percentiles 0/10/50/90/100 of each SM's end, from the phase's "
+               "first start): " + "; ".join(f"{op} {sp[op]['end']}" for op in sp) + ".")
+    return "\n".join(out) + "\n"
+
+
 def main(argv=None):
     """Profile one steady-state decode step of a workload and print its breakdown.
 
@@ -163,12 +199,19 @@ def main(argv=None):
 
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default="llama1b_bs1")
+    ap.add_argument("--markdown", action="store_true", help="print the report tables instead of JSON")
+    ap.add_argument("--from-json", default=None, help="render a saved JSON summary (no GPU)")
     ap.add_argument("--ring-pages", type=int, default=0)
     ap.add_argument("--dyn-percent", type=int, default=0, help="claimed share of the streaming phases (0: none)")
     ap.add_argument("--max-seq-extra", type=int, default=181,
                     help="max_seq = prompt + this (181: bench.py's default sizing, which sets the "
                          "attention slices per kv head)")
     args = ap.parse_args(argv)
+    if args.from_json:
+        with open(args.from_json) as f:
+            saved = json.load(f)
+        print(markdown(saved) if args.markdown else json.dumps(saved, indent=1))
+        return
     wl = configs.WORKLOADS[args.workload]
     nb, P = wl["batch"], max(wl["prompt_lens"])
     cfg = configs.model_config(args.workload, max_seq=P + max(8, args.max_seq_extra))
@@ -185,7 +228,7 @@ def main(argv=None):
     s = summarize(mk.profile_records())
     mk.close()
     out = {k: v for k, v in s.items() if k != "phase_end_us"}
-    print(json.dumps(out, indent=1))
+    print(markdown(out) if args.markdown else json.dumps(out, indent=1))
 
 
 if __name__ == "__main__":

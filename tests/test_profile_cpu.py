@@ -5,7 +5,7 @@ persistent_megakernel_02_b200.profile.summarize derives from raw records."""
 import numpy as np
 import pytest
 
-from persistent_megakernel_02_b200.profile import OPS, summarize
+from persistent_megakernel_02_b200.profile import OPS, markdown, summarize
 
 OP = {v: k for k, v in OPS.items()}
 
@@ -59,3 +59,11 @@ def test_chain_and_spread_use_the_middle_layers():
     assert sp["lm"]["end"][0] == pytest.approx((20100 - 10100) / 1e3)
     assert sp["lm"]["end"][-1] == pytest.approx((22200 - 10100) / 1e3)
     assert sp["lm"]["end_by_sm"] == [10.0, 12.1]
+
+
+def test_markdown_report_lists_every_op_present():
+    text = markdown(summarize(_records()), bench_us=456.4)
+    assert "bench without stamps: 456.4 us" in text
+    rows = [ln for ln in text.splitlines() if ln.startswith("| gu ") or ln.startswith("| lm ")]
+    assert len(rows) == 2
+    assert "| 0 | gu |" in text and "| 1 | gu |" in text
