@@ -155,10 +155,11 @@ def max_over_ranks(value: float, dist=None, device="cpu") -> float:
     return float(t.item())
 
 
-def oracle_sample(cfg, prompt, n_steps, w_host=None, time_budget_s=25.0):
+def oracle_sample(cfg, prompt, n_steps, w_host=None, time_budget_s=25.0, warmup=0):
     """Time the CPU oracle (as it stands) on a bounded sample of the workload:
-    the prompt is run untimed, then up to n_steps greedy decode steps are timed
-    (stopping once the budget is spent).  Returns (us per step, steps, threads)."""
+    the prompt and `warmup` greedy decode steps run untimed, then up to n_steps
+    greedy decode steps are timed (stopping once the budget is spent).  Returns
+    (us per step, timed steps, threads)."""
     import numpy as np
 
     from oracle import OracleModel, argmax_lowest
@@ -170,6 +171,10 @@ def oracle_sample(cfg, prompt, n_steps, w_host=None, time_budget_s=25.0):
         logits = orc.step(int(t), p, cache)
     pos = len(prompt)
     tok = int(argmax_lowest(logits))
+    for _ in range(warmup):
+        logits = orc.step(tok, pos, cache)
+        tok = int(argmax_lowest(logits))
+        pos += 1
     t0 = time.perf_counter()
     done = 0
     while done < n_steps:
@@ -198,13 +203,13 @@ def run_reference(args, cfg, wl):
 
     w = synth.make_weights(cfg, device="cpu")
     prompt = synth.prompt_tokens(cfg, 0, wl["prompt_lens"][0]).numpy()
-    us, done, threads = oracle_sample(cfg, prompt, max(1, args.warmup + args.steps), host_weights(w),
-                                      time_budget_s=args.ref_budget)
-    sample = (f"{done} greedy decode steps after an untimed {len(prompt)}-token prompt, "
-              f"workload {wl['name']}")
+    us, done, threads = oracle_sample(cfg, prompt, max(1, args.steps), host_weights(w),
+                                      time_budget_s=args.ref_budget, warmup=args.warmup)
+    sample = (f"{done} greedy decode steps timed after an untimed {len(prompt)}-token prompt and "
+              f"{args.warmup} untimed steps, workload {wl['name']}")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(us, 1), "unit": "us/step",
-        "n_gpus": args.gpus, "steps": done, "warmup": 0, "ms_per_step": round(us / 1000, 3),
+        "n_gpus": args.gpus, "steps": done, "warmup": args.warmup, "ms_per_step": round(us / 1000, 3),
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic", "config": _config_obj(wl, cfg),
         "cpu_baseline": {"value": round(us, 1), "unit": "us/step", "cores": threads,
