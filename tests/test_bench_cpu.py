@@ -1,0 +1,38 @@
+"""Host-side pieces of bench.py (no GPU): the recorded ncu traffic is reported only
+while the kernel sources hash to the value it was captured with."""
+
+import os
+import shutil
+
+import bench
+
+
+def _copy_tree(tmp_path):
+    root = tmp_path / "repo"
+    src = os.path.join(bench.ROOT, "persistent_megakernel_02_b200", "csrc")
+    shutil.copytree(src, root / "persistent_megakernel_02_b200" / "csrc")
+    (root / "profiles").mkdir()
+    return root
+
+
+def _write(root, workload, sha, per_step):
+    (root / "profiles" / f"mk_decode_kernel_{workload}_traffic.txt").write_text(
+        "# comment line: ignored\n"
+        f"workload: {workload}\nkernel_src_sha256_16: {sha}\n"
+        f"dram_bytes_read: 1\ndram_bytes_write: 2\ndram_bytes_per_step: {per_step}\n")
+
+
+def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
+    root = _copy_tree(tmp_path)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    sha = bench.kernel_src_hash()
+    _write(root, "wl_a", sha, 123456789)
+    assert bench.recorded_traffic("wl_a") == 123456789.0
+    _write(root, "wl_b", "0" * 16, 5)
+    assert bench.recorded_traffic("wl_b") is None
+    assert bench.recorded_traffic("no_such_workload") is None
+    # any change to a kernel source changes the hash
+    f = root / "persistent_megakernel_02_b200" / "csrc" / "mk_plan.h"
+    f.write_text(f.read_text() + "\n")
+    assert bench.kernel_src_hash() != sha
+    assert bench.recorded_traffic("wl_a") is None
