@@ -36,3 +36,19 @@ def test_traffic_reported_only_for_the_captured_sources(tmp_path, monkeypatch):
     f.write_text(f.read_text() + "\n")
     assert bench.kernel_src_hash() != sha
     assert bench.recorded_traffic("wl_a") is None
+
+
+def test_clock_summary_parses_nvidia_smi_samples():
+    """Median SM clock under load, the maximum, and every throttle reason seen active
+    (the fields of ClockSampler.FIELDS, in that order)."""
+    c = bench.ClockSampler(0)
+    c.lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 850.5, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = c.summary()
+    assert s == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    assert bench.ClockSampler(0).summary()["samples"] == 0
