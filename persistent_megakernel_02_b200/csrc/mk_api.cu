@@ -15,6 +15,19 @@
 
 using namespace mk;
 
+namespace mk {
+// host-side handles of mk_decode_kernel<nbt, spec>, one translation unit each (mk_inst.cu)
+#define MK_DECL(s) \
+  const void* decode_kernel_s##s##_n1(); \
+  const void* decode_kernel_s##s##_n2(); \
+  const void* decode_kernel_s##s##_n4(); \
+  const void* decode_kernel_s##s##_n8();
+MK_DECL(0)
+MK_DECL(1)
+MK_DECL(2)
+#undef MK_DECL
+}  // namespace mk
+
 struct mk_ctx {
   mk_config cfg{};
   Dims D{};
@@ -249,17 +262,20 @@ void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w, const mk_ctx*
   }
 }
 
-template <int SPEC>
-const void* kernel_for_spec(int nbt) {
-  switch (nbt) {
-    case 1: return (const void*)mk_decode_kernel<1, SPEC>;
-    case 2: return (const void*)mk_decode_kernel<2, SPEC>;
-    case 4: return (const void*)mk_decode_kernel<4, SPEC>;
-    default: return (const void*)mk_decode_kernel<8, SPEC>;
-  }
-}
+// The kernel instantiations live in their own translation units (mk_inst.cu,
+// compiled once per specialisation).
 const void* kernel_for(int nbt, int spec) {
-  return spec == 1 ? kernel_for_spec<1>(nbt) : spec == 2 ? kernel_for_spec<2>(nbt) : kernel_for_spec<0>(nbt);
+#define MK_PICK(s)                             \
+  switch (nbt) {                               \
+    case 1: return decode_kernel_s##s##_n1();  \
+    case 2: return decode_kernel_s##s##_n2();  \
+    case 4: return decode_kernel_s##s##_n4();  \
+    default: return decode_kernel_s##s##_n8(); \
+  }
+  if (spec == 1) MK_PICK(1)
+  if (spec == 2) MK_PICK(2)
+  MK_PICK(0)
+#undef MK_PICK
 }
 
 mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {

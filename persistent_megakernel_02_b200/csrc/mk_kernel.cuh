@@ -180,7 +180,7 @@ static_assert(sizeof(Misc) <= 8192 - 8 * (128 + 64), "Misc does not fit its shar
 
 __device__ __forceinline__ bool aborted(const KParams& p) { return ld_relaxed_u32(&p.err->abort) != 0; }
 
-__device__ __noinline__ void raise_error(const KParams& p, uint32_t code, uint32_t instr, uint32_t info,
+static __device__ __noinline__ void raise_error(const KParams& p, uint32_t code, uint32_t instr, uint32_t info,
                                          bool abort) {
   if (atomicCAS(&p.err->code, 0u, code) == 0u) {
     p.err->sm = blockIdx.x;
@@ -192,7 +192,7 @@ __device__ __noinline__ void raise_error(const KParams& p, uint32_t code, uint32
 }
 
 // Spin until *c >= target (acquire), the abort flag rises, or the time limit passes.
-__device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, uint32_t target,
+static __device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, uint32_t target,
                                           uint32_t instr) {
   if (ld_acquire_u32(c) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -211,7 +211,7 @@ __device__ __noinline__ bool wait_counter(const KParams& p, const uint32_t* c, u
 
 // Spin until the hint counter *c reaches target (relaxed: the data it announces
 // is validated element by element), the abort flag rises, or the time passes.
-__device__ __noinline__ bool wait_hint(const KParams& p, const uint32_t* c, uint32_t target, uint32_t instr) {
+static __device__ __noinline__ bool wait_hint(const KParams& p, const uint32_t* c, uint32_t target, uint32_t instr) {
   if (ld_relaxed_u32(c) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -229,7 +229,7 @@ __device__ __noinline__ bool wait_hint(const KParams& p, const uint32_t* c, uint
 
 // Re-read an activation element group until no element holds the sentinel
 // (bounded; on timeout or abort the CTA stops and zeros are returned).
-__device__ __noinline__ float4 poll4_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+static __device__ __noinline__ float4 poll4_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     const float4 v = ld_relaxed_f4(src);
@@ -245,7 +245,7 @@ __device__ __noinline__ float4 poll4_slow(const KParams& p, const float* src, ui
   misc->stop = 1;
   return make_float4(0.f, 0.f, 0.f, 0.f);
 }
-__device__ __noinline__ float2 poll2_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+static __device__ __noinline__ float2 poll2_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     const float2 v = ld_relaxed_f2(src);
@@ -261,7 +261,7 @@ __device__ __noinline__ float2 poll2_slow(const KParams& p, const float* src, ui
   misc->stop = 1;
   return make_float2(0.f, 0.f);
 }
-__device__ __noinline__ float poll1_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
+static __device__ __noinline__ float poll1_slow(const KParams& p, const float* src, uint32_t instr, Misc* misc) {
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     const float v = ld_relaxed_f1(src);
@@ -385,7 +385,7 @@ __device__ __forceinline__ AttnPlan attn_plan(int S, int rep, int npg, int s) {
 
 // Producer: wait until the consumers have entered instruction seq - 15, so the
 // dyn_end entry of seq - 16 is no longer read.
-__device__ __noinline__ bool wait_consumers(const KParams& p, Misc* misc, uint32_t seq, uint32_t instr) {
+static __device__ __noinline__ bool wait_consumers(const KParams& p, Misc* misc, uint32_t seq, uint32_t instr) {
   if (misc->cons_seq + 16u > seq) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -477,7 +477,7 @@ __device__ __forceinline__ void issue_matvec_page(const KParams& p, const Instr&
 // touches global memory only for the tape (the next instruction is loaded while
 // the current one is issued) and the page table; every other address comes from
 // the instruction, so the issue loop never stalls on a dependent load.
-__device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
+static __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, uint64_t* full, uint64_t* empty,
                                       Misc* misc) {
   const Dims& D = p.D;
   const uint32_t NP = (uint32_t)p.ring_pages;
@@ -619,7 +619,7 @@ struct Chunk8 {
   float4 l[NBT], h[NBT];
 };
 template <int NBT>
-__device__ __noinline__ Chunk8<NBT> stage_one_slow(const KParams& p, const float* src, int ld, uint32_t ii,
+static __device__ __noinline__ Chunk8<NBT> stage_one_slow(const KParams& p, const float* src, int ld, uint32_t ii,
                                                    Misc* misc) {
   Chunk8<NBT> r;
   Spin sp(p, misc);
@@ -643,7 +643,7 @@ __device__ __noinline__ Chunk8<NBT> stage_one_slow(const KParams& p, const float
 }
 // one 8-element chunk of each lane's residual accumulator, until all 1 + n_ks terms are in
 template <int NBT>
-__device__ __noinline__ Chunk8<NBT> acc_chunk_slow(const KParams& p, const unsigned long long* src, int ld,
+static __device__ __noinline__ Chunk8<NBT> acc_chunk_slow(const KParams& p, const unsigned long long* src, int ld,
                                                    uint32_t ii, Misc* misc) {
   Chunk8<NBT> r;
   const uint32_t want = 1u + (uint32_t)p.D.n_ks;
@@ -810,7 +810,7 @@ __device__ __forceinline__ void resid_issue(const KParams& p, const Misc* misc, 
   r.src = acc_of(p, misc, layer - 1) + (size_t)b * p.D.H + row;
   r.acc = ld_relaxed_u64(r.src);
 }
-__device__ __noinline__ unsigned long long resid_slow(const KParams& p, Misc* misc, const unsigned long long* src,
+static __device__ __noinline__ unsigned long long resid_slow(const KParams& p, Misc* misc, const unsigned long long* src,
                                                       uint32_t ii) {
   const uint32_t want = 1u + (uint32_t)p.D.n_ks;
   Spin sp(p, misc);
@@ -878,7 +878,7 @@ __device__ __forceinline__ unsigned long long* lm_keys(const KParams& p, const M
 }
 
 template <int NBT>
-__device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBest<NBT> best) {
+static __device__ __noinline__ void lm_finish(const KParams& p, Misc* misc, const LmBest<NBT> best) {
   const Dims& D = p.D;
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
 #pragma unroll
@@ -1623,7 +1623,7 @@ __device__ __forceinline__ uint32_t attn_units_body(const KParams& p, const Inst
   return used;
 }
 template <int DH, int REP, bool KV16F>
-__device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+static __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
                                             float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii) {
   return attn_units_body<DH, REP, KV16F>(p, I, page_base, ring, act, full, empty, misc, ii);
 }
@@ -1631,7 +1631,7 @@ __device__ __noinline__ uint32_t attn_units(const KParams& p, const Instr& I, ui
 // ---------------------------------------------------------------- consumers: ops
 
 template <int OPK, int RT, int NBT>
-__device__ __noinline__ void mv_units_call(const KParams& p, const Instr& I, uint32_t pb, uint8_t* ring,
+static __device__ __noinline__ void mv_units_call(const KParams& p, const Instr& I, uint32_t pb, uint8_t* ring,
                                            const float* act, int K, uint64_t* full, uint64_t* empty, Misc* misc,
                                            uint32_t ii) {
   mv_units<OPK, RT, NBT>(p, I, pb, ring, act, K, full, empty, misc, ii);
@@ -1690,7 +1690,7 @@ __device__ __forceinline__ uint32_t attn_dispatch(const KParams& p, const Instr&
 }
 
 template <int NBT, int SPEC>
-__device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* act, uint64_t* full,
+static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, float* act, uint64_t* full,
                                       uint64_t* empty, Misc* misc) {
   const Dims& D = p.D;
   const int ct = threadIdx.x - 32;
