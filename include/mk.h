@@ -235,6 +235,17 @@ typedef struct {
 mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
                         int32_t dyn_percent, mk_plan_report* rep);
 
+/* The RoPE inverse frequencies this library builds its (cos, sin) table from:
+ * out[i] = rope_theta^(-2i/head_dim) for i < head_dim/2, rescaled by the Llama-3
+ * rule when cfg->rope_scaling != 0 (see mk_config).  Host only, no GPU; the table
+ * itself holds cos and sin of pos * out[i], computed in double and rounded to
+ * float.  The RoPE rotation is the fused "RMSNorm + QKV + RoPE" instruction of
+ * the Hazy megakernel article (section "Megakernel: a deep-fusion design from
+ * scratch"); the frequency rule is the published Llama-3 one, which the pages
+ * name ("RoPE theta 500000 with Llama-3 scaling") without spelling out.
+ *   out  host double[n], n >= head_dim/2 (else MK_ERR_INVALID_ARG) */
+mk_status mk_rope_inv_freq(const mk_config* cfg, double* out, int32_t n);
+
 /* ---- greedy head without allocation ----
  *
  * No counterpart in the pages: a convenience entry point of this library.

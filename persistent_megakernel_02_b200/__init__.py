@@ -18,7 +18,7 @@ import os
 from .build import LIB
 
 __all__ = ["Megakernel", "MkError", "plan_check", "version", "lib", "STATUS",
-           "greedy_head_noalloc"]
+           "greedy_head_noalloc", "rope_inv_freq"]
 
 STATUS = {
     0: "MK_OK",
@@ -105,6 +105,8 @@ _SIGS = {
     "mk_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "mk_plan_check": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                      ctypes.c_int32, ctypes.POINTER(MkPlanReport)]),
+    "mk_rope_inv_freq": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.POINTER(ctypes.c_double),
+                                        ctypes.c_int32]),
     "mk_profile_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
                                        ctypes.POINTER(ctypes.c_int32),
                                        ctypes.POINTER(ctypes.c_int32)]),
@@ -161,6 +163,15 @@ def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0, dyn_percent: int =
     _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, dyn_percent, ctypes.byref(rep)),
            "mk_plan_check")
     return {f: getattr(rep, f) for f, _ in MkPlanReport._fields_}
+
+
+def rope_inv_freq(cfg: dict):
+    """The RoPE inverse frequencies the library's table is built from (host only)."""
+    n = int(cfg["head_dim"]) // 2
+    out = (ctypes.c_double * n)()
+    c = config_struct(cfg)
+    _check(lib().mk_rope_inv_freq(ctypes.byref(c), out, n), "mk_rope_inv_freq")
+    return list(out)
 
 
 def greedy_head_noalloc(hidden, final_norm, lm_head, rms_eps, ids, logits=None, stream=None):

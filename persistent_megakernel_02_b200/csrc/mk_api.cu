@@ -131,7 +131,10 @@ std::string dims_from_config(const mk_config* c, int n_sm, Dims* D) {
   return why;
 }
 
-// inverse frequencies theta^(-2i/d) with the optional Llama-3 rescaling of long wavelengths
+// Inverse frequencies theta^(-2i/d), i < d/2, with the optional Llama-3 rescaling:
+// wavelengths 2 pi / f shorter than orig/high_freq are kept, longer than
+// orig/low_freq divided by the factor, and in between blended linearly in
+// orig/wavelength, f' = (1 - s) f / factor + s f with s = (orig/wl - low)/(high - low).
 std::vector<double> inv_freq(const mk_config* c) {
   const int half = c->head_dim / 2;
   std::vector<double> f(half);
@@ -429,6 +432,17 @@ mk_status status_of(const ErrWord& e) {
 }
 
 }  // namespace
+
+extern "C" mk_status mk_rope_inv_freq(const mk_config* cfg, double* out, int32_t n) {
+  if (!cfg || !out || cfg->head_dim < 2 || n < cfg->head_dim / 2) return MK_ERR_INVALID_ARG;
+  if (!(cfg->rope_theta > 0.f)) return MK_ERR_INVALID_ARG;
+  if (cfg->rope_scaling && (!(cfg->rope_factor > 0.f) || !(cfg->rope_low_freq > 0.f) ||
+                            !(cfg->rope_high_freq > cfg->rope_low_freq) || cfg->rope_orig_max <= 0))
+    return MK_ERR_INVALID_ARG;
+  const std::vector<double> f = inv_freq(cfg);
+  for (size_t i = 0; i < f.size(); ++i) out[i] = f[i];
+  return MK_OK;
+}
 
 extern "C" mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
                                    int32_t dyn_percent, mk_plan_report* rep) {

@@ -109,3 +109,29 @@ def test_noalloc_head_rejects_bad_arguments_on_the_host():
     assert mk.STATUS[f(ids, 0, 64, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_INVALID_ARG"
     assert mk.STATUS[f(ids, 9, 64, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_UNSUPPORTED"
     assert mk.STATUS[f(ids, 8, 4096, ids, ids, 10, 1e-5, None, ids, None)] == "MK_ERR_UNSUPPORTED"
+
+
+def test_library_rope_frequencies_match_the_published_rule():
+    """The inverse frequencies the library builds its RoPE table from equal the
+    hand-derived Llama-3 band values (oracle pins) and the oracle's own, on the
+    1B shape (scaled) and the 8B shape (unscaled, d = 128)."""
+    from oracle import rope_inv_freq as oracle_inv_freq
+    from tests.test_oracle_pins import LLAMA3_BAND_GOLDEN, LLAMA3_SCALING
+
+    lib_f = mk.rope_inv_freq(configs.model_config("llama1b_bs1"))
+    for i, want in LLAMA3_BAND_GOLDEN.items():
+        assert lib_f[i] == pytest.approx(want, rel=1e-13), i
+    for wl, scaling in (("llama1b_bs1", LLAMA3_SCALING), ("llama8b_bs1", None), ("tiny", None)):
+        cfg = configs.model_config(wl)
+        got = mk.rope_inv_freq(cfg)
+        want = oracle_inv_freq(cfg["head_dim"], cfg["rope_theta"], scaling)
+        assert got == pytest.approx(list(want), rel=1e-13), wl
+
+
+def test_rope_inv_freq_rejects_bad_arguments():
+    cfg = configs.model_config("llama1b_bs1")
+    c = mk.config_struct(cfg)
+    out = (ctypes.c_double * 32)()
+    assert mk.lib().mk_rope_inv_freq(ctypes.byref(c), out, 31) == 1
+    bad = dict(cfg, rope_high_freq=0.5)
+    assert mk.lib().mk_rope_inv_freq(ctypes.byref(mk.config_struct(bad)), out, 32) == 1

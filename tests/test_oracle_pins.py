@@ -68,6 +68,51 @@ def test_llama3_scaling_regimes():
     assert np.all(np.diff(sc) < 0)
 
 
+# Llama-3 frequency scaling at the Llama-3.2-1B setting (d = 64, theta = 5e5,
+# factor 32, low-frequency factor 1, high-frequency factor 4, original context
+# 8192), derived by hand from the published rule at 40-digit precision:
+#   f_i = 5e5^(-2i/64);  wavelength wl_i = 2 pi / f_i;
+#   wl < 8192/4 = 2048: keep f;  wl > 8192/1 = 8192: f/32;
+#   else s = (8192/wl - 1) / (4 - 1) and f' = (1 - s) f/32 + s f.
+#   i   f_i                      wl_i           8192/wl      s                 f'_i
+#   14  3.21144599475259090e-3   1956.497       4.18707      (below 2048)      = f
+#   15  2.13111953691196530e-3   2948.303       2.77854789   0.592849295003    1.29054792820926375e-3
+#   16  1.41421356237309503e-3   4442.883       1.84384782   0.281282605163    4.29556796559368208e-4
+#   17  9.38473870357380241e-4   6695.109       1.22357969   0.074526564161    9.70828780262767289e-5
+#   18  6.22772421914595986e-4   10089.055      (above 8192)                   1.94616381848311246e-5
+# (i = 16: f = 1/sqrt(5e5), so wl = 2 pi sqrt(5e5) = 4442.8829..., and
+#  f' = f (0.718717/32 + 0.281283) = 0.303743 f.)
+LLAMA3_BAND_GOLDEN = {
+    14: 3.21144599475259090e-3,
+    15: 1.29054792820926375e-3,
+    16: 4.29556796559368208e-4,
+    17: 9.70828780262767289e-5,
+    18: 1.94616381848311246e-5,
+}
+# What three plausible misreadings of the band would give at i = 15, 16, 17:
+# blending linearly in wavelength between the edges, blending the inverse
+# frequency (harmonic) with the same weight, and swapping the two weights.
+LLAMA3_BAND_MISREADINGS = {
+    "blend in wavelength": {15: 1.82859762853031086e-3, 16: 8.80190766379930316e-4,
+                            17: 2.50826798817474299e-4},
+    "blend in 1/frequency": {15: 1.56450658892072502e-4, 16: 6.07473809782372115e-5,
+                             17: 3.16094340067713531e-5},
+    "weights swapped": {15: 9.07169094231200413e-4, 16: 1.02885093963788615e-3,
+                        17: 8.70718300779771675e-4},
+}
+LLAMA3_SCALING = dict(factor=32.0, low_freq=1.0, high_freq=4.0, orig_max=8192)
+
+
+def test_llama3_scaling_band_golden_values():
+    sc = rope_inv_freq(64, 500000.0, LLAMA3_SCALING)
+    for i, want in LLAMA3_BAND_GOLDEN.items():
+        assert sc[i] == pytest.approx(want, rel=1e-13), i
+    # every plausible misreading of the band misses the golden values by far
+    for name, vals in LLAMA3_BAND_MISREADINGS.items():
+        for i, wrong in vals.items():
+            assert abs(wrong - LLAMA3_BAND_GOLDEN[i]) > 0.2 * LLAMA3_BAND_GOLDEN[i], (name, i)
+
+
 def test_rope_half_split_pairs_and_sign():
     # d = 4: pair 0 is (x[0], x[2]); rotating e0 by +90 degrees gives e2
     x = np.array([1.0, 0.0, 0.0, 0.0])
