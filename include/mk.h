@@ -267,7 +267,10 @@ mk_status mk_rope_inv_freq(const mk_config* cfg, double* out, int32_t n);
  * itself.  Calls that overlap on the GPU (e.g. on two streams) race on it: order
  * them on one stream.  The first call on a device looks up the array's device
  * address with that device current; make that first call before any stream
- * capture.
+ * capture.  That look-up is kept for the life of the process and is not redone
+ * after a cudaDeviceReset, so the entry point is not usable on a device that has
+ * been reset.  A call made while an earlier CUDA error is pending on the calling
+ * thread returns MK_ERR_CUDA without launching and leaves that error in place.
  *
  *   hidden_dev   device float[nb][hidden]
  *   final_norm   device bf16[hidden];   lm_head  device bf16[vocab][hidden] (16-byte aligned)

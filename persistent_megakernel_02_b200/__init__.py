@@ -180,12 +180,45 @@ def greedy_head_noalloc(hidden, final_norm, lm_head, rms_eps, ids, logits=None, 
     For callers that cannot allocate device memory on their call path: the call
     uses only a static scratch array inside the library.  ``hidden`` is a CUDA
     float32 [nb, H] tensor, ``final_norm`` bf16 [H], ``lm_head`` bf16 [V, H],
-    ``ids`` int32 [nb], ``logits`` float32 [nb, V] or None.  Asynchronous; raises
-    MkError on a rejected request.
+    ``ids`` int32 with at least nb elements, ``logits`` float32 [nb, V] or None,
+    all contiguous and on the current CUDA device.  The C entry point sees raw
+    pointers only, so every shape, dtype, layout and device is checked here
+    first; a mismatch raises MkError(MK_ERR_INVALID_ARG) before anything is
+    launched.  Asynchronous.
     """
-    nb, H = hidden.shape
+    import torch
+
+    def bad(why):
+        raise MkError(1, f"mk_greedy_head_noalloc: {why}")
+
+    if hidden.dim() != 2:
+        bad("hidden must be a [nb, hidden] tensor")
+    nb, H = (int(x) for x in hidden.shape)
+    if lm_head.dim() != 2 or int(lm_head.shape[1]) != H:
+        bad("lm_head must be [vocab, hidden]")
+    V = int(lm_head.shape[0])
+    want = [("hidden", hidden, torch.float32, (nb, H)),
+            ("final_norm", final_norm, torch.bfloat16, (H,)),
+            ("lm_head", lm_head, torch.bfloat16, (V, H))]
+    if logits is not None:
+        want.append(("logits", logits, torch.float32, (nb, V)))
+    for name, t, dtype, shape in want:
+        if t.dtype != dtype:
+            bad(f"{name} must be {dtype}, got {t.dtype}")
+        if tuple(t.shape) != shape:
+            bad(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+        if not t.is_contiguous():
+            bad(f"{name} must be contiguous")
+    if ids.dtype != torch.int32 or ids.dim() != 1 or ids.numel() < nb or not ids.is_contiguous():
+        bad("ids must be a contiguous int32 vector of at least nb elements")
+    tensors = [t for _, t, _, _ in want] + [ids]
+    if not all(t.is_cuda for t in tensors):
+        bad("every tensor must be on a CUDA device")
+    dev = torch.cuda.current_device()
+    if any(t.device.index != dev for t in tensors):
+        bad(f"every tensor must be on the current CUDA device ({dev})")
     _check(lib().mk_greedy_head_noalloc(hidden.data_ptr(), nb, H, final_norm.data_ptr(),
-                                        lm_head.data_ptr(), lm_head.shape[0], rms_eps,
+                                        lm_head.data_ptr(), V, rms_eps,
                                         None if logits is None else logits.data_ptr(),
                                         ids.data_ptr(), _stream_handle(stream)),
            "mk_greedy_head_noalloc")
@@ -236,6 +269,7 @@ class Megakernel:
                  n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0,
                  dyn_percent: int = 0):
         self.cfg = dict(cfg)
+        self._host_io = None
         self._weights = weights
         self._arrays = {}
         for name in self._LAYER:
@@ -277,13 +311,19 @@ class Megakernel:
         import numpy as np
 
         nb = len(positions)
-        ids = (ctypes.c_int32 * nb)()
+        if len(tokens) != nb or not 1 <= nb <= 8:
+            raise MkError(1, "mk_decode_step_host: one token and one position per lane, 1..8 lanes")
+        if self._host_io is None:  # argument buffers reused by every call
+            self._host_io = tuple((ctypes.c_int32 * 8)() for _ in range(3))
+        tk, ps, ids = self._host_io
+        for i in range(nb):
+            tk[i] = tokens[i]
+            ps[i] = positions[i]
         lg = np.empty((nb, self.cfg["vocab"]), dtype=np.float32) if want_logits else None
         _check(lib().mk_decode_step_host(
-            self._h, nb, _i32_array(tokens), _i32_array(positions),
-            None if lg is None else lg.ctypes.data_as(ctypes.c_void_p), ids,
+            self._h, nb, tk, ps, None if lg is None else lg.ctypes.data_as(ctypes.c_void_p), ids,
             _stream_handle(stream)), "mk_decode_step_host")
-        return list(ids), lg
+        return ids[:nb], lg
 
     def prefill(self, seq, tokens, start_pos=0, logits_last=None, want_id=True, stream=None):
         """Run the prompt of slot ``seq`` token by token; returns the last greedy id."""

@@ -65,13 +65,23 @@ struct mk_ctx {
   float2* rope = nullptr;
   int* tok_stage = nullptr;
   int tok_stage_cap = 0;
-  int* ids_scratch = nullptr;
+  // Host-path I/O: one device block [ids int32[8] | error word], so a host step
+  // reads both back with a single copy, and its pinned host mirror; tokens of a
+  // host step go in through pinned staging.
+  unsigned char* io_dev = nullptr;
+  int* ids_scratch = nullptr;       // io_dev + 0
+  unsigned char* io_host = nullptr; // pinned, kIoBytes
+  int* tok_host = nullptr;          // pinned, int32[8]
+  int* tok_dev = nullptr;           // device, int32[8]
   float* logits_scratch = nullptr;
   unsigned long long step = 0;
   long long* prof = nullptr;
   int prof_stride = 0;
   std::vector<void*> allocs;
 };
+
+constexpr int kIoErrOff = 32;  // the error word's offset in the I/O block (after 8 ids)
+constexpr int kIoBytes = kIoErrOff + (int)sizeof(ErrWord);
 
 static const char* kVersion = "mk 0.1 (sm_100a persistent decode megakernel)";
 
@@ -325,7 +335,12 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   MK_TRY(from_cuda(cudaMemcpy(h->page_table, pt.data(), pt.size() * 4, cudaMemcpyHostToDevice)));
   h->n_counters = n_counters(D);
   MK_TRY(dalloc(h, &h->counters, (size_t)2 * h->n_counters));
-  MK_TRY(dalloc(h, &h->err, 1));
+  MK_TRY(dalloc(h, &h->io_dev, (size_t)kIoBytes));
+  h->ids_scratch = reinterpret_cast<int*>(h->io_dev);
+  h->err = reinterpret_cast<ErrWord*>(h->io_dev + kIoErrOff);
+  MK_TRY(dalloc(h, &h->tok_dev, kMaxNB));
+  MK_TRY(from_cuda(cudaMallocHost(&h->io_host, kIoBytes)));
+  MK_TRY(from_cuda(cudaMallocHost(&h->tok_host, sizeof(int) * kMaxNB)));
   // RoPE table: cos/sin of pos * inv_freq[i], computed in double
   const int half = D.d / 2;
   std::vector<double> f = inv_freq(&h->cfg);
@@ -337,7 +352,6 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
     }
   MK_TRY(dalloc(h, &h->rope, tab.size()));
   MK_TRY(from_cuda(cudaMemcpy(h->rope, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice)));
-  MK_TRY(dalloc(h, &h->ids_scratch, kMaxNB));
   // shared memory and kernel attributes
   int max_dyn = 0;
   MK_TRY(from_cuda(cudaDeviceGetAttribute(&max_dyn, cudaDevAttrMaxSharedMemoryPerBlockOptin, h->dev)));
@@ -544,6 +558,8 @@ extern "C" mk_status mk_destroy(mk_handle h) {
   cudaDeviceSynchronize();
   for (void* p : h->allocs) cudaFree(p);
   if (h->tok_stage) cudaFree(h->tok_stage);
+  if (h->io_host) cudaFreeHost(h->io_host);
+  if (h->tok_host) cudaFreeHost(h->tok_host);
   if (h->logits_scratch) cudaFree(h->logits_scratch);
   delete h;
   return MK_OK;
@@ -594,22 +610,23 @@ extern "C" mk_status mk_decode_step_host(mk_handle h, int32_t nb, const int32_t*
   if (nb < 1 || nb > h->D.max_batch) return MK_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   cudaSetDevice(h->dev);
-  if (h->tok_stage_cap < kMaxNB) {
-    if (h->tok_stage) cudaFree(h->tok_stage);
-    h->tok_stage = nullptr;
-    MK_TRY(from_cuda(cudaMalloc(&h->tok_stage, sizeof(int) * kMaxNB)));
-    h->tok_stage_cap = kMaxNB;
-  }
   if (logits_host && !h->logits_scratch)
     MK_TRY(from_cuda(cudaMalloc(&h->logits_scratch, sizeof(float) * (size_t)kMaxNB * h->D.V)));
-  MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_stage, tokens_host, sizeof(int) * nb, cudaMemcpyHostToDevice, st)));
-  MK_TRY(mk_decode_step(h, nb, h->tok_stage, positions, logits_host ? h->logits_scratch : nullptr,
+  // tokens in through pinned staging; the step; ids and the error word back in one
+  // copy into pinned memory; one wait for the stream
+  memcpy(h->tok_host, tokens_host, sizeof(int) * nb);
+  MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_dev, h->tok_host, sizeof(int) * nb, cudaMemcpyHostToDevice, st)));
+  MK_TRY(mk_decode_step(h, nb, h->tok_dev, positions, logits_host ? h->logits_scratch : nullptr,
                         h->ids_scratch, stream));
-  MK_TRY(from_cuda(cudaMemcpyAsync(ids_host, h->ids_scratch, sizeof(int) * nb, cudaMemcpyDeviceToHost, st)));
+  MK_TRY(from_cuda(cudaMemcpyAsync(h->io_host, h->io_dev, kIoBytes, cudaMemcpyDeviceToHost, st)));
   if (logits_host)
     MK_TRY(from_cuda(cudaMemcpyAsync(logits_host, h->logits_scratch, sizeof(float) * (size_t)nb * h->D.V,
                                      cudaMemcpyDeviceToHost, st)));
-  return mk_sync(h, stream);
+  MK_TRY(from_cuda(cudaStreamSynchronize(st)));
+  memcpy(ids_host, h->io_host, sizeof(int) * nb);
+  ErrWord e;
+  memcpy(&e, h->io_host + kIoErrOff, sizeof e);
+  return status_of(e);
 }
 
 extern "C" mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_host, int32_t n,

@@ -387,6 +387,7 @@ extern "C" mk_status mk_matvec_engine(int32_t engine, const void* W, int32_t row
   const int grid_cap = n_sm > 0 && n_sm < sms ? n_sm : sms;
   const unsigned long long limit = (unsigned long long)(wait_limit_ms > 0 ? wait_limit_ms : 1000) * 1000000ull;
   cudaStream_t st = (cudaStream_t)stream;
+  if (cudaPeekAtLastError() != cudaSuccess) return MK_ERR_CUDA;  // not this call's error to clear
   const unsigned zero = 0;
   if (cudaMemcpyToSymbolAsync(g_eng_err, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MK_ERR_CUDA;

@@ -135,7 +135,10 @@ __global__ void __launch_bounds__(kHeadThreads) greedy_head_kernel(
 }
 
 // Device address of the static array, looked up once per device (with that
-// device current) on the first call that runs there.
+// device current) on the first call that runs there, together with the kernel's
+// shared-memory attribute.  Both belong to the device's primary context: after a
+// cudaDeviceReset the cached values are stale, so this entry point is not usable
+// again in that process once its device has been reset.
 std::mutex g_setup_mutex;
 void* g_scratch_ptr[64];
 int g_sm_count[64];
@@ -182,8 +185,11 @@ extern "C" mk_status mk_greedy_head_noalloc(const float* hidden_dev, int32_t nb,
   blocks = blocks < 4 * sms ? blocks : 4 * sms;
   if (blocks > kMaxBlocks) blocks = kMaxBlocks;
   const size_t smem = (size_t)nb * hidden * sizeof(float);
+  // An error left pending by some earlier call of the caller's is not this call's
+  // to report or to clear: refuse to launch and leave it in place.
+  if (cudaPeekAtLastError() != cudaSuccess) return MK_ERR_CUDA;
   greedy_head_kernel<<<blocks, kHeadThreads, smem, (cudaStream_t)stream>>>(
       hidden_dev, nb, hidden, (const uint16_t*)final_norm, (const uint16_t*)lm_head, vocab, rms_eps,
       logits_dev, ids_dev, (unsigned char*)scratch);
-  return cudaGetLastError() == cudaSuccess ? MK_OK : MK_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? MK_OK : MK_ERR_CUDA;  // this launch's own error
 }

@@ -175,6 +175,22 @@ def make_weights(cfg: dict, device="cpu", seed: int | None = None,
     return w
 
 
+def to_device(w: dict, device) -> dict:
+    """The weight dict of :func:`make_weights` copied to ``device`` (bits unchanged).
+
+    Generating on the CPU and copying keeps the device free of the generator's
+    many small integer kernels (useful where a launch record is kept)."""
+    out = {}
+    for k, v in w.items():
+        if v is None:
+            out[k] = None
+        elif isinstance(v, list):
+            out[k] = [t.to(device) for t in v]
+        else:
+            out[k] = v.to(device)
+    return out
+
+
 def prompt_tokens(cfg: dict, seq: int, n: int, device="cpu") -> torch.Tensor:
     """Prompt of sequence ``seq``: n tokens uniform in [0, vocab), seed 1 + seq."""
     return tokens(n, cfg["vocab"], seed=cfg.get("prompt_seed", 1) + seq, device=device)

@@ -18,6 +18,14 @@ MAX_ABS = 5e-2
 REL_L2 = 1e-2
 MARGIN = 0.1
 
+# (case, worst max-abs, worst rel-L2, steps compared, ids compared) of every
+# parity case that ran; tests/conftest.py prints them in the session summary
+PARITY_RECORDS = []
+
+
+def record(case, worst, steps, ids_checked):
+    PARITY_RECORDS.append((case, float(worst[0]), float(worst[1]), int(steps), int(ids_checked)))
+
 
 def gpu_weights(cfg, zero_layers=False):
     return synth.make_weights(cfg, device="cuda", zero_layers=zero_layers)

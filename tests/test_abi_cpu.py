@@ -135,3 +135,32 @@ def test_rope_inv_freq_rejects_bad_arguments():
     assert mk.lib().mk_rope_inv_freq(ctypes.byref(c), out, 31) == 1
     bad = dict(cfg, rope_high_freq=0.5)
     assert mk.lib().mk_rope_inv_freq(ctypes.byref(mk.config_struct(bad)), out, 32) == 1
+
+
+def test_noalloc_head_binding_rejects_bad_tensors_before_launch():
+    """The C entry point sees raw pointers only; the binding refuses a wrong dtype,
+    a wrong shape, a non-contiguous operand, a short ids buffer and host tensors
+    before anything reaches the library (CPU tensors: nothing can launch)."""
+    import torch
+
+    from persistent_megakernel_02_b200 import MkError, greedy_head_noalloc
+
+    H, V, nb = 64, 128, 2
+    hidden = torch.zeros((nb, H), dtype=torch.float32)
+    gain = torch.ones(H, dtype=torch.bfloat16)
+    lm = torch.zeros((V, H), dtype=torch.bfloat16)
+    ids = torch.zeros(nb, dtype=torch.int32)
+    cases = {
+        "hidden dtype": (hidden.to(torch.bfloat16), gain, lm, ids, None),
+        "gain dtype": (hidden, gain.float(), lm, ids, None),
+        "lm_head non-contiguous": (hidden, gain, torch.zeros((H, V), dtype=torch.bfloat16).t(), ids, None),
+        "lm_head wrong width": (hidden, gain, torch.zeros((V, H + 8), dtype=torch.bfloat16), ids, None),
+        "lm_head sliced": (hidden, gain, torch.zeros((V, 2 * H), dtype=torch.bfloat16)[:, :H], ids, None),
+        "ids short": (hidden, gain, lm, ids[:1], None),
+        "ids dtype": (hidden, gain, lm, ids.long(), None),
+        "logits shape": (hidden, gain, lm, ids, torch.zeros((nb, V + 1))),
+        "host tensors": (hidden, gain, lm, ids, torch.zeros((nb, V))),
+    }
+    for what, (h, g, w, i, lg) in cases.items():
+        with pytest.raises(MkError, match="INVALID_ARG"):
+            greedy_head_noalloc(h, g, w, 1e-5, i, lg)

@@ -6,10 +6,14 @@ output must equal what mk_decode_step computes for the same hidden state.  With
 every layer matrix zero, the decode step's final hidden state is exactly the
 token's embedding row, so feeding that row to the head must reproduce the
 step's logits and greedy ids -- checked on two calls in a row, each of which
-reuses the scratch the previous one left behind.  Collected last, so a run that
-stops at the first failure has run every other test first.
+reuses the scratch the previous one left behind.  Random hidden states are
+checked against a float64 norm + matvec + argmax (8 lanes of 2048, which needs
+the >48 KiB shared-memory staging), and an exact tie between rows that different
+blocks stream must go to the lower row.  Collected last, so a run that stops at
+the first failure has run every other test first.
 """
 
+import numpy as np
 import pytest
 import torch
 
@@ -55,13 +59,67 @@ def test_noalloc_head_matches_decode_step(wl, nb):
     mk.close()
 
 
+def _f64_head(hidden, gain, lm, eps):
+    """float64 RMSNorm (gain applied) + LM-head matvec of every lane."""
+    x = hidden.double().cpu().numpy()
+    g = gain.double().cpu().numpy()
+    W = lm.double().cpu().numpy()
+    n = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * g
+    return n @ W.T
+
+
+def test_noalloc_head_random_hidden_matches_float64():
+    from persistent_megakernel_02_b200 import greedy_head_noalloc
+
+    nb, H, V = 8, 2048, 32000
+    lm = synth.normal_bf16((V, H), 3, 11, device="cuda")
+    gain = (synth.normal_bf16((H,), 3, 12, std=0.2, device="cuda").float() + 1.0).to(torch.bfloat16)
+    hidden = synth.normal_bf16((nb, H), 3, 13, std=1.5, device="cuda").float().contiguous()
+    for call in range(2):  # two calls in a row share the scratch array
+        ids = torch.full((nb,), -1, dtype=torch.int32, device="cuda")
+        lg = torch.empty((nb, V), dtype=torch.float32, device="cuda")
+        greedy_head_noalloc(hidden, gain, lm, 1e-5, ids, lg)
+        torch.cuda.synchronize()
+        want = _f64_head(hidden, gain, lm, 1e-5)
+        got = lg.cpu().numpy()
+        assert np.abs(got - want).max() < 1e-4, f"call {call}"
+        for b in range(nb):
+            top = np.sort(want[b])[-2:]
+            if top[1] - top[0] > 1e-3:
+                assert ids[b].item() == int(np.argmax(want[b])), (call, b)
+        hidden = -hidden  # the second call sees a different state
+
+
+def test_noalloc_head_ties_across_blocks_take_the_lowest_row():
+    """Rows 100 and 25000 (and 7 and 30000) are identical, and the hidden state
+    is that row, so the two logits tie exactly at the top; the rows are streamed
+    by different blocks, and the lower row must win whichever one is the copy."""
+    from persistent_megakernel_02_b200 import greedy_head_noalloc
+
+    H, V = 2048, 32000
+    lm = synth.normal_bf16((V, H), 5, 21, device="cuda")
+    lm[25000] = lm[100]
+    lm[7] = lm[30000]
+    gain = torch.ones(H, dtype=torch.bfloat16, device="cuda")
+    hidden = torch.stack([lm[100], lm[30000]]).float().contiguous()
+    ids = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    lg = torch.empty((2, V), dtype=torch.float32, device="cuda")
+    greedy_head_noalloc(hidden, gain, lm, 1e-5, ids, lg)
+    torch.cuda.synchronize()
+    assert lg[0, 100].item() == lg[0, 25000].item()
+    assert lg[1, 7].item() == lg[1, 30000].item()
+    assert ids.tolist() == [100, 7]
+
+
 def test_noalloc_head_rejects_oversized_requests():
     from persistent_megakernel_02_b200 import MkError, greedy_head_noalloc
 
     g = torch.ones(4096, dtype=torch.bfloat16, device="cuda")
     lm = torch.zeros((64, 4096), dtype=torch.bfloat16, device="cuda")
+    g64 = torch.ones(64, dtype=torch.bfloat16, device="cuda")
+    lm64 = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
     ids = torch.empty(9, dtype=torch.int32, device="cuda")
     with pytest.raises(MkError, match="UNSUPPORTED"):  # 9 lanes: beyond the scratch array
-        greedy_head_noalloc(torch.zeros((9, 64), device="cuda"), g[:64], lm[:, :64], 1e-5, ids)
+        greedy_head_noalloc(torch.zeros((9, 64), device="cuda"), g64, lm64, 1e-5, ids)
     with pytest.raises(MkError, match="UNSUPPORTED"):  # 8 x 4096 floats: beyond the staging
         greedy_head_noalloc(torch.zeros((8, 4096), device="cuda"), g, lm, 1e-5, ids)
