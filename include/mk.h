@@ -120,6 +120,9 @@ typedef struct {
   int32_t dyn_percent;       /* share of the gate/up, down and LM-head rows that SMs claim
                                 at run time instead of taking from a fixed range: 0 = none
                                 (default), 1..90 = that percent; else MK_ERR_INVALID_ARG */
+  int32_t prefill_tokenwise; /* 1: mk_prefill runs every prompt token through the decode
+                                kernel, one step per token; 0 (default): prompts of 17 or
+                                more tokens run batched on the tensor cores (see mk_prefill) */
 } mk_options;
 
 /* Create a handle: validates the config, lowers it into per-SM instruction
@@ -165,10 +168,22 @@ mk_status mk_decode_step_host(mk_handle h, int32_t nb, const int32_t* tokens_hos
                               int32_t* ids_host, void* stream);
 
 /* Prefill sequence slot `seq` with n HOST tokens at positions start_pos ..
- * start_pos+n-1: one launch that runs one decode step per token.  logits_last_dev (device
- * float[vocab], nullable) and id_last_host (host int32*, nullable) receive the
- * last position's logits and greedy id; when id_last_host is non-NULL the call
- * waits for the stream.  The prompt is copied before the call returns. */
+ * start_pos+n-1 (the cache must hold positions 0 .. start_pos-1).  When the shape
+ * allows it (hidden, n_heads*head_dim and n_kv_heads*head_dim multiples of 128,
+ * ffn a multiple of 64) and n >= 17, tokens 0 .. n-2 run batched, in passes of
+ * at most 2048 tokens: per layer RMSNorm, the QKV GEMM on tcgen05 tensor cores
+ * (RoPE and the K/V cache writes fused), causal attention over the cache, the O
+ * GEMM, the gate/up GEMM (SwiGLU fused) and the down GEMM, with activations split
+ * into bf16 high and low parts so the products keep fp32-level accuracy; then the
+ * last token runs through the decode kernel.  Otherwise (or with
+ * mk_options.prefill_tokenwise) one launch runs one decode step per token.
+ * Prefill has the shape of a GEMM where decode has that of a matvec: "One
+ * Megakernel is Not Enough: Predicting Where to Cut for Streaming Inference",
+ * section "Why where to cut matters more than whether to fuse".
+ * logits_last_dev (device float[vocab], nullable) and id_last_host (host int32*,
+ * nullable) receive the last position's logits and greedy id; when id_last_host
+ * is non-NULL the call waits for the stream.  The prompt is copied before the
+ * call returns. */
 mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_host, int32_t n,
                      int32_t start_pos, float* logits_last_dev, int32_t* id_last_host,
                      void* stream);

@@ -68,6 +68,7 @@ class MkOptions(ctypes.Structure):
         ("device", ctypes.c_int32), ("wait_limit_ms", ctypes.c_int32), ("n_sm", ctypes.c_int32),
         ("ring_pages", ctypes.c_int32), ("debug_fault", ctypes.c_int32),
         ("profile", ctypes.c_int32), ("dyn_percent", ctypes.c_int32),
+        ("prefill_tokenwise", ctypes.c_int32),
     ]
 
 
@@ -260,14 +261,15 @@ class Megakernel:
     'wq', 'wk', 'wv', 'wo', 'mlp_norm', 'w_gate', 'w_up', 'w_down' -- contiguous
     bf16 CUDA tensors.  The handle keeps references to them.  The keyword options
     are mk_options' fields (include/mk.h); ``dyn_percent`` > 0 leaves that share of
-    the gate/up, down and LM-head rows to run-time claims.
+    the gate/up, down and LM-head rows to run-time claims; ``prefill_tokenwise`` = 1
+    runs prompts token by token through the decode kernel instead of batched.
     """
 
     _LAYER = ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")
 
     def __init__(self, cfg: dict, weights: dict, device: int = 0, wait_limit_ms: int = 1000,
                  n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0,
-                 dyn_percent: int = 0):
+                 dyn_percent: int = 0, prefill_tokenwise: int = 0):
         self.cfg = dict(cfg)
         self._host_io = None
         self._weights = weights
@@ -283,7 +285,7 @@ class Megakernel:
         )
         opt = MkOptions(device=device, wait_limit_ms=wait_limit_ms, n_sm=n_sm,
                         ring_pages=ring_pages, debug_fault=debug_fault, profile=profile,
-                        dyn_percent=dyn_percent)
+                        dyn_percent=dyn_percent, prefill_tokenwise=prefill_tokenwise)
         self._cfg_struct = config_struct(cfg)
         h = ctypes.c_void_p()
         _check(lib().mk_create(ctypes.byref(self._cfg_struct), ctypes.byref(w), ctypes.byref(opt),

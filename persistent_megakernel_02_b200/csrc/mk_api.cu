@@ -12,6 +12,7 @@
 #include "../../include/mk.h"
 #include "mk_kernel.cuh"
 #include "mk_plan.h"
+#include "mk_prefill.h"
 
 using namespace mk;
 
@@ -77,9 +78,17 @@ struct mk_ctx {
   unsigned long long step = 0;
   long long* prof = nullptr;
   int prof_stride = 0;
+  // batched prefill on the tensor cores (mk_prefill.cu); null: prompts run token by
+  // token through the decode kernel
+  PrefillPlan* pf = nullptr;
   std::vector<void*> allocs;
 };
 
+// Prompts of at least this many tokens take the batched prefill (the rest run
+// token by token through the decode kernel).
+constexpr int kPrefillBatchMin = 16;
+// tokens per batched-prefill pass (bounds its workspace)
+constexpr int kPrefillChunk = 2048;
 constexpr int kIoErrOff = 32;  // the error word's offset in the I/O block (after 8 ids)
 constexpr int kIoBytes = kIoErrOff + (int)sizeof(ErrWord);
 
@@ -523,6 +532,8 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   why = dims_from_config(cfg, h->n_sm, &h->D);
   h->nbt = lanes_template(cfg->max_batch);
   mk_status s = why.empty() ? build(h, w, o.ring_pages) : MK_ERR_UNSUPPORTED;
+  if (s == MK_OK && !o.prefill_tokenwise && prefill_supported(h->D))
+    s = prefill_create(h->D, w, std::min(kPrefillChunk, h->D.max_seq), &h->pf);
   if (s == MK_OK && o.profile) {
     int stride = 1;
     for (const Tape& t : h->tapes)
@@ -557,6 +568,7 @@ extern "C" mk_status mk_destroy(mk_handle h) {
   cudaSetDevice(h->dev);
   cudaDeviceSynchronize();
   for (void* p : h->allocs) cudaFree(p);
+  prefill_destroy(h->pf);
   if (h->tok_stage) cudaFree(h->tok_stage);
   if (h->io_host) cudaFreeHost(h->io_host);
   if (h->tok_host) cudaFreeHost(h->tok_host);
@@ -650,10 +662,26 @@ extern "C" mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_
   // pageable source: the copy completes before the call returns
   MK_TRY(from_cuda(cudaMemcpyAsync(h->tok_stage, tokens_host, sizeof(int) * n, cudaMemcpyHostToDevice, st)));
   MK_TRY(from_cuda(cudaStreamSynchronize(st)));
-  // one launch runs the whole prompt: step i takes token i at position start_pos + i;
-  // only the last step's logits are kept, every step overwrites the greedy id
   int pos = start_pos, slot = seq;
-  MK_TRY(launch_step(h, 1, h->tok_stage, &pos, &slot, logits_last_dev, h->ids_scratch, st, n,
+  const int* first = h->tok_stage;
+  if (h->pf && n - 1 >= kPrefillBatchMin) {
+    // every token but the last through the batched layers (their K/V rows into the
+    // cache); the last one through the decode kernel, which gives its logits and id
+    PrefillCtx c;
+    c.D = &h->D;
+    c.kv = h->kv;
+    c.page_table = h->page_table;
+    c.rope = h->rope;
+    c.err_code = &h->err->code;
+    c.wait_limit_ns = h->wait_limit_ns;
+    MK_TRY(prefill_run(h->pf, c, h->tok_stage, n - 1, seq, start_pos, st));
+    pos = start_pos + n - 1;
+    first = h->tok_stage + n - 1;
+    n = 1;
+  }
+  // one launch runs the (rest of the) prompt: step i takes token i at position
+  // pos + i; only the last step's logits are kept, every step overwrites the id
+  MK_TRY(launch_step(h, 1, first, &pos, &slot, logits_last_dev, h->ids_scratch, st, n,
                      /*chain=*/0, /*ids_stride=*/0, /*logits_last=*/1));
   if (id_last_host) {
     MK_TRY(from_cuda(cudaMemcpyAsync(id_last_host, h->ids_scratch, sizeof(int), cudaMemcpyDeviceToHost, st)));

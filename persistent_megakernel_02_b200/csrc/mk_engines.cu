@@ -27,6 +27,7 @@
 #include "../../include/mk.h"
 #include "mk_matvec.cuh"
 #include "mk_plan.h"
+#include "mk_tc.cuh"
 
 namespace {
 
@@ -65,49 +66,10 @@ constexpr int kTcThreads = 256;  // warp 0: TMA, warp 1: MMA, warps 4-7: accumul
 constexpr int kTcMaxK = 4096;
 constexpr int kTcTmemCols = 32;  // two accumulators of N = 16 fp32 columns
 
-// Shared-memory matrix descriptor of a K-major operand in the 128-byte swizzled
-// canonical layout: 8-row groups 1024 bytes apart, rows 128 bytes apart.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1 << 16;             // leading byte offset (unused with a swizzle)
-  d |= (uint64_t)(1024 >> 4) << 32;   // stride byte offset: next 8-row group
-  d |= (uint64_t)1 << 46;             // descriptor version of sm_100
-  d |= (uint64_t)2 << 61;             // 128-byte swizzle
-  return d;
-}
-// Instruction descriptor: D fp32, A and B bf16, both K-major, M = 128, N = 16.
-constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTcN >> 3) << 17) |
-                              ((uint32_t)(kTcRows >> 4) << 24);
+constexpr uint32_t kTcIdesc = idesc_bf16(kTcRows, kTcN);
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t acc) {
-  const uint32_t z = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(acc), "r"(z), "r"(z), "r"(z), "r"(z));
-}
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
-                                            uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
-
-// bf16 bits of x rounded to nearest even, and of the remainder
-__device__ __forceinline__ void split_bf16(float x, uint16_t& hi, uint16_t& lo) {
-  const __nv_bfloat16 h = __float2bfloat16_rn(x);
-  hi = __bfloat16_as_ushort(h);
-  lo = __bfloat16_as_ushort(__float2bfloat16_rn(x - __bfloat162float(h)));
+  umma_f16(tmem_d, adesc, bdesc, kTcIdesc, acc);
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
