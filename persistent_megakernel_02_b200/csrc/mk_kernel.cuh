@@ -1148,281 +1148,293 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
 
 // ---------------------------------------------------------------- consumers: attention
 
-// Split-KV GQA decode attention for the slices of this instruction.  A slice
-// covers a contiguous range of KV pages of one (lane, kv head).  Every page is
-// shared by the 8 warps, each taking PL/8 of its positions: a lane scores one
-// (position, query head) pair, then each warp folds its positions into an
-// online-softmax partial (running max m, sum l, unnormalised o) for the REP
-// query heads of the group.  After the slice the CTA combines the warps'
-// partials into the slice partial, and the last slice to finish (atomic
-// counter) merges all slices of the (lane, kv head) into o.
-// One unit: query heads [hq0, hq0 + NH) of kv head g (NH = REP, or 1 in the head
-// split) over pages [pb, pe) of lane b's context (npg pages); se > 1 only with
-// NH = REP.  Returns false when the CTA stopped.
-template <int DH, int REP, int NH, bool KV16F>
+// Split-KV GQA decode attention of one slice: the REP query heads of kv head g
+// over KV pages [pb, pe) of lane b's context (npg pages).  The pages are dealt to
+// the 8 warps like matvec pages (warp w takes the slice's pages w, w + 8, ...),
+// and each warp folds its pages into an online-softmax state of its own (running
+// max m, sum l, unnormalised o per query head): per page, a lane scores its
+// PL / 32 positions against every head, the warp reduces each head's maximum and
+// sum, writes the probabilities to its own shared-memory rows, and P V runs with
+// a lane per DH / 32 output dims.  Warps work on different pages at the same
+// time, so a slice of n pages costs about n / 8 page latencies, not n.  After the
+// slice the CTA merges the 8 warp states into the slice's partial; a slice that
+// covers all pages writes o directly, otherwise the last slice to finish (atomic
+// counter) merges all slices of the (lane, kv head) into o.  This step's K/V row
+// comes from the fp32 copy the QKV instruction published, rounded as the cache
+// holds it, and is patched into the last page by the warp that owns that page.
+// Returns false when the CTA stopped.
+template <int DH, int REP, bool KV16F>
 __device__ __forceinline__ bool attn_one(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
                                          float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii,
-                                         int b, int g, int hq0, int pb, int pe, int npg, int s, int se) {
+                                         int b, int g, int pb, int pe, int npg, int s, int se) {
   constexpr int DC = DH / 8;                 // 16-byte chunks per K/V row
   constexpr int PL = kPageBytes / (4 * DH);  // positions per KV page
-  constexpr int RPW = PL / kConsumerWarps;   // positions of a page per warp
-  constexpr int PAIRS = RPW * NH;            // (position, head) scores per warp
-  constexpr int SPL = (PAIRS + 31) / 32;     // scores per lane
+  constexpr int TPL = PL / 32;               // positions per lane in a page
   constexpr int DPL = DH / 32;               // output dims per lane
   constexpr int CS = DH + 2;                 // partial record: o[DH], m, l
-  static_assert(32 % REP == 0 && 32 % NH == 0, "heads must divide 32");
+  static_assert(PL % 32 == 0, "positions per page");
+  static_assert(kConsumerWarps * PL * REP <= kConsumerWarps * REP * CS, "probabilities alias the combine scratch");
   const Dims& D = p.D;
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const uint32_t NP = (uint32_t)p.ring_pages;
   float4* qlo = reinterpret_cast<float4*>(act);
-  float4* qhi = qlo + NH * DC;
+  float4* qhi = qlo + REP * DC;
   const uint32_t sqlo = smem_u32(qlo), sqhi = smem_u32(qhi);
-  float* comb = act + NH * DH;
+  float* comb = act + REP * DH;
+  float* pw = comb + cw * PL * REP;  // this warp's probabilities [PL][REP] (aliases comb until the merge)
   const float scale = 1.0f / sqrtf((float)DH);
-  const int myh = lane % NH;  // the query head (of the unit's NH) of every score this lane computes
-  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;  // this layer's activation block
-  const uint32_t used = 0;
-  {
-    const int pos = misc->pos[b];
-    const int np_ = pe - pb;
-    // the warp owning this step's position (if this slice holds it) fetches the
-    // fp32 K/V row the QKV instruction published, rounded as the cache holds it,
-    // overlapping the q load
-    const int rcur_all = pos - (npg - 1) * PL;  // row of pos within the last page
-    const bool own_cur = pe == npg && rcur_all / RPW == cw;
-    uint32_t kcur[DH / 64], vcur[DH / 64];
-    if (own_cur) {
-      const float* kn = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + g * DH + lane * (DH / 32);
-      const float* vn = kn + D.kvdim;
-      float kf[DH / 32], vf[DH / 32];
-      if constexpr (DH == 64) {
-        float2 k2 = ld_relaxed_f2(kn), v2 = ld_relaxed_f2(vn);
-        ready(k2, p, kn, ii, misc);
-        ready(v2, p, vn, ii, misc);
-        kf[0] = k2.x; kf[1] = k2.y; vf[0] = v2.x; vf[1] = v2.y;
-      } else {
-        float4 k4 = ld_relaxed_f4(kn), v4 = ld_relaxed_f4(vn);
-        ready(k4, p, kn, ii, misc);
-        ready(v4, p, vn, ii, misc);
-        kf[0] = k4.x; kf[1] = k4.y; kf[2] = k4.z; kf[3] = k4.w;
-        vf[0] = v4.x; vf[1] = v4.y; vf[2] = v4.z; vf[3] = v4.w;
-      }
+  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
+  const int pos = misc->pos[b];
+  const int np_ = pe - pb;
+  // the warp that owns the slice's last page patches this step's K/V row into it
+  const bool own_cur = pe == npg && (np_ - 1) % kConsumerWarps == cw;
+  const int rcur = pos - (npg - 1) * PL;
+  uint32_t kcur[DH / 64], vcur[DH / 64];
+  if (own_cur) {
+    const float* kn = lay + p.off_kvn + (size_t)b * 2 * D.kvdim + g * DH + lane * (DH / 32);
+    const float* vn = kn + D.kvdim;
+    float kf[DH / 32], vf[DH / 32];
+    if constexpr (DH == 64) {
+      float2 k2 = ld_relaxed_f2(kn), v2 = ld_relaxed_f2(vn);
+      ready(k2, p, kn, ii, misc);
+      ready(v2, p, vn, ii, misc);
+      kf[0] = k2.x; kf[1] = k2.y; vf[0] = v2.x; vf[1] = v2.y;
+    } else {
+      float4 k4 = ld_relaxed_f4(kn), v4 = ld_relaxed_f4(vn);
+      ready(k4, p, kn, ii, misc);
+      ready(v4, p, vn, ii, misc);
+      kf[0] = k4.x; kf[1] = k4.y; kf[2] = k4.z; kf[3] = k4.w;
+      vf[0] = v4.x; vf[1] = v4.y; vf[2] = v4.z; vf[3] = v4.w;
+    }
+#pragma unroll
+    for (int e = 0; e < DH / 64; ++e) {
+      kcur[e] = KV16F ? (uint32_t)f2h(kf[2 * e]) | ((uint32_t)f2h(kf[2 * e + 1]) << 16)
+                      : (uint32_t)f2bf(kf[2 * e]) | ((uint32_t)f2bf(kf[2 * e + 1]) << 16);
+      vcur[e] = KV16F ? (uint32_t)f2h(vf[2 * e]) | ((uint32_t)f2h(vf[2 * e + 1]) << 16)
+                      : (uint32_t)f2bf(vf[2 * e]) | ((uint32_t)f2bf(vf[2 * e + 1]) << 16);
+    }
+  }
+  for (int e = ct; e < REP * DC; e += 256) {
+    const int h = e / DC, c = e % DC;
+    const float* src = lay + p.off_q + (size_t)b * D.qdim + (g * REP + h) * DH + c * 8;
+    float4 a0 = ld_relaxed_f4(src), a1 = ld_relaxed_f4(src + 4);
+    ready(a0, p, src, ii, misc);
+    ready(a1, p, src + 4, ii, misc);
+    a0.x *= scale; a0.y *= scale; a0.z *= scale; a0.w *= scale;
+    a1.x *= scale; a1.y *= scale; a1.z *= scale; a1.w *= scale;
+    qlo[h * DC + c] = a0;
+    qhi[h * DC + c] = a1;
+  }
+  cbar();
+
+  float m[REP], l[REP], o[REP][DPL];
+#pragma unroll
+  for (int h = 0; h < REP; ++h) {
+    m[h] = -CUDART_INF_F;
+    l[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
+  }
+  RingPos rp;
+  rp.init(page_base + cw, NP);
+  for (int j = cw; j < np_; j += kConsumerWarps, rp.advance(kConsumerWarps, NP)) {
+    const uint32_t slot = rp.slot;
+    const bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) misc->stop = 1;
+      break;
+    }
+    uint8_t* pg = ring + (size_t)slot * kPageBytes;
+    uint8_t* vpg = pg + PL * DH * 2;
+    const int cnt = min(PL, pos + 1 - (pb + j) * PL);  // positions of this page up to pos, >= 1
+    const bool patch = own_cur && j == np_ - 1;
+    if (patch) {  // this step's K/V, written by the QKV instruction, replace the stale copy
 #pragma unroll
       for (int e = 0; e < DH / 64; ++e) {
-        kcur[e] = KV16F ? (uint32_t)f2h(kf[2 * e]) | ((uint32_t)f2h(kf[2 * e + 1]) << 16)
-                        : (uint32_t)f2bf(kf[2 * e]) | ((uint32_t)f2bf(kf[2 * e + 1]) << 16);
-        vcur[e] = KV16F ? (uint32_t)f2h(vf[2 * e]) | ((uint32_t)f2h(vf[2 * e + 1]) << 16)
-                        : (uint32_t)f2bf(vf[2 * e]) | ((uint32_t)f2bf(vf[2 * e + 1]) << 16);
-      }
-    }
-    for (int e = ct; e < NH * DC; e += 256) {
-      const int h = e / DC, c = e % DC;
-      const float* src = lay + p.off_q + (size_t)b * D.qdim + (hq0 + h) * DH + c * 8;
-      float4 a0 = ld_relaxed_f4(src), a1 = ld_relaxed_f4(src + 4);
-      ready(a0, p, src, ii, misc);
-      ready(a1, p, src + 4, ii, misc);
-      a0.x *= scale; a0.y *= scale; a0.z *= scale; a0.w *= scale;
-      a1.x *= scale; a1.y *= scale; a1.z *= scale; a1.w *= scale;
-      qlo[h * DC + c] = a0;
-      qhi[h * DC + c] = a1;
-    }
-    cbar();
-
-    float m[NH], l[NH], o[NH][DPL];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      m[h] = -CUDART_INF_F;
-      l[h] = 0.f;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
-    }
-    RingPos rp;
-    rp.init(page_base + used, NP);
-    for (int j = 0; j < np_; ++j, rp.advance(1, NP)) {
-      const uint32_t slot = rp.slot;
-      bool ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        if (lane == 0) misc->stop = 1;
-        break;
-      }
-      uint8_t* pg = ring + (size_t)slot * kPageBytes;
-      uint8_t* vpg = pg + PL * DH * 2;
-      const int p0 = (pb + j) * PL;
-      const int cnt = min(PL, pos + 1 - p0);  // valid positions, >= 1
-      const int rcur = pos - p0;              // this step's position, if in this page
-      const int r0 = cw * RPW;
-      const bool patch = rcur >= r0 && rcur < r0 + RPW;
-      if (patch) {  // this step's K/V, written by the QKV instruction, replace the stale copy
-#pragma unroll
-        for (int e = 0; e < DH / 64; ++e) {
-          reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane * (DH / 64) + e] = kcur[e];
-          reinterpret_cast<uint32_t*>(vpg + rcur * DH * 2)[lane * (DH / 64) + e] = vcur[e];
-        }
-        __syncwarp();
-      }
-      // scores: lane -> pair pi = lane + 32 t -> (position r0 + pi / NH, head pi % NH)
-      float sc[SPL];
-      const uint32_t kb = smem_u32(pg);
-#pragma unroll
-      for (int t = 0; t < SPL; ++t) {
-        const int pi = lane + 32 * t, row = r0 + pi / NH;
-        float sv = -CUDART_INF_F;
-        if (pi < PAIRS && row < cnt) {
-          float2 a2 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int cc = 0; cc < DC; ++cc) {
-            const int c = (cc + lane) & (DC - 1);  // lanes of a phase hit distinct banks
-            const uint4 kw = lds128(kb + (uint32_t)((row * DC + c) * 16));
-            const float4 ql = lds128f(sqlo + (uint32_t)((myh * DC + c) * 16));
-            const float4 qh = lds128f(sqhi + (uint32_t)((myh * DC + c) * 16));
-            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.x), kv_hi<KV16F>(kw.x)), make_float2(ql.x, ql.y), a2);
-            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.y), kv_hi<KV16F>(kw.y)), make_float2(ql.z, ql.w), a2);
-            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.z), kv_hi<KV16F>(kw.z)), make_float2(qh.x, qh.y), a2);
-            a2 = __ffma2_rn(make_float2(kv_lo<KV16F>(kw.w), kv_hi<KV16F>(kw.w)), make_float2(qh.z, qh.w), a2);
-          }
-          sv = a2.x + a2.y;
-        }
-        sc[t] = sv;
-      }
-      // per-head max over the warp's positions (lanes with equal lane % NH share a head)
-      float mx = sc[0];
-#pragma unroll
-      for (int t = 1; t < SPL; ++t) mx = fmaxf(mx, sc[t]);
-#pragma unroll
-      for (int off = NH; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      float mnew_mine = fmaxf(m[0], mx);
-#pragma unroll
-      for (int h = 1; h < NH; ++h)
-        if (h == myh) mnew_mine = fmaxf(m[h], mx);
-      float pr[SPL], ps = 0.f;
-#pragma unroll
-      for (int t = 0; t < SPL; ++t) {
-        pr[t] = sc[t] > -CUDART_INF_F ? __expf(sc[t] - mnew_mine) : 0.f;
-        ps += pr[t];
-      }
-#pragma unroll
-      for (int off = NH; off < 32; off <<= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, off);
-      // fold into the running state of every head (lane h holds head h's values)
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const float mh = __shfl_sync(0xFFFFFFFFu, mnew_mine, h);
-        const float sh = __shfl_sync(0xFFFFFFFFu, ps, h);
-        const float corr = mh > -CUDART_INF_F ? __expf(m[h] - mh) : 1.f;
-        l[h] = l[h] * corr + sh;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
-        m[h] = mh;
-      }
-      // o[h][dims of this lane] += p[h][position] * v[position][dims]
-      const uint32_t vb = smem_u32(vpg) + (uint32_t)(lane * DPL * 2);
-#pragma unroll
-      for (int rr = 0; rr < RPW; ++rr) {
-        if (r0 + rr >= cnt) break;
-        float vv[DPL];
-        if constexpr (DPL == 2) {
-          const uint32_t w = lds32(vb + (uint32_t)((r0 + rr) * DH * 2));
-          vv[0] = kv_lo<KV16F>(w); vv[1] = kv_hi<KV16F>(w);
-        } else {
-          const uint2 w = lds64(vb + (uint32_t)((r0 + rr) * DH * 2));
-          vv[0] = kv_lo<KV16F>(w.x); vv[1] = kv_hi<KV16F>(w.x); vv[2] = kv_lo<KV16F>(w.y); vv[3] = kv_hi<KV16F>(w.y);
-        }
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-          const int pi = rr * NH + h;
-          const float ph = __shfl_sync(0xFFFFFFFFu, pr[pi / 32], pi % 32);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(ph, vv[e], o[h][e]);
-        }
+        reinterpret_cast<uint32_t*>(pg + rcur * DH * 2)[lane * (DH / 64) + e] = kcur[e];
+        reinterpret_cast<uint32_t*>(vpg + rcur * DH * 2)[lane * (DH / 64) + e] = vcur[e];
       }
       __syncwarp();
-      if (patch) fence_proxy_async_smem();  // generic writes before the next bulk copy
-      if (lane == 0) mbar_arrive_cnt(&empty[slot], 1u);  // one of the 8 warps
     }
-    // combine the warps' partials into this slice's partial
-    float* mine = comb + cw * NH * CS;
+    // scores: position lane + 32 t against every head
+    float2 a2[TPL][REP];
 #pragma unroll
-    for (int h = 0; h < NH; ++h) {
+    for (int t = 0; t < TPL; ++t)
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) mine[h * CS + lane * DPL + e] = o[h][e];
-      if (lane == 0) { mine[h * CS + DH] = m[h]; mine[h * CS + DH + 1] = l[h]; }
-    }
-    cbar();
-    if (misc->stop) { cbar(); return false; }
-    if (se == 1) {
-      // the only slice of these heads: normalise and write the output, then signal
-      for (int e = ct; e < NH * DH; e += 256) {
-        const int h = e / DH, i = e % DH;
-        float M = -CUDART_INF_F;
-        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * NH + h) * CS + DH]);
-        float L = 0.f, O = 0.f;
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = comb[(w * NH + h) * CS + DH];
-          if (mw > -CUDART_INF_F) {
-            const float f = __expf(mw - M);
-            L += comb[(w * NH + h) * CS + DH + 1] * f;
-            O += comb[(w * NH + h) * CS + i] * f;
-          }
+      for (int h = 0; h < REP; ++h) a2[t][h] = make_float2(0.f, 0.f);
+    const uint32_t kb = smem_u32(pg);
+#pragma unroll 2
+    for (int cc = 0; cc < DC; ++cc) {
+      const int c = (cc + lane) & (DC - 1);  // lanes of a phase hit distinct banks
+      uint4 kw[TPL];
+#pragma unroll
+      for (int t = 0; t < TPL; ++t) kw[t] = lds128(kb + (uint32_t)(((lane + 32 * t) * DC + c) * 16));
+#pragma unroll
+      for (int h = 0; h < REP; ++h) {
+        const float4 ql = lds128f(sqlo + (uint32_t)((h * DC + c) * 16));
+        const float4 qh = lds128f(sqhi + (uint32_t)((h * DC + c) * 16));
+#pragma unroll
+        for (int t = 0; t < TPL; ++t) {
+          float2 acc = a2[t][h];
+          acc = __ffma2_rn(make_float2(kv_lo<KV16F>(kw[t].x), kv_hi<KV16F>(kw[t].x)), make_float2(ql.x, ql.y), acc);
+          acc = __ffma2_rn(make_float2(kv_lo<KV16F>(kw[t].y), kv_hi<KV16F>(kw[t].y)), make_float2(ql.z, ql.w), acc);
+          acc = __ffma2_rn(make_float2(kv_lo<KV16F>(kw[t].z), kv_hi<KV16F>(kw[t].z)), make_float2(qh.x, qh.y), acc);
+          acc = __ffma2_rn(make_float2(kv_lo<KV16F>(kw[t].w), kv_hi<KV16F>(kw[t].w)), make_float2(qh.z, qh.w), acc);
+          a2[t][h] = acc;
         }
-        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (hq0 + h) * DH + i, canon(O / L));
       }
-      cbar();
-      if (ct == 0) red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
-      cbar();
-      return true;
     }
-    if constexpr (NH == REP) {
-    float* part = p.part + ((size_t)(b * D.Hkv + g) * p.S + s) * REP * CS;
+    // online softmax per head over this page's positions
+#pragma unroll
+    for (int h = 0; h < REP; ++h) {
+      float sc[TPL], mx = -CUDART_INF_F;
+#pragma unroll
+      for (int t = 0; t < TPL; ++t) {
+        sc[t] = lane + 32 * t < cnt ? a2[t][h].x + a2[t][h].y : -CUDART_INF_F;
+        mx = fmaxf(mx, sc[t]);
+      }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o2));
+      const float mn = fmaxf(m[h], mx);  // finite: position 0 of every page is valid
+      const float corr = __expf(m[h] - mn);
+      float ps = 0.f;
+#pragma unroll
+      for (int t = 0; t < TPL; ++t) {
+        const float pr = sc[t] > -CUDART_INF_F ? __expf(sc[t] - mn) : 0.f;
+        pw[(lane + 32 * t) * REP + h] = pr;
+        ps += pr;
+      }
+#pragma unroll
+      for (int o2 = 16; o2 > 0; o2 >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, o2);
+      l[h] = l[h] * corr + ps;
+      m[h] = mn;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) o[h][e] *= corr;
+    }
+    __syncwarp();
+    // o[h][dims of this lane] += p[position][h] * v[position][dims]
+    const uint32_t vb = smem_u32(vpg) + (uint32_t)(lane * DPL * 2);
+#pragma unroll 4
+    for (int r = 0; r < cnt; ++r) {
+      float vv[DPL];
+      if constexpr (DPL == 2) {
+        const uint32_t w = lds32(vb + (uint32_t)(r * DH * 2));
+        vv[0] = kv_lo<KV16F>(w); vv[1] = kv_hi<KV16F>(w);
+      } else {
+        const uint2 w = lds64(vb + (uint32_t)(r * DH * 2));
+        vv[0] = kv_lo<KV16F>(w.x); vv[1] = kv_hi<KV16F>(w.x); vv[2] = kv_lo<KV16F>(w.y); vv[3] = kv_hi<KV16F>(w.y);
+      }
+      float ph[REP];
+      if constexpr (REP % 4 == 0) {
+#pragma unroll
+        for (int h = 0; h < REP; h += 4) {
+          const float4 p4 = *reinterpret_cast<const float4*>(pw + r * REP + h);
+          ph[h] = p4.x; ph[h + 1] = p4.y; ph[h + 2] = p4.z; ph[h + 3] = p4.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < REP; ++h) ph[h] = pw[r * REP + h];
+      }
+#pragma unroll
+      for (int h = 0; h < REP; ++h)
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(ph[h], vv[e], o[h][e]);
+    }
+    __syncwarp();
+    if (patch) fence_proxy_async_smem();  // generic writes before the next bulk copy into the slot
+    if (lane == 0) mbar_arrive_cnt(&empty[slot], kConsumerWarps);
+  }
+  cbar();  // every warp is done with its probabilities (they alias comb)
+  // the warps' states into comb, then merged into this slice's partial
+  float* mine = comb + cw * REP * CS;
+#pragma unroll
+  for (int h = 0; h < REP; ++h) {
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) mine[h * CS + lane * DPL + e] = o[h][e];
+    if (lane == 0) { mine[h * CS + DH] = m[h]; mine[h * CS + DH + 1] = l[h]; }
+  }
+  cbar();
+  if (misc->stop) { cbar(); return false; }
+  if (se == 1) {
+    // the only slice of these heads: normalise and write the output, then signal
     for (int e = ct; e < REP * DH; e += 256) {
       const int h = e / DH, i = e % DH;
       float M = -CUDART_INF_F;
       for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * REP + h) * CS + DH]);
       float L = 0.f, O = 0.f;
-      if (M > -CUDART_INF_F)
-        for (int w = 0; w < kConsumerWarps; ++w) {
-          const float mw = comb[(w * REP + h) * CS + DH];
-          if (mw > -CUDART_INF_F) {
-            const float f = __expf(mw - M);
-            L += comb[(w * REP + h) * CS + DH + 1] * f;
-            O += comb[(w * REP + h) * CS + i] * f;
-          }
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float mw = comb[(w * REP + h) * CS + DH];
+        if (mw > -CUDART_INF_F) {
+          const float f = __expf(mw - M);
+          L += comb[(w * REP + h) * CS + DH + 1] * f;
+          O += comb[(w * REP + h) * CS + i] * f;
         }
-      part[h * CS + i] = O;
-      if (i == 0) { part[h * CS + DH] = M; part[h * CS + DH + 1] = L; }
+      }
+      st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
+    }
+    cbar();
+    if (ct == 0) red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
+    cbar();
+    return true;
+  }
+  float* part = p.part + ((size_t)(b * D.Hkv + g) * p.S + s) * REP * CS;
+  for (int e = ct; e < REP * DH; e += 256) {
+    const int h = e / DH, i = e % DH;
+    float M = -CUDART_INF_F;
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, comb[(w * REP + h) * CS + DH]);
+    float L = 0.f, O = 0.f;
+    if (M > -CUDART_INF_F)
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float mw = comb[(w * REP + h) * CS + DH];
+        if (mw > -CUDART_INF_F) {
+          const float f = __expf(mw - M);
+          L += comb[(w * REP + h) * CS + DH + 1] * f;
+          O += comb[(w * REP + h) * CS + i] * f;
+        }
+      }
+    part[h * CS + i] = O;
+    if (i == 0) { part[h * CS + DH] = M; part[h * CS + DH + 1] = L; }
+  }
+  cbar();
+  if (ct == 0) {
+    const uint32_t old = atom_acq_rel_add(p.ctr + ctr_part(D, I.layer, b, g), 1u);
+    misc->last = (old == (uint32_t)se - 1);
+  }
+  cbar();
+  if (misc->last) {
+    const float* pp = p.part + (size_t)(b * D.Hkv + g) * p.S * REP * CS;
+    for (int e = ct; e < REP * DH; e += 256) {
+      const int h = e / DH, i = e % DH;
+      float M = -CUDART_INF_F;
+      for (int t = 0; t < se; ++t) M = fmaxf(M, __ldcg(pp + (t * REP + h) * CS + DH));
+      float L = 0.f, O = 0.f;
+      for (int t = 0; t < se; ++t) {
+        const float mt = __ldcg(pp + (t * REP + h) * CS + DH);
+        if (mt > -CUDART_INF_F) {
+          const float f = __expf(mt - M);
+          L += __ldcg(pp + (t * REP + h) * CS + DH + 1) * f;
+          O += __ldcg(pp + (t * REP + h) * CS + i) * f;
+        }
+      }
+      st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
     }
     cbar();
     if (ct == 0) {
-      const uint32_t old = atom_acq_rel_add(p.ctr + ctr_part(D, I.layer, b, g), 1u);
-      misc->last = (old == (uint32_t)se - 1);
+      p.ctr[ctr_part(D, I.layer, b, g)] = 0u;  // the next step's slices count from zero
+      red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
     }
-    cbar();
-    if (misc->last) {
-      const float* pp = p.part + (size_t)(b * D.Hkv + g) * p.S * REP * CS;
-      for (int e = ct; e < REP * DH; e += 256) {
-        const int h = e / DH, i = e % DH;
-        float M = -CUDART_INF_F;
-        for (int t = 0; t < se; ++t) M = fmaxf(M, __ldcg(pp + (t * REP + h) * CS + DH));
-        float L = 0.f, O = 0.f;
-        for (int t = 0; t < se; ++t) {
-          const float mt = __ldcg(pp + (t * REP + h) * CS + DH);
-          if (mt > -CUDART_INF_F) {
-            const float f = __expf(mt - M);
-            L += __ldcg(pp + (t * REP + h) * CS + DH + 1) * f;
-            O += __ldcg(pp + (t * REP + h) * CS + i) * f;
-          }
-        }
-        st_relaxed_f32(lay + p.off_o + (size_t)b * D.qdim + (g * REP + h) * DH + i, canon(O / L));
-      }
-      cbar();
-      if (ct == 0) {
-        p.ctr[ctr_part(D, I.layer, b, g)] = 0u;  // the next step's slices count from zero
-        red_relaxed_add(p.ctr + ctr_layer(I.layer, C_ATTN), 1u);
-      }
-    }
-    cbar();
-    }  // NH == REP
   }
-  (void)used;
+  cbar();
   return true;
+}
+
+// attn_one out of line: only contexts beyond the short-context form reach it, and
+// inlined into the specialised kernels it raised the register count of every op.
+template <int DH, int REP, bool KV16F>
+__device__ __noinline__ bool attn_one_call(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+                                           float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii,
+                                           int b, int g, int pb, int pe, int npg, int s, int se) {
+  return attn_one<DH, REP, KV16F>(p, I, page_base, ring, act, full, empty, misc, ii, b, g, pb, pe, npg, s, se);
 }
 
 // Short-context attention of one query head (the head split of attn_plan):
@@ -1615,8 +1627,8 @@ __device__ __forceinline__ uint32_t attn_units_body(const KParams& p, const Inst
       ok = attn_flat<DH, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, g * REP + ap.head,
                                 npg);
     else
-      ok = attn_one<DH, REP, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g,
-                                         g * REP, ap.pb, ap.pe, npg, s, ap.se);
+      ok = attn_one_call<DH, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, ap.pb,
+                                         ap.pe, npg, s, ap.se);
     if (!ok) break;
     used += (uint32_t)(ap.pe - ap.pb);
   }
