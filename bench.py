@@ -236,6 +236,8 @@ def main():
     ap.add_argument("--impl", default="mk", choices=["mk", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=25.0)
+    ap.add_argument("--region-cut", type=int, default=0, choices=[0, 1],
+                    help="1: each decode step is two launches (decoder layers, then LM head)")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per decode step from an ncu capture of this kernel (optional)")
     args = ap.parse_args()
@@ -269,10 +271,19 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
     w = synth.make_weights(cfg, device="cuda")
-    mk = Megakernel(cfg, w, device=local)
+    mk = Megakernel(cfg, w, device=local, region_cut=args.region_cut)
     stream = torch.cuda.current_stream()
     prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
     firsts = [mk.prefill(b, prompts[b]) for b in range(nb)]
+    # prefill time of the workload's prompts (again, warm: the same rows are rewritten)
+    torch.cuda.synchronize()
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for b in range(nb):
+        mk.prefill(b, prompts[b], want_id=False, stream=stream)
+    p1.record(stream)
+    torch.cuda.synchronize()
+    prefill_ms = p0.elapsed_time(p1)
     ids = torch.tensor(firsts, dtype=torch.int32, device="cuda")
     pos0 = [len(p) for p in prompts]
 
@@ -343,7 +354,12 @@ def main():
                      "kernel": "mk::mk_decode_kernel<1>" if nb == 1 else f"mk::mk_decode_kernel<{nb}>"},
         "e2e": {"value": round(e2e_us, 2), "unit": "us/step", "h2d_bytes_per_step": 4 * nb,
                 "d2h_bytes_per_step": 4 * nb},
-        "gpu_launches": 1,
+        "gpu_launches": 2 * args.steps if args.region_cut else 1,
+        "prefill": {"tokens": sum(len(p) for p in prompts), "ms": round(prefill_ms, 3),
+                    "tokens_per_s": round(sum(len(p) for p in prompts) / (prefill_ms * 1e-3), 1),
+                    "path": "batched (tcgen05 GEMMs + causal attention), last token through the decode kernel"
+                    if min(len(p) for p in prompts) >= 17 else "token by token through the decode kernel"},
+        "region_cut": args.region_cut,
         "us_per_step_one_launch_per_step": round(us_single, 2),
         "clocks": clk.summary(),
     }

@@ -123,6 +123,12 @@ typedef struct {
   int32_t prefill_tokenwise; /* 1: mk_prefill runs every prompt token through the decode
                                 kernel, one step per token; 0 (default): prompts of 17 or
                                 more tokens run batched on the tensor cores (see mk_prefill) */
+  int32_t region_cut;        /* 1: every decode step is two launches of the persistent
+                                kernel, the decoder layers and then the final norm + LM head
+                                + argmax (the region cut of "One Megakernel is Not Enough:
+                                Predicting Where to Cut for Streaming Inference", section
+                                "Four observations"); results are identical.  0 (default):
+                                one launch per step, or per n steps with mk_decode_steps */
 } mk_options;
 
 /* Create a handle: validates the config, lowers it into per-SM instruction
@@ -243,12 +249,14 @@ typedef struct {
 
 /* Lower `cfg` for `n_sm` SMs and `nb` active lanes, run the CPU tape simulator
  * over the result and fill `rep`.  `dyn_percent` is mk_options.dyn_percent (the
- * share of the streaming phases claimed at run time, 0..90).  `fault` != 0 plants
+ * share of the streaming phases claimed at run time, 0..90); `region` is the part
+ * of the step the tape holds: 0 the whole step, 1 the decoder layers, 2 the final
+ * norm + LM head (the two launches of mk_options.region_cut).  `fault` != 0 plants
  * a fault in the tape first (1: one signal dropped, 2: one wait target raised by
  * one, 3: one instruction's claim range of the LM head shortened by one row
  * block, with dyn_percent > 0) so tests can see the simulator report it. */
 mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                        int32_t dyn_percent, mk_plan_report* rep);
+                        int32_t dyn_percent, int32_t region, mk_plan_report* rep);
 
 /* The RoPE inverse frequencies this library builds its (cos, sin) table from:
  * out[i] = rope_theta^(-2i/head_dim) for i < head_dim/2, rescaled by the Llama-3

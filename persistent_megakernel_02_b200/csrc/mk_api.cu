@@ -46,6 +46,11 @@ struct mk_ctx {
     uint32_t* sm_off = nullptr;
   };
   std::vector<DevTape> dtapes;
+  // region cut (mk_options.region_cut): tapes hold the decoder layers only, and the
+  // final norm + LM head + argmax runs as a second launch from lm_tapes
+  int region_cut = 0;
+  std::vector<Tape> lm_tapes;
+  std::vector<DevTape> lm_dtapes;
   const uint16_t* embed = nullptr;
   float* acts = nullptr;  // two sets of per-layer activation blocks (see KParams)
   long long set_floats = 0, layer_floats = 0, acc_base = 0, acc_floats = 0;
@@ -303,17 +308,24 @@ const void* kernel_for(int nbt, int spec) {
 mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   const Dims& D = h->D;
   MK_TRY(pack_weights(h, w));
-  // tapes, one per active batch size
-  for (int nb = 1; nb <= D.max_batch; ++nb) {
-    h->tapes.push_back(lower(D, h->n_sm, nb, h->dyn_percent));
-    Tape& t = h->tapes.back();
+  // tapes, one per active batch size (two with the region cut: layers, LM head)
+  auto upload = [&](Tape& t, std::vector<mk_ctx::DevTape>& dst) -> mk_status {
     resolve_pointers(t, D, w, h);
     mk_ctx::DevTape dt;
     MK_TRY(dalloc(h, &dt.instrs, t.instrs.size()));
     MK_TRY(dalloc(h, &dt.sm_off, t.sm_off.size()));
     MK_TRY(from_cuda(cudaMemcpy(dt.instrs, t.instrs.data(), t.instrs.size() * sizeof(Instr), cudaMemcpyHostToDevice)));
     MK_TRY(from_cuda(cudaMemcpy(dt.sm_off, t.sm_off.data(), t.sm_off.size() * 4, cudaMemcpyHostToDevice)));
-    h->dtapes.push_back(dt);
+    dst.push_back(dt);
+    return MK_OK;
+  };
+  for (int nb = 1; nb <= D.max_batch; ++nb) {
+    h->tapes.push_back(lower(D, h->n_sm, nb, h->dyn_percent, h->region_cut ? REGION_LAYERS : REGION_ALL));
+    MK_TRY(upload(h->tapes.back(), h->dtapes));
+    if (h->region_cut) {
+      h->lm_tapes.push_back(lower(D, h->n_sm, nb, h->dyn_percent, REGION_LM));
+      MK_TRY(upload(h->lm_tapes.back(), h->lm_dtapes));
+    }
   }
   h->embed = (const uint16_t*)w->embed;
   // scratch and state
@@ -385,10 +397,11 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
 // One launch of n_steps decode steps (see KParams for the token / ids / logits modes).
 mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, const int* slot,
                       float* logits, int* ids, cudaStream_t st, int n_steps = 1, int chain = 1,
-                      int ids_stride = 0, int logits_last = 0) {
+                      int ids_stride = 0, int logits_last = 0, int region = REGION_ALL) {
   const Dims& D = h->D;
-  const Tape& t = h->tapes[nb - 1];
-  const mk_ctx::DevTape& dt = h->dtapes[nb - 1];
+  const bool lm = region == REGION_LM;
+  const Tape& t = lm ? h->lm_tapes[nb - 1] : h->tapes[nb - 1];
+  const mk_ctx::DevTape& dt = lm ? h->lm_dtapes[nb - 1] : h->dtapes[nb - 1];
   KParams p{};
   p.instrs = dt.instrs;
   p.sm_off = dt.sm_off;
@@ -438,8 +451,30 @@ mk_status launch_step(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, 
   cudaError_t e = cudaLaunchCooperativeKernel(kernel_for(nbt, h->spec), dim3(h->n_sm), dim3(kThreads), args,
                                               (size_t)h->sm.total, st);
   h->step++;
-  if (e == cudaSuccess) h->steps_run += (unsigned long long)n_steps;
+  // the layers launch of a cut step shares the LM launch's activation set
+  if (e == cudaSuccess && region != REGION_LAYERS) h->steps_run += (unsigned long long)n_steps;
   return from_cuda(e);
+}
+
+// n_steps decode steps (the launch_step modes).  One launch, or with the region cut
+// two per step: the layers, then the LM head.  Step t of a cut run reads its tokens
+// where the single launch's step t would (the previous step's ids when chained),
+// writes its ids and logits where that step would, at positions pos[b] + t.
+mk_status run_steps(mk_ctx* h, int nb, const int* tokens_dev, const int* pos, const int* slot, float* logits,
+                    int* ids, cudaStream_t st, int n_steps, int chain, int ids_stride, int logits_last) {
+  if (!h->region_cut)
+    return launch_step(h, nb, tokens_dev, pos, slot, logits, ids, st, n_steps, chain, ids_stride, logits_last);
+  const size_t V = (size_t)h->D.V;
+  for (int t = 0; t < n_steps; ++t) {
+    const int* tok = (chain && t > 0) ? ids + (size_t)(t - 1) * ids_stride : tokens_dev + (size_t)(chain ? 0 : t) * nb;
+    int pt[kMaxNB];
+    for (int b = 0; b < nb; ++b) pt[b] = pos[b] + t;
+    float* lg = logits_last ? (t == n_steps - 1 ? logits : nullptr) : (logits ? logits + (size_t)t * nb * V : nullptr);
+    int* id = ids + (size_t)t * ids_stride;
+    MK_TRY(launch_step(h, nb, tok, pt, slot, nullptr, id, st, 1, 0, 0, 0, REGION_LAYERS));
+    MK_TRY(launch_step(h, nb, tok, pt, slot, lg, id, st, 1, 0, 0, 0, REGION_LM));
+  }
+  return MK_OK;
 }
 
 mk_status read_error(mk_ctx* h, ErrWord* out) {
@@ -468,14 +503,15 @@ extern "C" mk_status mk_rope_inv_freq(const mk_config* cfg, double* out, int32_t
 }
 
 extern "C" mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                                   int32_t dyn_percent, mk_plan_report* rep) {
+                                   int32_t dyn_percent, int32_t region, mk_plan_report* rep) {
   if (!cfg || !rep || n_sm < 1 || dyn_percent < 0 || dyn_percent > 90) return MK_ERR_INVALID_ARG;
+  if (region < REGION_ALL || region > REGION_LM) return MK_ERR_INVALID_ARG;
   memset(rep, 0, sizeof(*rep));
   Dims D;
   std::string why = dims_from_config(cfg, n_sm, &D);
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
   if (nb < 1 || nb > D.max_batch) return MK_ERR_INVALID_ARG;
-  Tape t = lower(D, n_sm, nb, dyn_percent > 0 ? dyn_percent : kDynPercent);
+  Tape t = lower(D, n_sm, nb, dyn_percent > 0 ? dyn_percent : kDynPercent, region);
   if (fault == 3) {  // shrink the LM head's claim range by one unit on one SM
     for (auto& I : t.instrs)
       if (I.op == OP_LM && I.pool) { I.pool_u1 -= 1; break; }
@@ -510,6 +546,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   if (opt) o = *opt;
   if (o.wait_limit_ms < 0 || o.n_sm < 0 || o.ring_pages < 0 || o.device < 0) return MK_ERR_INVALID_ARG;
   if (o.dyn_percent < 0 || o.dyn_percent > 90) return MK_ERR_INVALID_ARG;
+  if (o.region_cut != 0 && o.region_cut != 1) return MK_ERR_INVALID_ARG;
   Dims D;
   std::string why = dims_from_config(cfg, 148, &D);  // validation only; rederived below
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
@@ -529,6 +566,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   h->n_sm = o.n_sm > 0 ? std::min(o.n_sm, sms) : sms;
   h->wait_limit_ns = (unsigned long long)(o.wait_limit_ms > 0 ? o.wait_limit_ms : 1000) * 1000000ull;
   h->dyn_percent = o.dyn_percent > 0 ? o.dyn_percent : kDynPercent;
+  h->region_cut = o.region_cut ? 1 : 0;
   why = dims_from_config(cfg, h->n_sm, &h->D);
   h->nbt = lanes_template(cfg->max_batch);
   mk_status s = why.empty() ? build(h, w, o.ring_pages) : MK_ERR_UNSUPPORTED;
@@ -536,8 +574,9 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
     s = prefill_create(h->D, w, std::min(kPrefillChunk, h->D.max_seq), &h->pf);
   if (s == MK_OK && o.profile) {
     int stride = 1;
-    for (const Tape& t : h->tapes)
-      for (int sm = 0; sm < h->n_sm; ++sm) stride = std::max(stride, (int)(t.sm_off[sm + 1] - t.sm_off[sm]));
+    for (const auto* ts : {&h->tapes, &h->lm_tapes})
+      for (const Tape& t : *ts)
+        for (int sm = 0; sm < h->n_sm; ++sm) stride = std::max(stride, (int)(t.sm_off[sm + 1] - t.sm_off[sm]));
     h->prof_stride = stride;
     s = dalloc(h, &h->prof, (size_t)h->n_sm * stride * kProfSlots);
   }
@@ -588,7 +627,7 @@ extern "C" mk_status mk_decode_step(mk_handle h, int32_t nb, const int32_t* toke
     slot[b] = b;
   }
   cudaSetDevice(h->dev);
-  return launch_step(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream);
+  return run_steps(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream, 1, 1, 0, 0);
 }
 
 extern "C" mk_status mk_decode_steps(mk_handle h, int32_t nb, int32_t n_steps, const int32_t* tokens_dev,
@@ -602,8 +641,8 @@ extern "C" mk_status mk_decode_steps(mk_handle h, int32_t nb, int32_t n_steps, c
     slot[b] = b;
   }
   cudaSetDevice(h->dev);
-  return launch_step(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream, n_steps,
-                     /*chain=*/1, /*ids_stride=*/nb, /*logits_last=*/0);
+  return run_steps(h, nb, tokens_dev, positions, slot, logits_dev, ids_dev, (cudaStream_t)stream, n_steps,
+                   /*chain=*/1, /*ids_stride=*/nb, /*logits_last=*/0);
 }
 
 extern "C" mk_status mk_sync(mk_handle h, void* stream) {
@@ -681,8 +720,8 @@ extern "C" mk_status mk_prefill(mk_handle h, int32_t seq, const int32_t* tokens_
   }
   // one launch runs the (rest of the) prompt: step i takes token i at position
   // pos + i; only the last step's logits are kept, every step overwrites the id
-  MK_TRY(launch_step(h, 1, first, &pos, &slot, logits_last_dev, h->ids_scratch, st, n,
-                     /*chain=*/0, /*ids_stride=*/0, /*logits_last=*/1));
+  MK_TRY(run_steps(h, 1, first, &pos, &slot, logits_last_dev, h->ids_scratch, st, n,
+                   /*chain=*/0, /*ids_stride=*/0, /*logits_last=*/1));
   if (id_last_host) {
     MK_TRY(from_cuda(cudaMemcpyAsync(id_last_host, h->ids_scratch, sizeof(int), cudaMemcpyDeviceToHost, st)));
     return mk_sync(h, stream);

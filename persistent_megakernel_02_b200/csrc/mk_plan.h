@@ -85,9 +85,18 @@ struct Dims {
   int kv_fp16;    // KV cache element: 0 bf16, 1 fp16
 };
 
+// Which part of a decode step a tape holds.  The whole step is one launch; the
+// region cut splits it into two launches, the decoder layers and then the final
+// norm + LM head + argmax ("One Megakernel is Not Enough: Predicting Where to Cut
+// for Streaming Inference", section "Four observations": two megakernels can beat
+// one for a language model).  The LM-head tape waits on no counter: the launch
+// boundary orders it after the layers.
+enum Region : int { REGION_ALL = 0, REGION_LAYERS = 1, REGION_LM = 2 };
+
 // One tape: the instruction lists of every SM for one active batch size.
 struct Tape {
   int nb = 0;
+  int region = REGION_ALL;
   int S = 1;                      // attention slices per (lane, kv head)
   int n_counters = 0;
   std::vector<uint32_t> sm_off;   // n_sm + 1 offsets into instrs
@@ -135,7 +144,7 @@ std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, i
 int attn_slices(const Dims& D, int n_sm, int nb);
 // dyn_percent: share of the gate/up, down and LM-head units claimed at run time
 // (0: every unit statically assigned)
-Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent = kDynPercent);
+Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent = kDynPercent, int region = REGION_ALL);
 
 struct SimReport {
   bool deadlock_free = false, coverage_ok = false, targets_ok = false;

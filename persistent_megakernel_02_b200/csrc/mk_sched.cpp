@@ -143,9 +143,10 @@ struct Assigner {
 };
 }  // namespace
 
-Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent) {
+Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent, int region) {
   Tape t;
   t.nb = nb;
+  t.region = region;
   t.S = attn_slices(D, n_sm, nb);
   t.n_counters = n_counters(D);
   std::vector<int64_t> load(n_sm, 0);
@@ -195,7 +196,7 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent) {
       }
   };
 
-  for (int l = 0; l < D.L; ++l) {
+  for (int l = 0; l < (region == REGION_LM ? 0 : D.L); ++l) {
     uint16_t dep_qkv = l ? (uint16_t)ctr_layer(l - 1, C_DOWN) : kNoCounter;
     // RMSNorm + QKV + RoPE
     auto a = as.run(D.n_qkv, unit_bytes(D, OP_QKV, t.S), 0, n_sm);
@@ -225,7 +226,10 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent) {
     }
   }
   // final norm + LM head + argmax: every SM takes part (possibly with no rows)
-  phase(OP_LM, D.L, D.n_lm, 0, n_sm, (uint16_t)ctr_layer(D.L - 1, C_DOWN), kNoCounter, 0, pool_lm(D), true);
+  // (in its own launch it waits on nothing: the launch boundary orders it)
+  if (region != REGION_LAYERS)
+    phase(OP_LM, D.L, D.n_lm, 0, n_sm, region == REGION_LM ? kNoCounter : (uint16_t)ctr_layer(D.L - 1, C_DOWN),
+          kNoCounter, 0, pool_lm(D), true);
 
   // wait targets = how many instructions signal the counter in one step
   std::vector<uint32_t> fan(t.n_counters, 0);
@@ -355,10 +359,20 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
   };
   r.coverage_ok = !cover_err && all_one(cq) && all_one(co) && all_one(cg) && all_one(cd) &&
                   all_one(ca) && all_one(cl);
+  if (t.region != REGION_ALL) {  // each part covers its own ops once and the other's not at all
+    auto all_zero = [](const std::vector<int>& v) {
+      for (int x : v)
+        if (x != 0) return false;
+      return true;
+    };
+    const bool layers_ok = all_one(cq) && all_one(co) && all_one(cg) && all_one(cd) && all_one(ca);
+    const bool layers_none = all_zero(cq) && all_zero(co) && all_zero(cg) && all_zero(cd) && all_zero(ca);
+    r.coverage_ok = !cover_err && (t.region == REGION_LAYERS ? layers_ok && all_zero(cl) : layers_none && all_one(cl));
+  }
   r.targets_ok = true;
   for (const Instr& I : t.instrs)
     if (I.dep != kNoCounter && signals[I.dep] != (int64_t)I.dep_target) r.targets_ok = false;
-  if (signals[ctr_lm(D)] != n_sm) r.targets_ok = false;
+  if (signals[ctr_lm(D)] != (t.region == REGION_LAYERS ? 0 : n_sm)) r.targets_ok = false;
   if (!r.coverage_ok && r.error.empty()) r.error = "coverage";
   if (!r.targets_ok && r.error.empty()) r.error = "targets";
   return r;

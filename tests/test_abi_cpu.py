@@ -164,3 +164,25 @@ def test_noalloc_head_binding_rejects_bad_tensors_before_launch():
     for what, (h, g, w, i, lg) in cases.items():
         with pytest.raises(MkError, match="INVALID_ARG"):
             greedy_head_noalloc(h, g, w, 1e-5, i, lg)
+
+
+@pytest.mark.parametrize("wl", list(configs.WORKLOADS))
+def test_region_cut_tapes_are_deadlock_free_and_split_the_outputs(wl):
+    """The two launches of the region cut: the layers tape produces every layer
+    output once and no LM-head tile, the LM-head tape every LM-head tile once and
+    nothing else, each deadlock-free with exact wait targets."""
+    cfg = configs.model_config(wl)
+    for nb in sorted({1, cfg["max_batch"]}):
+        for region in (1, 2):
+            r = mk.plan_check(cfg, 148, nb, region=region)
+            assert r["deadlock_free"] and r["coverage_ok"] and r["targets_ok"], (wl, nb, region, r)
+    whole = mk.plan_check(cfg, 148, 1)
+    layers = mk.plan_check(cfg, 148, 1, region=1)
+    lm = mk.plan_check(cfg, 148, 1, region=2)
+    assert layers["n_instr_total"] + lm["n_instr_total"] == whole["n_instr_total"]
+
+
+def test_plan_check_rejects_an_unknown_region():
+    c = mk.config_struct(configs.model_config("tiny"))
+    rep = mk.MkPlanReport()
+    assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 3, ctypes.byref(rep)) == 1

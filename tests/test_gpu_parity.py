@@ -386,3 +386,32 @@ def test_out_of_range_device_token_is_reported():
     mk.decode_step(tok, [0], ids)
     assert STATUS[mk.status()] == "MK_OK"
     mk.close()
+
+
+@pytest.mark.parametrize("wl,nb", [("tiny", 3), ("llama1b_bs1", 1)])
+def test_region_cut_gives_the_single_launch_results_bit_for_bit(wl, nb):
+    """Two launches per step (layers, then the LM head) compute exactly what one
+    launch does: the same code per output row and fixed-point residuals, so a
+    chained multi-step run and a token-by-token prefill give identical logits and
+    ids with and without the cut."""
+    cfg = configs.model_config(wl, max_batch=nb, max_seq=64)
+    w = H.gpu_weights(cfg)
+    lens = [5 + 3 * b for b in range(nb)]
+    prompts = [synth.prompt_tokens(cfg, b, n).tolist() for b, n in enumerate(lens)]
+    n, V = 6, cfg["vocab"]
+    runs = []
+    for cut in (0, 1):
+        mk = _mk(cfg, w, region_cut=cut, prefill_tokenwise=1)
+        lg0 = torch.empty(V, dtype=torch.float32, device="cuda")
+        first = [mk.prefill(b, prompts[b], logits_last=lg0) for b in range(nb)]
+        tok = torch.tensor(first, dtype=torch.int32, device="cuda")
+        ids = torch.empty((n, nb), dtype=torch.int32, device="cuda")
+        lg = torch.empty((n, nb, V), dtype=torch.float32, device="cuda")
+        mk.decode_steps(tok, lens, n, ids, lg)
+        mk.sync()
+        mk.close()
+        runs.append((first, lg0.cpu().numpy(), ids.cpu().numpy(), lg.cpu().numpy()))
+    assert runs[0][0] == runs[1][0]
+    np.testing.assert_array_equal(runs[0][1], runs[1][1])
+    np.testing.assert_array_equal(runs[0][2], runs[1][2])
+    np.testing.assert_array_equal(runs[0][3], runs[1][3])
