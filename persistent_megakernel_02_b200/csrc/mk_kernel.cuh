@@ -1428,15 +1428,6 @@ __device__ __forceinline__ bool attn_one(const KParams& p, const Instr& I, uint3
   return true;
 }
 
-// attn_one out of line: only contexts beyond the short-context form reach it, and
-// inlined into the specialised kernels it raised the register count of every op.
-template <int DH, int REP, bool KV16F>
-__device__ __noinline__ bool attn_one_call(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
-                                           float* act, uint64_t* full, uint64_t* empty, Misc* misc, uint32_t ii,
-                                           int b, int g, int pb, int pe, int npg, int s, int se) {
-  return attn_one<DH, REP, KV16F>(p, I, page_base, ring, act, full, empty, misc, ii, b, g, pb, pe, npg, s, se);
-}
-
 // Short-context attention of one query head (the head split of attn_plan):
 // every position of lane b's context (npg <= kHeadSplitPages pages, at most 256
 // positions) is scored at once, one position per thread, then a block-wide
@@ -1627,8 +1618,8 @@ __device__ __forceinline__ uint32_t attn_units_body(const KParams& p, const Inst
       ok = attn_flat<DH, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, g * REP + ap.head,
                                 npg);
     else
-      ok = attn_one_call<DH, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, ap.pb,
-                                         ap.pe, npg, s, ap.se);
+      ok = attn_one<DH, REP, KV16F>(p, I, page_base + used, ring, act, full, empty, misc, ii, b, g, ap.pb, ap.pe,
+                                    npg, s, ap.se);
     if (!ok) break;
     used += (uint32_t)(ap.pe - ap.pb);
   }
