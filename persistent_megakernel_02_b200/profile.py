@@ -134,8 +134,22 @@ def summarize(rec: np.ndarray) -> dict:
                           units=q([r["t_last_warp"] - r["t_staged"] for r in rs if r["t_staged"]]),
                           end=q([r["t_sig"] - f for r in rs]),
                           end_by_sm=[round((r["t_sig"] - f) / 1e3, 1) for r in sorted(rs, key=lambda r: r["sm"])])
+    # Share of the SMs' time (n_sm x step) the consumers spent waiting on other SMs:
+    # at instruction barriers (the slowest warp of the previous instruction, and the
+    # hint-counter wait where enabled) and re-reading activations not yet written
+    # (the polls that replace counter waits; summed over a CTA's 8 consumer warps,
+    # so divided by 8), next to the share spent waiting for weight pages to land.
+    n_sm = rec.shape[0]
+    sm_time = n_sm * max(1, t1 - t0)
+    barrier_ns = sum(r["t_dep"] - r["t_start"] for r in rows)
+    poll_ns = sum(r["slow_ns"] for r in rows) / 8.0
+    page_ns = sum(r["c_wait"] for r in rows) / 8.0
+    wait_share = {"barrier": round(barrier_ns / sm_time, 4), "data_poll": round(poll_ns / sm_time, 4),
+                  "barrier_plus_poll": round((barrier_ns + poll_ns) / sm_time, 4),
+                  "page_wait": round(page_ns / sm_time, 4)}
     return {
         "step_us": (t1 - t0) / 1e3,
+        "wait_share": wait_share,
         "spread_p0_10_50_90_100_us": spread,
         "chain_first_last_end_us": chain,
         "per_op": {k: {kk: round(vv, 3) if isinstance(vv, float) else vv for kk, vv in v.items()}
@@ -179,6 +193,13 @@ def markdown(s: dict, bench_us: float | None = None) -> str:
     sp = s["spread_p0_10_50_90_100_us"]
     out.append("Spread between SMs (percentiles 0/10/50/90/100 of each SM's end, from the phase's "
                "first start): " + "; ".join(f"{op} {sp[op]['end']}" for op in sp) + ".")
+    ws = s.get("wait_share")
+    if ws:
+        out.append("")
+        out.append(f"Wait share of the SMs' time (148 SMs x step): instruction barriers {100 * ws['barrier']:.1f} %, "
+                   f"re-reads of activations not yet written {100 * ws['data_poll']:.1f} % "
+                   f"(together {100 * ws['barrier_plus_poll']:.1f} %: the dependency waits that replace "
+                   f"counter waits); waits for weight pages to land {100 * ws['page_wait']:.1f} %.")
     return "\n".join(out) + "\n"
 
 

@@ -67,3 +67,19 @@ def test_markdown_report_lists_every_op_present():
     rows = [ln for ln in text.splitlines() if ln.startswith("| gu ") or ln.startswith("| lm ")]
     assert len(rows) == 2
     assert "| 0 | gu |" in text and "| 1 | gu |" in text
+
+
+def test_wait_share_of_the_sms_time():
+    """Barrier waits (t_dep - t_start) and re-read time (summed over a CTA's 8
+    warps) as shares of n_sm x step; page waits beside them."""
+    rec = _records()
+    rec[0, 0, 17] = 8 * 400    # 400 ns of re-reads per warp on SM 0's first instruction
+    rec[1, 2, 7] = 8 * 1000    # 1000 ns of page waits per warp on SM 1's LM head
+    s = summarize(rec)
+    sm_time = 2 * (22200 - 1000)
+    barrier = (100 + 300 + 100 + 200 + 100 + 200)
+    assert s["wait_share"]["barrier"] == pytest.approx(barrier / sm_time, abs=1e-4)
+    assert s["wait_share"]["data_poll"] == pytest.approx(400 / sm_time, abs=1e-4)
+    assert s["wait_share"]["barrier_plus_poll"] == pytest.approx((barrier + 400) / sm_time, abs=1e-4)
+    assert s["wait_share"]["page_wait"] == pytest.approx(1000 / sm_time, abs=1e-4)
+    assert "Wait share" in markdown(s)
