@@ -238,6 +238,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=25.0)
     ap.add_argument("--region-cut", type=int, default=0, choices=[0, 1],
                     help="1: each decode step is two launches (decoder layers, then LM head)")
+    ap.add_argument("--tensor-core-units", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="8-lane matvecs on tcgen05: 0 measured default, 1 none, 2 LM head, 3 gate/up, 4 both")
     ap.add_argument("--traffic-bytes", type=float, default=None,
                     help="DRAM bytes per decode step from an ncu capture of this kernel (optional)")
     args = ap.parse_args()
@@ -271,7 +273,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         pg = dist
     w = synth.make_weights(cfg, device="cuda")
-    mk = Megakernel(cfg, w, device=local, region_cut=args.region_cut)
+    mk = Megakernel(cfg, w, device=local, region_cut=args.region_cut, tensor_core_units=args.tensor_core_units)
     stream = torch.cuda.current_stream()
     prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
     firsts = [mk.prefill(b, prompts[b]) for b in range(nb)]
@@ -360,6 +362,7 @@ def main():
                     "path": "batched (tcgen05 GEMMs + causal attention), last token through the decode kernel"
                     if min(len(p) for p in prompts) >= 17 else "token by token through the decode kernel"},
         "region_cut": args.region_cut,
+        "tensor_core_units": args.tensor_core_units,
         "us_per_step_one_launch_per_step": round(us_single, 2),
         "clocks": clk.summary(),
     }

@@ -129,6 +129,13 @@ typedef struct {
                                 Predicting Where to Cut for Streaming Inference", section
                                 "Four observations"); results are identical.  0 (default):
                                 one launch per step, or per n steps with mk_decode_steps */
+  int32_t tensor_core_units; /* which matvecs of the 8-lane kernel (5-8 lanes) run on the
+                                tcgen05 tensor cores (128-row blocks, accumulators in tensor
+                                memory) where the shape allows it (the Llama-3.2-1B-shaped
+                                kernel): 0 (default) the choice measured faster -- the LM head
+                                on tcgen05, gate/up on CUDA cores --, 1 none (CUDA cores
+                                everywhere), 2 the LM head, 3 gate/up, 4 both; other values:
+                                MK_ERR_INVALID_ARG */
 } mk_options;
 
 /* Create a handle: validates the config, lowers it into per-SM instruction
@@ -251,12 +258,14 @@ typedef struct {
  * over the result and fill `rep`.  `dyn_percent` is mk_options.dyn_percent (the
  * share of the streaming phases claimed at run time, 0..90); `region` is the part
  * of the step the tape holds: 0 the whole step, 1 the decoder layers, 2 the final
- * norm + LM head (the two launches of mk_options.region_cut).  `fault` != 0 plants
+ * norm + LM head (the two launches of mk_options.region_cut); `tensor_core_units` is
+ * mk_options.tensor_core_units (which 8-lane matvecs are tensor-core units).  `fault` != 0 plants
  * a fault in the tape first (1: one signal dropped, 2: one wait target raised by
  * one, 3: one instruction's claim range of the LM head shortened by one row
  * block, with dyn_percent > 0) so tests can see the simulator report it. */
 mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                        int32_t dyn_percent, int32_t region, mk_plan_report* rep);
+                        int32_t dyn_percent, int32_t region, int32_t tensor_core_units,
+                        mk_plan_report* rep);
 
 /* The RoPE inverse frequencies this library builds its (cos, sin) table from:
  * out[i] = rope_theta^(-2i/head_dim) for i < head_dim/2, rescaled by the Llama-3

@@ -69,6 +69,7 @@ class MkOptions(ctypes.Structure):
         ("ring_pages", ctypes.c_int32), ("debug_fault", ctypes.c_int32),
         ("profile", ctypes.c_int32), ("dyn_percent", ctypes.c_int32),
         ("prefill_tokenwise", ctypes.c_int32), ("region_cut", ctypes.c_int32),
+        ("tensor_core_units", ctypes.c_int32),
     ]
 
 
@@ -105,7 +106,8 @@ _SIGS = {
     "mk_clear_error": (ctypes.c_int, [ctypes.c_void_p]),
     "mk_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "mk_plan_check": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
-                                     ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(MkPlanReport)]),
+                                     ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                     ctypes.POINTER(MkPlanReport)]),
     "mk_rope_inv_freq": (ctypes.c_int, [ctypes.POINTER(MkConfig), ctypes.POINTER(ctypes.c_double),
                                         ctypes.c_int32]),
     "mk_profile_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64,
@@ -157,13 +159,15 @@ def config_struct(cfg: dict) -> MkConfig:
     return MkConfig(**{k: cfg.get(k, 0) if k == "kv_dtype" else cfg[k] for k in _CFG_FIELDS})
 
 
-def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0, dyn_percent: int = 0, region: int = 0) -> dict:
+def plan_check(cfg: dict, n_sm: int, nb: int, fault: int = 0, dyn_percent: int = 0, region: int = 0,
+               tensor_core_units: int = 0) -> dict:
     """Lower ``cfg`` on the host and run the tape simulator (no GPU needed).
-    ``region``: 0 the whole step, 1 the decoder layers, 2 the LM head (region cut)."""
+    ``region``: 0 the whole step, 1 the decoder layers, 2 the LM head (region cut);
+    ``tensor_core_units``: mk_options.tensor_core_units."""
     rep = MkPlanReport()
     c = config_struct(cfg)
-    _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, dyn_percent, region, ctypes.byref(rep)),
-           "mk_plan_check")
+    _check(lib().mk_plan_check(ctypes.byref(c), n_sm, nb, fault, dyn_percent, region, tensor_core_units,
+                               ctypes.byref(rep)), "mk_plan_check")
     return {f: getattr(rep, f) for f, _ in MkPlanReport._fields_}
 
 
@@ -264,14 +268,17 @@ class Megakernel:
     are mk_options' fields (include/mk.h); ``dyn_percent`` > 0 leaves that share of
     the gate/up, down and LM-head rows to run-time claims; ``prefill_tokenwise`` = 1
     runs prompts token by token through the decode kernel instead of batched;
-    ``region_cut`` = 1 runs each decode step as two launches (layers, LM head).
+    ``region_cut`` = 1 runs each decode step as two launches (layers, LM head);
+    ``tensor_core_units`` picks the 8-lane matvecs on tcgen05 (0 measured default,
+    1 none, 2 LM head, 3 gate/up, 4 both).
     """
 
     _LAYER = ("attn_norm", "wq", "wk", "wv", "wo", "mlp_norm", "w_gate", "w_up", "w_down")
 
     def __init__(self, cfg: dict, weights: dict, device: int = 0, wait_limit_ms: int = 1000,
                  n_sm: int = 0, ring_pages: int = 0, debug_fault: int = 0, profile: int = 0,
-                 dyn_percent: int = 0, prefill_tokenwise: int = 0, region_cut: int = 0):
+                 dyn_percent: int = 0, prefill_tokenwise: int = 0, region_cut: int = 0,
+                 tensor_core_units: int = 0):
         self.cfg = dict(cfg)
         self._host_io = None
         self._weights = weights
@@ -288,7 +295,7 @@ class Megakernel:
         opt = MkOptions(device=device, wait_limit_ms=wait_limit_ms, n_sm=n_sm,
                         ring_pages=ring_pages, debug_fault=debug_fault, profile=profile,
                         dyn_percent=dyn_percent, prefill_tokenwise=prefill_tokenwise,
-                        region_cut=region_cut)
+                        region_cut=region_cut, tensor_core_units=tensor_core_units)
         self._cfg_struct = config_struct(cfg)
         h = ctypes.c_void_p()
         _check(lib().mk_create(ctypes.byref(self._cfg_struct), ctypes.byref(w), ctypes.byref(opt),

@@ -65,6 +65,8 @@ struct mk_ctx {
   // the layer matrices in page order (pack_weights): every unit's page is one
   // contiguous 16 KiB block, so the producer moves it with a single bulk copy
   uint16_t *pk_qkv = nullptr, *pk_gu = nullptr, *pk_dn = nullptr;
+  // tensor-core tiles (Dims::tc): gate/up per layer, LM head
+  uint16_t *pk_gu_tc = nullptr, *pk_lm_tc = nullptr;
   uint32_t* counters = nullptr;
   int n_counters = 0;
   ErrWord* err = nullptr;
@@ -140,7 +142,31 @@ mk_status dalloc(mk_ctx* h, T** p, size_t count) {
   return MK_OK;
 }
 
-std::string dims_from_config(const mk_config* c, int n_sm, Dims* D) {
+// Kernel specialisation of a shape (mk_kernel.cuh, Spec): 1 and 2 when every unit
+// has the same row count and the attention one known form, else 0.
+int kernel_spec(const Dims& D) {
+  const int rq = 2 * D.RP, ro = D.Ro, rg = 2 * D.Rgu, rd = D.Rdn, rl = D.Rlm;
+  if (rq == 4 && ro == 4 && rg == 4 && rd == 4 && rl == 4 && D.d == 64 && D.rep == 4 && !D.kv_fp16) return 1;
+  if (rq == 2 && ro == 2 && rg == 2 && rd == 2 && rl == 2 && D.d == 128 && D.rep == 4 && D.kv_fp16) return 2;
+  return 0;
+}
+
+// Whether the 8-lane kernel can run gate/up and the LM head on the tensor cores:
+// the specialised Llama-3.2-1B-shaped kernel, whose staged activation (8 lanes x
+// hidden fp32) has room for the MMA operand (16 rows of bf16 high/low parts x hidden).
+bool tc_units(const Dims& D) {
+  return kernel_spec(D) == 1 && lanes_template(D.max_batch) == 8 && D.H % 64 == 0 && D.F % 64 == 0 &&
+         D.H >= 64 && D.H <= 2048;
+}
+
+// Tensor-core units of the 8-lane kernel by default (mk_options.tensor_core_units 0):
+// the engine each op measured faster on with 8 lanes (bit 0 LM head, bit 1 gate/up).
+// Llama-3.2-1B shape, batch 8, one box: CUDA cores 1505.9 us/step, LM head on tcgen05
+// 1467.9, gate/up on tcgen05 1714.2, both 1669.7 -- the LM head's long stream gains,
+// gate/up (one 32-page block per SM, 20 SMs without one) loses.
+constexpr int kTcDefault = 1;
+
+std::string dims_from_config(const mk_config* c, int n_sm, Dims* D, int tc_sel = 0) {
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return "rms_eps must be finite and >= 0";
   if (!(c->rope_theta > 0.f)) return "rope_theta must be positive";
   if (c->rope_scaling) {
@@ -152,6 +178,7 @@ std::string dims_from_config(const mk_config* c, int n_sm, Dims* D) {
   std::string why = derive_dims(c->n_layers, c->hidden, c->n_heads, c->n_kv_heads, c->head_dim, c->ffn,
                                 c->vocab, c->tied, c->rms_eps, c->max_batch, c->max_seq, n_sm, D);
   D->kv_fp16 = c->kv_dtype;
+  if (why.empty()) D->tc = tc_units(*D) ? (tc_sel == 0 ? kTcDefault : tc_sel - 1) : 0;
   return why;
 }
 
@@ -198,6 +225,7 @@ mk_status check_weights(const mk_config* c, const mk_weights* w) {
 }
 
 // Packed-layer sizes (elements per layer).
+size_t pk_gu_tc_elems(const Dims& D) { return (size_t)D.n_gu_tc * D.nkt * 128 * 64; }
 size_t pk_qkv_elems(const Dims& D) { return (size_t)D.n_qkv * 2 * D.RP * D.H; }
 size_t pk_gu_elems(const Dims& D) { return (size_t)D.n_gu * 2 * D.Rgu * D.H; }
 size_t pk_dn_elems(const Dims& D) { return (size_t)D.n_ks * D.H * D.KS; }
@@ -211,6 +239,38 @@ __global__ void pack_rows_kernel(const uint4* const* src, uint4* dst, long long 
     const uint4* s = src[r];
     dst[e] = s ? s[e - r * row_u4] : make_uint4(0u, 0u, 0u, 0u);
   }
+}
+
+// Tensor-core tiles: block u, K tile kt is 128 rows x 64 bf16, row r's 16-byte
+// chunk c stored at chunk (c ^ (r & 7)) of its 128-byte row (the 128-byte swizzle
+// the MMA's shared-memory descriptor reads), tiles one after another in (u, kt)
+// order, so the kernel streams every 16 KiB tile with one bulk copy.  Row r of
+// block u comes from src[u * 128 + r] (zeros where null); rows are nkt * 64 long.
+__global__ void pack_tc_tiles_kernel(const uint4* const* src, uint4* dst, long long n_rows, int nkt) {
+  const long long n = n_rows * nkt * 8;  // 16-byte chunks
+  for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(e & 7);
+    const long long rest = e >> 3;
+    const int r = (int)(rest & 127);
+    const long long ut = rest >> 7;  // u * nkt + kt
+    const int kt = (int)(ut % nkt);
+    const long long u = ut / nkt;
+    const uint4* s = src[u * 128 + r];
+    dst[(ut * 128 + r) * 8 + (c ^ (r & 7))] = s ? s[(size_t)kt * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+mk_status pack_tc_tiles(const std::vector<const void*>& rows, void* dst, int nkt) {
+  const uint4** d_src = nullptr;
+  MK_TRY(from_cuda(cudaMalloc(&d_src, rows.size() * sizeof(void*))));
+  cudaError_t e = cudaMemcpy(d_src, rows.data(), rows.size() * sizeof(void*), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) {
+    pack_tc_tiles_kernel<<<1184, 256>>>(d_src, static_cast<uint4*>(dst), (long long)rows.size(), nkt);
+    e = cudaGetLastError();
+  }
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  cudaFree(d_src);
+  return from_cuda(e);
 }
 
 mk_status pack_rows(const std::vector<const void*>& rows, void* dst, int row_bytes) {
@@ -269,6 +329,24 @@ mk_status pack_weights(mk_ctx* h, const mk_weights* w) {
       for (int r = 0; r < D.H; ++r)
         rows.push_back(static_cast<const uint16_t*>(w->w_down[l]) + (size_t)r * D.F + (size_t)ks * D.KS);
   MK_TRY(pack_rows(rows, h->pk_dn, D.KS * 2));
+  if (D.tc & 2) {  // tensor-core tiles of gate/up, gate and up rows interleaved
+    MK_TRY(dalloc(h, &h->pk_gu_tc, pk_gu_tc_elems(D) * D.L));
+    rows.clear();
+    for (int l = 0; l < D.L; ++l)
+      for (int u = 0; u < D.n_gu_tc; ++u)
+        for (int r = 0; r < 128; ++r) {
+          const uint16_t* m = static_cast<const uint16_t*>((r & 1) ? w->w_up[l] : w->w_gate[l]);
+          rows.push_back(m + (size_t)(64 * u + (r >> 1)) * rowH);
+        }
+    MK_TRY(pack_tc_tiles(rows, h->pk_gu_tc, D.nkt));
+  }
+  if (D.tc & 1) {  // tensor-core tiles of the LM head (rows past the vocabulary zero)
+    MK_TRY(dalloc(h, &h->pk_lm_tc, (size_t)D.n_lm_tc * D.nkt * 128 * 64));
+    rows.clear();
+    const uint16_t* lm = static_cast<const uint16_t*>(D.tied ? w->embed : w->lm_head);
+    for (int v = 0; v < D.n_lm_tc * 128; ++v) rows.push_back(v < D.V ? lm + (size_t)v * rowH : nullptr);
+    MK_TRY(pack_tc_tiles(rows, h->pk_lm_tc, D.nkt));
+  }
   return MK_OK;
 }
 
@@ -284,6 +362,8 @@ void resolve_pointers(Tape& t, const Dims& D, const mk_weights* w, const mk_ctx*
       case OP_GU: I.ptr[0] = h->pk_gu + pk_gu_elems(D) * l; I.ptr[3] = w->mlp_norm[l]; break;
       case OP_DOWN: I.ptr[0] = h->pk_dn + pk_dn_elems(D) * l; break;
       case OP_LM: I.ptr[0] = lm; I.ptr[3] = w->final_norm; break;
+      case OP_GU_TC: I.ptr[0] = h->pk_gu_tc + pk_gu_tc_elems(D) * l; I.ptr[3] = w->mlp_norm[l]; break;
+      case OP_LM_TC: I.ptr[0] = h->pk_lm_tc; I.ptr[3] = w->final_norm; break;
       default: break;
     }
   }
@@ -379,10 +459,7 @@ mk_status build(mk_ctx* h, const mk_weights* w, int want_pages) {
   h->sm = smem_layout(D, h->nbt, max_dyn, want_pages);
   if (h->sm.ring_pages < kConsumerWarps) return MK_ERR_UNSUPPORTED;
   if (h->sm.ring_pages > 64) return MK_ERR_UNSUPPORTED;
-  // the specialised kernel when every unit has the same row count and the attention one known form
-  const int rq = 2 * D.RP, ro = D.Ro, rg = 2 * D.Rgu, rd = D.Rdn, rl = D.Rlm;
-  if (rq == 4 && ro == 4 && rg == 4 && rd == 4 && rl == 4 && D.d == 64 && D.rep == 4 && !D.kv_fp16) h->spec = 1;
-  else if (rq == 2 && ro == 2 && rg == 2 && rd == 2 && rl == 2 && D.d == 128 && D.rep == 4 && D.kv_fp16) h->spec = 2;
+  h->spec = kernel_spec(D);
   for (int nbt : {1, 2, 4, 8})
     MK_TRY(from_cuda(cudaFuncSetAttribute(kernel_for(nbt, h->spec), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           h->sm.total)));
@@ -503,12 +580,14 @@ extern "C" mk_status mk_rope_inv_freq(const mk_config* cfg, double* out, int32_t
 }
 
 extern "C" mk_status mk_plan_check(const mk_config* cfg, int32_t n_sm, int32_t nb, int32_t fault,
-                                   int32_t dyn_percent, int32_t region, mk_plan_report* rep) {
+                                   int32_t dyn_percent, int32_t region, int32_t tensor_core_units,
+                                   mk_plan_report* rep) {
   if (!cfg || !rep || n_sm < 1 || dyn_percent < 0 || dyn_percent > 90) return MK_ERR_INVALID_ARG;
   if (region < REGION_ALL || region > REGION_LM) return MK_ERR_INVALID_ARG;
+  if (tensor_core_units < 0 || tensor_core_units > 4) return MK_ERR_INVALID_ARG;
   memset(rep, 0, sizeof(*rep));
   Dims D;
-  std::string why = dims_from_config(cfg, n_sm, &D);
+  std::string why = dims_from_config(cfg, n_sm, &D, tensor_core_units);
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
   if (nb < 1 || nb > D.max_batch) return MK_ERR_INVALID_ARG;
   Tape t = lower(D, n_sm, nb, dyn_percent > 0 ? dyn_percent : kDynPercent, region);
@@ -547,6 +626,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   if (o.wait_limit_ms < 0 || o.n_sm < 0 || o.ring_pages < 0 || o.device < 0) return MK_ERR_INVALID_ARG;
   if (o.dyn_percent < 0 || o.dyn_percent > 90) return MK_ERR_INVALID_ARG;
   if (o.region_cut != 0 && o.region_cut != 1) return MK_ERR_INVALID_ARG;
+  if (o.tensor_core_units < 0 || o.tensor_core_units > 4) return MK_ERR_INVALID_ARG;
   Dims D;
   std::string why = dims_from_config(cfg, 148, &D);  // validation only; rederived below
   if (!why.empty()) return MK_ERR_UNSUPPORTED;
@@ -567,7 +647,7 @@ extern "C" mk_status mk_create(const mk_config* cfg, const mk_weights* w, const 
   h->wait_limit_ns = (unsigned long long)(o.wait_limit_ms > 0 ? o.wait_limit_ms : 1000) * 1000000ull;
   h->dyn_percent = o.dyn_percent > 0 ? o.dyn_percent : kDynPercent;
   h->region_cut = o.region_cut ? 1 : 0;
-  why = dims_from_config(cfg, h->n_sm, &h->D);
+  why = dims_from_config(cfg, h->n_sm, &h->D, o.tensor_core_units);
   h->nbt = lanes_template(cfg->max_batch);
   mk_status s = why.empty() ? build(h, w, o.ring_pages) : MK_ERR_UNSUPPORTED;
   if (s == MK_OK && !o.prefill_tokenwise && prefill_supported(h->D))

@@ -43,6 +43,7 @@
 #include "mk_device.cuh"
 #include "mk_matvec.cuh"
 #include "mk_plan.h"
+#include "mk_tc.cuh"
 
 namespace mk {
 
@@ -172,6 +173,11 @@ struct Misc {
   volatile uint32_t cons_seq;
   volatile uint32_t last_claim;
   int entry_abort;
+  // Tensor-core units (8-lane kernel of the Llama-3.2-1B shape family): the two
+  // accumulators in tensor memory (written: tc_accf, read back: tc_acce) and the
+  // tensor-memory base address.
+  uint64_t tc_accf[2], tc_acce[2];
+  uint32_t tmem_base;
 };
 // the misc region is what smem_layout leaves after the barriers: 8192 - 8 * (128 + 64)
 static_assert(sizeof(Misc) <= 8192 - 8 * (128 + 64), "Misc does not fit its shared-memory region");
@@ -542,6 +548,19 @@ static __device__ __noinline__ void producer(const KParams& p, uint8_t* ring, ui
           rp.advance(1, NP);
         }
       }
+    } else if (I.op == OP_GU_TC || I.op == OP_LM_TC) {
+      // a unit is a 128-row block: its nkt K tiles, each one contiguous 16 KiB tile
+      const uint16_t* base = static_cast<const uint16_t*>(I.ptr[0]);
+      for (uint32_t k = 0; k < I.n_units && ok; ++k)
+        for (int kt = 0; kt < D.nkt && ok; ++kt) {
+          if (!(ok = wait_mbar(p, &empty[rp.slot], rp.sphase ^ 1u, E_WAIT_EMPTY, ii, true))) break;
+          mbar_arrive_expect_tx(&full[rp.fidx], (uint32_t)kPageBytes);
+          bulk_g2s(ring + (size_t)rp.slot * kPageBytes,
+                   base + ((size_t)(I.u0 + k) * D.nkt + kt) * (kPageBytes / 2), (uint32_t)kPageBytes,
+                   &full[rp.fidx], pol);
+          ++pidx;
+          rp.advance(1, NP);
+        }
     } else {
       // The static units, then (dynamic tail) the chunks this SM claims from the
       // phase's pool.  Three claims are in flight at a time (the first one issued
@@ -681,9 +700,13 @@ static __device__ __noinline__ Chunk8<NBT> acc_chunk_slow(const KParams& p, cons
 // applies RMSNorm with the bf16 gain.  Lanes >= nb are zero.
 enum { ST_EMB = 0, ST_ONE = 1, ST_ACC = 2 };
 
-template <int NBT, int MODE, bool NORM>
+// BOP: write the staged values instead as the tensor cores' B operand (8 lanes,
+// K-major, 128-byte swizzle): row b the bf16 high part of lane b, row 8 + b the low
+// part, one 2 KiB tile per 64 K (16 rows x 128 bytes, 8-row groups 1 KiB apart).
+template <int NBT, int MODE, bool NORM, bool BOP = false>
 __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, const float* src, int ld,
                                       int K, const uint16_t* gain, uint32_t ii) {
+  static_assert(!BOP || NBT == 8, "the B operand holds 8 lanes");
   const int ct = threadIdx.x - 32, cw = ct >> 5, lane = ct & 31;
   const int nch = K >> 3;
   float4* lo = reinterpret_cast<float4*>(act);
@@ -769,10 +792,21 @@ __device__ __forceinline__ void stage(const KParams& p, float* act, Misc* misc, 
           v[e] *= g[e];
         }
       }
-      lo[b * nch + c] = make_float4(v[0], v[1], v[2], v[3]);
-      hi[b * nch + c] = make_float4(v[4], v[5], v[6], v[7]);
+      if constexpr (BOP) {
+        uint16_t h8[8], l8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) split_bf16(v[e], h8[e], l8[e]);
+        uint8_t* tile = reinterpret_cast<uint8_t*>(act) + (size_t)(c >> 3) * 2048;
+        const int cs = ((c & 7) ^ (b & 7)) << 4;
+        *reinterpret_cast<uint4*>(tile + (b & 7) * 128 + cs) = *reinterpret_cast<const uint4*>(h8);
+        *reinterpret_cast<uint4*>(tile + 1024 + (b & 7) * 128 + cs) = *reinterpret_cast<const uint4*>(l8);
+      } else {
+        lo[b * nch + c] = make_float4(v[0], v[1], v[2], v[3]);
+        hi[b * nch + c] = make_float4(v[4], v[5], v[6], v[7]);
+      }
     }
   }
+  if constexpr (BOP) fence_proxy_async_smem();  // the tensor cores read the operand through the async proxy
   if (NORM) {
 #pragma unroll
     for (int b = 0; b < NBT; ++b) {
@@ -1144,6 +1178,130 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
   __syncwarp();
   if (lane == 0 && I.sig != kNoCounter) red_relaxed_add(p.ctr + I.sig, 1u);
   if constexpr (OPK == OP_LM) lm_finish<NBT>(p, misc, best);
+}
+
+// ---------------------------------------------------------------- consumers: tensor-core units
+
+// Gate/up (OP_GU_TC) or the LM head (OP_LM_TC) of the 8-lane kernel on the
+// tcgen05 tensor cores: a unit is a 128-row block of the weights over the whole
+// K, streamed as nkt ring pages of 128 rows x 64 (16 KiB, pre-swizzled when the
+// handle was created).  The staged activation is the B operand (stage<..., BOP>):
+// 8 lanes' bf16 high parts then their low parts, N = 16, so the fp32 accumulator
+// D[row][b] + D[row][8 + b] keeps the activations' fp32-level accuracy.  Consumer
+// warp 0, lane 0 issues the MMAs (M = 128, N = 16, K = 16; four per page) into one
+// of two 16-column accumulators in tensor memory and releases each page's ring
+// slot by committing to its empty barrier (it completes when the MMAs have read
+// the page, without the issuer waiting for them); warps 4-7
+// (lane quarters 0-3 of tensor memory, one block row per thread) read an
+// accumulator back, scale it by the lanes' 1/rms and run the epilogue: for
+// gate/up, whose block rows alternate gate and up rows of the same ffn index, the
+// two values meet by one shuffle and the even lane writes silu(g) * u; for the LM
+// head, logits and the running argmax.  tc_n / tc_q count the units and pages of
+// every tensor-core instruction so far in this launch (tc_n gives the accumulator
+// barriers' parities).  Measured faster than the CUDA cores with 8 lanes, where the CUDA-core
+// matvec reads 32 bytes of activations from shared memory per 16 bytes of weights.
+template <int OPK>
+static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
+                                                const float* act, uint64_t* full, uint64_t* empty, Misc* misc,
+                                                uint32_t ii, uint32_t& tc_n, uint32_t& tc_q) {
+  constexpr int NBT = 8;
+  static_assert(OPK == OP_GU_TC || OPK == OP_LM_TC, "tensor-core op");
+  const Dims& D = p.D;
+  const int ct = threadIdx.x - 32, lane = ct & 31;
+  const int warp = threadIdx.x >> 5;  // 1..8; warp w reads tensor-memory lanes 32 (w % 4) ..
+  const uint32_t NP = (uint32_t)p.ring_pages;
+  const int nkt = D.nkt;
+  const uint32_t tmem = misc->tmem_base;
+  const uint32_t bsm = smem_u32(act);
+  constexpr uint32_t kIdesc = idesc_bf16(128, 16);
+  float rinv[NBT];
+  norm_scales<NBT>(p, misc, D.H, rinv);
+  float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
+  float* lg = nullptr;
+  if (OPK == OP_LM_TC && p.logits) {
+    if (!p.logits_last) lg = p.logits + (size_t)misc->step * p.nb * D.V;
+    else if (misc->step == p.n_steps - 1) lg = p.logits;
+  }
+  LmBest<NBT> best;
+#pragma unroll
+  for (int b = 0; b < NBT; ++b) { best.v[b] = -CUDART_INF_F; best.i[b] = 0x7FFFFFFF; }
+
+  if (warp == 1) {
+    if (lane == 0) {  // the MMA issuer
+      RingPos rp;
+      rp.init(page_base, NP);
+      bool ok = true;
+      for (uint32_t k = 0; k < I.n_units; ++k) {
+        const uint32_t n = tc_n + k, buf = n & 1u;
+        // the epilogue has read this accumulator's previous unit
+        if (ok) ok = wait_mbar(p, &misc->tc_acce[buf], ((n >> 1) & 1u) ^ 1u, E_WAIT_FULL, ii, true);
+        tc_fence_after();
+        for (int kt = 0; kt < nkt; ++kt, rp.advance(1, NP)) {
+          if (ok) ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+          if (ok) {
+            tc_fence_after();
+            const uint32_t a = smem_u32(ring + (size_t)rp.slot * kPageBytes), bb = bsm + (uint32_t)kt * 2048u;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              umma_f16(tmem + buf * 16u, sw128_desc(a + 32u * j), sw128_desc(bb + 32u * j), kIdesc,
+                       (kt | j) != 0 ? 1u : 0u);
+          }
+          // the slot is free once these MMAs have read the page: each commit arrives
+          // on its empty barrier when every MMA issued so far has completed, and the
+          // barrier counts the 8 arrivals a consumer page release gives
+#pragma unroll
+          for (int c = 0; c < kConsumerWarps; ++c) umma_commit(&empty[rp.slot]);
+          ++tc_q;
+        }
+        umma_commit(&misc->tc_accf[buf]);  // the unit's accumulator is complete
+      }
+    }
+  } else if (warp >= 4) {
+    if (warp <= 7) {  // the epilogue: tensor-memory lane quarter warp % 4
+      const int qd = warp & 3;
+      for (uint32_t k = 0; k < I.n_units; ++k) {
+        const uint32_t n = tc_n + k, buf = n & 1u;
+        const bool ok =
+            __all_sync(0xFFFFFFFFu, wait_mbar(p, &misc->tc_accf[buf], (n >> 1) & 1u, E_WAIT_FULL, ii, true));
+        tc_fence_after();
+        uint32_t r[16];
+        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + buf * 16u, r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&misc->tc_acce[buf]);
+        if (!ok) continue;
+        float v[NBT];
+#pragma unroll
+        for (int b = 0; b < NBT; ++b) v[b] = (__uint_as_float(r[b]) + __uint_as_float(r[8 + b])) * rinv[b];
+        const int u = (int)(I.u0 + k);
+        if constexpr (OPK == OP_GU_TC) {
+          const int row = 32 * qd + lane, f = 64 * u + (row >> 1);  // even rows gate, odd rows up
+#pragma unroll
+          for (int b = 0; b < NBT; ++b) {
+            const float up = __shfl_xor_sync(0xFFFFFFFFu, v[b], 1);
+            if (!(lane & 1) && b < p.nb && f < D.F)
+              st_relaxed_f32(lay + p.off_a + (size_t)b * D.F + f, canon(v[b] / (1.0f + __expf(-v[b])) * up));
+          }
+        } else {
+          const int row = 128 * u + 32 * qd + lane;
+          if (row < D.V) {
+#pragma unroll
+            for (int b = 0; b < NBT; ++b) {
+              if (b >= p.nb) break;
+              if (lm_better(v[b], row, best.v[b], best.i[b])) { best.v[b] = v[b]; best.i[b] = row; }
+              if (lg) lg[(size_t)b * D.V + row] = v[b];
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_n += I.n_units;
+  // this warp's share is written: bump the hint counter (every warp, as the matvec does)
+  __syncwarp();
+  if (lane == 0 && I.sig != kNoCounter) red_relaxed_add(p.ctr + I.sig, 1u);
+  if constexpr (OPK == OP_LM_TC) lm_finish<NBT>(p, misc, best);
 }
 
 // ---------------------------------------------------------------- consumers: attention
@@ -1700,6 +1858,16 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
   const uint32_t i0 = p.sm_off[blockIdx.x], i1 = p.sm_off[blockIdx.x + 1];
   uint32_t page_base = 0;
   const int half = D.d / 2;
+  // tensor-core units: the 8-lane kernel of the Llama-3.2-1B shape family holds two
+  // 16-column fp32 accumulators in tensor memory for the whole launch
+  constexpr bool kTC = NBT == 8 && SPEC == 1;
+  uint32_t tc_n = 0, tc_q = 0;
+  if constexpr (kTC) {
+    if (ct < 32) tmem_alloc(&misc->tmem_base, 32);
+    tc_fence_before();
+    cbar();
+    tc_fence_after();
+  }
   for (int t = 0; t < p.n_steps; ++t) {
   // step t begins once step t - 1 has written its ids everywhere (acquire): its
   // tokens, every read of its activations and every write of its KV rows are done
@@ -1824,6 +1992,24 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
         if (rec) rec[11] = (long long)globaltimer_ns();
         mv_dispatch<OP_LM, NBT, SPEC>(D.Rlm, p, I, page_base, ring, act, D.H, full, empty, misc, ii);
         break;
+      case OP_GU_TC:
+        if constexpr (kTC) {
+          stage<NBT, ST_ONE, true, true>(p, act, misc, lay + p.off_x1, D.H, D.H,
+                                         static_cast<const uint16_t*>(I.ptr[3]), ii);
+          if (rec) rec[11] = (long long)globaltimer_ns();
+          mv_units_tc<OP_GU_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n, tc_q);
+          used = I.n_units * (uint32_t)D.nkt;
+        }
+        break;
+      case OP_LM_TC:
+        if constexpr (kTC) {
+          stage<NBT, ST_ACC, true, true>(p, act, misc, reinterpret_cast<const float*>(acc_of(p, misc, D.L - 1)),
+                                         D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), ii);
+          if (rec) rec[11] = (long long)globaltimer_ns();
+          mv_units_tc<OP_LM_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n, tc_q);
+          used = I.n_units * (uint32_t)D.nkt;
+        }
+        break;
     }
     if (I.pool) used = (uint32_t)misc->dyn_end[((uint32_t)t * misc->n_instr + (ii - i0)) & 15] - page_base;
     page_base += used;
@@ -1854,6 +2040,12 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
   // a stop raised later in this step is acted on after the next step's barrier,
   // where every warp reads the flag at the same point
   }
+  if constexpr (kTC) {  // every MMA has completed (its accumulator was read back)
+    tc_fence_before();
+    cbar();
+    tc_fence_after();
+    if (ct < 32) tmem_dealloc(misc->tmem_base, 32);
+  }
 }
 
 // ---------------------------------------------------------------- the kernel
@@ -1880,6 +2072,10 @@ __global__ void __launch_bounds__(kThreads, 1) mk_decode_kernel(const __grid_con
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * p.ring_pages; ++i) mbar_init(&full[i], 1);
     for (int i = 0; i < p.ring_pages; ++i) mbar_init(&empty[i], kConsumerWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&misc->tc_accf[i], 1);
+      mbar_init(&misc->tc_acce[i], 4);  // the four epilogue warps
+    }
     fence_barrier_init();
     fence_proxy_async_smem();
     misc->stop = 0;

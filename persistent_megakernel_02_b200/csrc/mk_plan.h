@@ -31,6 +31,11 @@ enum Op : uint8_t {
   OP_GU = 4,    // RMSNorm(x) -> rows of Wgate and Wup -> a = silu(g) * u
   OP_DOWN = 5,  // rows of Wdown over one K slice . a -> that slice's partial of the residual
   OP_LM = 6,    // RMSNorm(x) -> rows of the LM head -> logits, running argmax; last reduces
+  // 8-lane kernels of handles with packed tensor-core tiles (Dims::tc): the same
+  // ops on tcgen05, a unit being one 128-row block over the whole K (nkt pages of
+  // 128 rows x 64 in the 128-byte swizzled layout)
+  OP_GU_TC = 7,  // block u: rows 2i / 2i + 1 = W_gate / W_up row 64 u + i -> a = silu(g) * u
+  OP_LM_TC = 8,  // block u: LM-head rows 128 u .. 128 u + 127 -> logits, running argmax
 };
 
 constexpr int kPageBytes = 16384;      // one ring page
@@ -83,6 +88,10 @@ struct Dims {
   float eps;
   int tied;
   int kv_fp16;    // KV cache element: 0 bf16, 1 fp16
+  // tensor-core units in the 8-lane tapes: bit 0 the LM head, bit 1 gate/up (0: none)
+  int tc;
+  int nkt;        // 64-wide K tiles of a hidden-size row (tc units)
+  int n_gu_tc, n_lm_tc;  // 128-row blocks of gate/up (F / 64) and of the LM head
 };
 
 // Which part of a decode step a tape holds.  The whole step is one launch; the
@@ -97,6 +106,7 @@ enum Region : int { REGION_ALL = 0, REGION_LAYERS = 1, REGION_LM = 2 };
 struct Tape {
   int nb = 0;
   int region = REGION_ALL;
+  int tc = 0;                     // gate/up and LM head as tensor-core units
   int S = 1;                      // attention slices per (lane, kv head)
   int n_counters = 0;
   std::vector<uint32_t> sm_off;   // n_sm + 1 offsets into instrs

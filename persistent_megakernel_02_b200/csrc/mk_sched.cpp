@@ -85,6 +85,10 @@ std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, i
   D.n_gu = (ffn + D.Rgu - 1) / D.Rgu;
   D.n_dn = (hidden + D.Rdn - 1) / D.Rdn;
   D.n_lm = (vocab + D.Rlm - 1) / D.Rlm;
+  D.tc = 0;  // enabled by the handle when its kernels can run the tensor-core units
+  D.nkt = hidden / 64;
+  D.n_gu_tc = ffn / 64;
+  D.n_lm_tc = (vocab + 127) / 128;
   if (n_counters(D) >= kNoCounter) return "too many counters for this shape";
   *out = D;
   return "";
@@ -104,6 +108,8 @@ static int64_t unit_bytes(const Dims& D, int op, int S) {
     case OP_GU: return 2LL * 2 * D.Rgu * D.H;
     case OP_DOWN: return 2LL * D.Rdn * D.KS;
     case OP_LM: return 2LL * D.Rlm * D.H;
+    case OP_GU_TC:
+    case OP_LM_TC: return (int64_t)D.nkt * kPageBytes;
     case OP_ATTN: {
       int pages = (D.pages_per_seq + S - 1) / S;
       return (int64_t)pages * kPageBytes;
@@ -147,6 +153,9 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent, int region) {
   Tape t;
   t.nb = nb;
   t.region = region;
+  // 5-8 lanes run the 8-lane kernel, whose LM head (bit 0) and gate/up (bit 1) may
+  // use the tensor cores
+  t.tc = lanes_template(nb) == 8 ? D.tc : 0;
   t.S = attn_slices(D, n_sm, nb);
   t.n_counters = n_counters(D);
   std::vector<int64_t> load(n_sm, 0);
@@ -214,8 +223,12 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent, int region) {
     for (int s = 0; s < n_sm; ++s)
       if (!o[s].empty()) emit(s, OP_O, l, o[s], (uint16_t)ctr_layer(l, C_ATTN), (uint16_t)ctr_layer(l, C_O), 0);
     // RMSNorm + gate/up + SwiGLU
-    phase(OP_GU, l, D.n_gu, 0, n_sm, (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0,
-          pool_gu(D, l), false);
+    if (t.tc & 2)
+      phase(OP_GU_TC, l, D.n_gu_tc, 0, n_sm, (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0, -1,
+            false);
+    else
+      phase(OP_GU, l, D.n_gu, 0, n_sm, (uint16_t)ctr_layer(l, C_O), (uint16_t)ctr_layer(l, C_GU), 0,
+            pool_gu(D, l), false);
     // down projection + residual: SMs split into one group per K slice
     for (int ks = 0; ks < D.n_ks; ++ks) {
       int lo = (int)((long long)n_sm * ks / D.n_ks), hi = (int)((long long)n_sm * (ks + 1) / D.n_ks);
@@ -228,8 +241,9 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent, int region) {
   // final norm + LM head + argmax: every SM takes part (possibly with no rows)
   // (in its own launch it waits on nothing: the launch boundary orders it)
   if (region != REGION_LAYERS)
-    phase(OP_LM, D.L, D.n_lm, 0, n_sm, region == REGION_LM ? kNoCounter : (uint16_t)ctr_layer(D.L - 1, C_DOWN),
-          kNoCounter, 0, pool_lm(D), true);
+    phase((t.tc & 1) ? OP_LM_TC : OP_LM, D.L, (t.tc & 1) ? D.n_lm_tc : D.n_lm, 0, n_sm,
+          region == REGION_LM ? kNoCounter : (uint16_t)ctr_layer(D.L - 1, C_DOWN), kNoCounter, 0,
+          (t.tc & 1) ? -1 : pool_lm(D), true);
 
   // wait targets = how many instructions signal the counter in one step
   std::vector<uint32_t> fan(t.n_counters, 0);
@@ -260,6 +274,9 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
   std::vector<int> cq((size_t)D.L * D.n_qkv, 0), co((size_t)D.L * D.n_o, 0),
       cg((size_t)D.L * D.n_gu, 0), cd((size_t)D.L * D.n_ks * D.n_dn, 0),
       ca((size_t)D.L * nb * D.Hkv * S, 0), cl(D.n_lm, 0);
+  // tensor-core tapes cover gate/up and/or the LM head in 128-row blocks instead
+  if (t.tc & 2) cg.assign((size_t)D.L * D.n_gu_tc, 0);
+  if (t.tc & 1) cl.assign(D.n_lm_tc, 0);
   std::vector<uint32_t> ip(n_sm);
   r.bytes_min = INT64_MAX; r.bytes_max = 0;
   // SMs taking part in each pool: each is expected to stream an equal share of it
@@ -321,9 +338,11 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
           switch (I.op) {
             case OP_QKV: bump(cq, (size_t)l * D.n_qkv + u); break;
             case OP_O: bump(co, (size_t)l * D.n_o + u); break;
-            case OP_GU: bump(cg, (size_t)l * D.n_gu + u); break;
+            case OP_GU: bump(cg, (size_t)l * D.n_gu + u); if (t.tc & 2) cover_err = true; break;
+            case OP_GU_TC: bump(cg, (size_t)l * D.n_gu_tc + u); if (!(t.tc & 2)) cover_err = true; break;
+            case OP_LM_TC: bump(cl, u); if (!(t.tc & 1)) cover_err = true; break;
             case OP_DOWN: bump(cd, ((size_t)l * D.n_ks + I.arg) * D.n_dn + u); break;
-            case OP_LM: bump(cl, u); break;
+            case OP_LM: bump(cl, u); if (t.tc & 1) cover_err = true; break;
             case OP_ATTN: {
               int b, g, sl;
               attn_unit(u, D.Hkv, S, &b, &g, &sl);
@@ -336,7 +355,7 @@ SimReport simulate(const Dims& D, int n_sm, const Tape& t) {
             }
           }
         }
-        if (I.op == OP_LM) { ctr[ctr_lm(D)]++; signals[ctr_lm(D)]++; }
+        if (I.op == OP_LM || I.op == OP_LM_TC) { ctr[ctr_lm(D)]++; signals[ctr_lm(D)]++; }
         if (I.sig != kNoCounter) { ctr[I.sig]++; signals[I.sig]++; }
         ip[s]++;
         progress = true;

@@ -15,7 +15,7 @@ import sys
 
 import numpy as np
 
-OPS = {1: "qkv", 2: "attn", 3: "o", 4: "gu", 5: "down", 6: "lm"}
+OPS = {1: "qkv", 2: "attn", 3: "o", 4: "gu", 5: "down", 6: "lm", 7: "gu_tc", 8: "lm_tc"}
 
 
 def flatten(rec: np.ndarray) -> list[dict]:
@@ -112,7 +112,7 @@ def summarize(rec: np.ndarray) -> dict:
     chain = []
     if mid:
         base = phases.get((mid[0], "qkv"), next(iter(phases.values())))["first_dep"]
-        order = ["qkv", "attn", "o", "gu", "down"]
+        order = ["qkv", "attn", "o", "gu", "gu_tc", "down"]
         for layer in mid:
             for op in order:
                 ph = phases.get((layer, op))
@@ -123,8 +123,8 @@ def summarize(rec: np.ndarray) -> dict:
     # head): percentiles of each SM's start, units time and end, from the phase's
     # first start
     spread = {}
-    for op in ("gu", "down", "lm"):
-        lay = mid[0] if op != "lm" and mid else None
+    for op in ("gu", "gu_tc", "down", "lm", "lm_tc"):
+        lay = mid[0] if op not in ("lm", "lm_tc") and mid else None
         rs = [r for r in rows if r["op"] == op and (lay is None or r["layer"] == lay)]
         if not rs:
             continue
@@ -171,7 +171,7 @@ def markdown(s: dict, bench_us: float | None = None) -> str:
     out.append("| op | window | barrier wait | stage | entry | first page | pages | dot/page | "
                "epilogue/page | page wait/page | slot wait/page | pages/SM |")
     out.append("|---|---|---|---|---|---|---|---|---|---|---|---|")
-    for op in ("qkv", "attn", "o", "gu", "down", "lm"):
+    for op in ("qkv", "attn", "o", "gu", "gu_tc", "down", "lm", "lm_tc"):
         if op not in po:
             continue
         d = po[op]

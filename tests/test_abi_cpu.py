@@ -185,4 +185,18 @@ def test_region_cut_tapes_are_deadlock_free_and_split_the_outputs(wl):
 def test_plan_check_rejects_an_unknown_region():
     c = mk.config_struct(configs.model_config("tiny"))
     rep = mk.MkPlanReport()
-    assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 3, ctypes.byref(rep)) == 1
+    assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 3, 0, ctypes.byref(rep)) == 1
+    assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 0, 5, ctypes.byref(rep)) == 1
+
+
+@pytest.mark.parametrize("units", [2, 3, 4])
+@pytest.mark.parametrize("region", [0, 1, 2])
+def test_tensor_core_unit_tapes_cover_their_blocks(units, region):
+    """With 5-8 lanes the Llama-3.2-1B-shaped kernel can run the LM head (2), gate/up
+    (3) or both (4) as 128-row tensor-core blocks: every block once, the CUDA-core
+    form of the same op not at all, deadlock-free, in each region of a cut too; 1-4
+    lanes keep the CUDA-core ops."""
+    cfg = configs.model_config("llama1b_bs8")
+    for nb in (8, 5, 4, 1):
+        r = mk.plan_check(cfg, 148, nb, region=region, tensor_core_units=units)
+        assert r["deadlock_free"] and r["coverage_ok"] and r["targets_ok"], (units, region, nb, r)

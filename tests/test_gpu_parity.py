@@ -415,3 +415,33 @@ def test_region_cut_gives_the_single_launch_results_bit_for_bit(wl, nb):
     np.testing.assert_array_equal(runs[0][1], runs[1][1])
     np.testing.assert_array_equal(runs[0][2], runs[1][2])
     np.testing.assert_array_equal(runs[0][3], runs[1][3])
+
+
+@pytest.mark.parametrize("nb,units", [(8, 4), (5, 4), (8, 2)])
+def test_tensor_core_units_match_oracle_and_cuda_cores(nb, units):
+    """5-8 lanes run the 8-lane kernel, whose gate/up and LM head can run on tcgen05
+    tensor cores (128-row blocks, accumulators in tensor memory).  A 2-layer model
+    of the Llama-3.2-1B shape with a ragged vocabulary (32001 rows: the last block
+    holds one row) matches the oracle at every teacher-forced step, and the same
+    handle on CUDA cores only within summation-order differences."""
+    cfg = configs.model_config("llama1b_bs8", max_batch=8, max_seq=96, n_layers=2, vocab=32001)
+    w = H.gpu_weights(cfg)
+    prompts = [synth.prompt_tokens(cfg, b, 20 + 7 * b).numpy() for b in range(nb)]
+    teacher = [synth.teacher_tokens(cfg, b, 6).numpy() for b in range(nb)]
+    runs = []
+    for sel in (units, 1):  # the tensor-core units asked for, then none
+        mk = _mk(cfg, w, tensor_core_units=sel)
+        runs.append(H.run_teacher_forced(mk, cfg, prompts, teacher, 6))
+        mk.close()
+    (pre, lg, ids), (pre_cc, lg_cc, _) = runs
+    np.testing.assert_allclose(lg, lg_cc, atol=5e-3, rtol=0)
+    orc = H.oracle_for(cfg, w)
+    worst, checked = (0.0, 0.0), 0
+    for b in range(nb):
+        w_pre, w_steps = H.oracle_teacher_forced(orc, prompts[b], teacher[b], 6)
+        H.compare_logits(pre[b], w_pre, f"lane {b} prefill")
+        for t in range(6):
+            e = H.compare_logits(lg[t, b], w_steps[t], f"lane {b} step {t}")
+            worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+            checked += H.compare_ids(ids[t, b], w_steps[t], f"lane {b} step {t}")
+    H.record(f"tensor-core units {units}, 2-layer 1B shape, vocab 32001, x{nb} lanes", worst, 6, checked)
