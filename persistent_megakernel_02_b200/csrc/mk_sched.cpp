@@ -94,9 +94,15 @@ std::string derive_dims(int n_layers, int hidden, int n_heads, int n_kv_heads, i
   return "";
 }
 
+// Attention units per (lane, kv head): as many as the SMs allow, but no more than
+// there is work for -- a slice per KV page for long contexts, and for short ones
+// (the kernel's head split, attn_plan) one unit per query head, so at least rep
+// even where a sequence has fewer pages than its kv head has query heads (short
+// max_seq); capping that at the page count disabled the head split (Llama-3.2-1B
+// batch 1 with max_seq 93: 487 us/step instead of 456).
 int attn_slices(const Dims& D, int n_sm, int nb) {
   int s = n_sm / (nb * D.Hkv);
-  s = std::max(1, std::min(s, D.pages_per_seq));
+  s = std::max(1, std::min(s, std::max(D.pages_per_seq, D.rep)));
   return std::min(s, 65535);
 }
 
