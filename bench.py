@@ -105,7 +105,7 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-KERNEL_SOURCES = ["mk_kernel.cuh", "mk_device.cuh", "mk_matvec.cuh", "mk_plan.h", "mk_sched.cpp", "mk_api.cu"]
+KERNEL_SOURCES = ["mk_kernel.cuh", "mk_device.cuh", "mk_matvec.cuh", "mk_tc.cuh", "mk_plan.h", "mk_sched.cpp", "mk_api.cu"]
 
 
 def kernel_src_hash() -> str:
