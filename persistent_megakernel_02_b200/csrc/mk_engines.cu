@@ -64,7 +64,8 @@ constexpr int kTcTileBytes = kTcRows * kTcKTile * 2;  // 16 KiB
 constexpr int kTcBTileBytes = kTcN * kTcKTile * 2;    // 2 KiB of activations per K tile
 constexpr int kTcThreads = 256;  // warp 0: TMA, warp 1: MMA, warps 4-7: accumulator read-back
 constexpr int kTcMaxK = 4096;
-constexpr int kTcTmemCols = 32;  // two accumulators of N = 16 fp32 columns
+constexpr int kTcAccs = 8;       // N = 16 accumulators per buffer: MMA j of tile kt -> (kt & 1) * 4 + j
+constexpr int kTcTmemCols = 2 * kTcAccs * kTcN;  // two buffers
 
 constexpr uint32_t kTcIdesc = idesc_bf16(kTcRows, kTcN);
 
@@ -155,8 +156,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t bbase = smem_u32(bsm + kt * kTcBTileBytes);
 #pragma unroll
           for (int j = 0; j < kTcKTile / 16; ++j)
-            umma_bf16(tmem + (uint32_t)(a * kTcN), sw128_desc(abase + j * 32), sw128_desc(bbase + j * 32),
-                      (kt | j) != 0 ? 1u : 0u);
+            umma_bf16(tmem + (uint32_t)((a * kTcAccs + (kt & 1) * 4 + j) * kTcN), sw128_desc(abase + j * 32),
+                      sw128_desc(bbase + j * 32), kt >= 2 ? 1u : 0u);
           umma_commit(&empty[s]);  // the tile's slot is free once these MMAs have read it
         }
         if (ok) umma_commit(&accf[a]);
@@ -172,19 +173,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int a = i & 1, use = i >> 1;
       if (!eng_wait(&accf[a], use & 1, limit_ns, 5)) break;
       tc_fence_after();
-      uint32_t r[16];
-      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * kTcN);
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-          "%14, %15}, [%16];"
-          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-            "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-          : "r"(taddr));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      // the accumulators the block wrote (tiles 0 and 1 start them), two per load
+      const int na = nkt >= 2 ? kTcAccs : kTcAccs / 2;
+      float y[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(a * kTcAccs * kTcN);
+      for (int c = 0; c < na; c += 2) {
+        uint32_t r[32];
+        tmem_ld32(taddr + (uint32_t)(c * kTcN), r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int b = 0; b < 8; ++b)
+          y[b] += (__uint_as_float(r[b]) + __uint_as_float(r[8 + b])) +
+                  (__uint_as_float(r[16 + b]) + __uint_as_float(r[24 + b]));
+      }
       const int row = blk * kTcRows + q * 32 + lane;
 #pragma unroll
       for (int b = 0; b < 8; ++b)
-        if (b < nb) Y[(size_t)b * rows + row] = __uint_as_float(r[b]) + __uint_as_float(r[8 + b]);
+        if (b < nb) Y[(size_t)b * rows + row] = y[b];
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acce[a]);

@@ -1189,17 +1189,23 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
 // 8 lanes' bf16 high parts then their low parts, N = 16, so the fp32 accumulator
 // D[row][b] + D[row][8 + b] keeps the activations' fp32-level accuracy.  Consumer
 // warp 0, lane 0 issues the MMAs (M = 128, N = 16, K = 16; four per page) into one
-// of two 16-column accumulators in tensor memory and releases each page's ring
-// slot by committing to its empty barrier (it completes when the MMAs have read
-// the page, without the issuer waiting for them); warps 4-7
-// (lane quarters 0-3 of tensor memory, one block row per thread) read an
-// accumulator back, scale it by the lanes' 1/rms and run the epilogue: for
+// of two accumulator buffers in tensor memory and releases each page's ring slot
+// by committing to its empty barrier (it completes when the MMAs have read the
+// page, without the issuer waiting for them).  A buffer is kTcAcc 16-column
+// accumulators: MMA j of page kt adds into accumulator (kt & 1) * 4 + j, so
+// consecutive MMAs never wait for one another's result (one accumulator for the
+// whole K chains them: each waits out the previous one's latency, ~0.55 us per
+// page measured).  Warps 4-7 (lane quarters 0-3 of tensor memory, one block row
+// per thread) read a buffer back, sum its accumulators, scale by the lanes'
+// 1/rms and run the epilogue: for
 // gate/up, whose block rows alternate gate and up rows of the same ffn index, the
 // two values meet by one shuffle and the even lane writes silu(g) * u; for the LM
 // head, logits and the running argmax.  tc_n / tc_q count the units and pages of
 // every tensor-core instruction so far in this launch (tc_n gives the accumulator
 // barriers' parities).  Measured faster than the CUDA cores with 8 lanes, where the CUDA-core
 // matvec reads 32 bytes of activations from shared memory per 16 bytes of weights.
+constexpr int kTcAcc = 8;                      // 16-column accumulators per buffer
+constexpr uint32_t kTcCols = 2 * kTcAcc * 16;  // tensor-memory columns: two buffers
 template <int OPK>
 static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
                                                 const float* act, uint64_t* full, uint64_t* empty, Misc* misc,
@@ -1214,6 +1220,7 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
   const uint32_t tmem = misc->tmem_base;
   const uint32_t bsm = smem_u32(act);
   constexpr uint32_t kIdesc = idesc_bf16(128, 16);
+  const int na = nkt >= 2 ? kTcAcc : kTcAcc / 2;  // accumulators a unit writes (pages 0 and 1 start them)
   float rinv[NBT];
   norm_scales<NBT>(p, misc, D.H, rinv);
   float* lay = misc->actset + (size_t)I.layer * p.layer_floats;
@@ -1226,8 +1233,12 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
 #pragma unroll
   for (int b = 0; b < NBT; ++b) { best.v[b] = -CUDART_INF_F; best.i[b] = 0x7FFFFFFF; }
 
+  // profile mode: the issuer's page waits (and the epilogue's time, per unit)
+  long long* prec = p.prof ? p.prof + ((size_t)blockIdx.x * p.prof_stride + (ii - misc->i0)) * kProfSlots : nullptr;
+  long long c_wait = 0, c_pages = 0, c_epi = 0;
   if (warp == 1) {
     if (lane == 0) {  // the MMA issuer
+      if (prec) { misc->warp_entry[0] = (long long)globaltimer_ns(); misc->warp_first[0] = 0; }
       RingPos rp;
       rp.init(page_base, NP);
       bool ok = true;
@@ -1237,20 +1248,27 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
         if (ok) ok = wait_mbar(p, &misc->tc_acce[buf], ((n >> 1) & 1u) ^ 1u, E_WAIT_FULL, ii, true);
         tc_fence_after();
         for (int kt = 0; kt < nkt; ++kt, rp.advance(1, NP)) {
+          const long long tw = prec ? (long long)globaltimer_ns() : 0;
           if (ok) ok = wait_mbar(p, &full[rp.fidx], rp.fphase, E_WAIT_FULL, ii, true);
+          if (prec) {
+            const long long now = (long long)globaltimer_ns();
+            c_wait += now - tw;
+            c_pages += 1;
+            if (misc->warp_first[0] == 0) misc->warp_first[0] = now;
+          }
           if (ok) {
             tc_fence_after();
             const uint32_t a = smem_u32(ring + (size_t)rp.slot * kPageBytes), bb = bsm + (uint32_t)kt * 2048u;
+            const uint32_t d = tmem + buf * (uint32_t)(kTcAcc * 16) + (uint32_t)(kt & 1) * 64u;
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              umma_f16(tmem + buf * 16u, sw128_desc(a + 32u * j), sw128_desc(bb + 32u * j), kIdesc,
-                       (kt | j) != 0 ? 1u : 0u);
+              umma_f16(d + 16u * j, sw128_desc(a + 32u * j), sw128_desc(bb + 32u * j), kIdesc, kt >= 2 ? 1u : 0u);
           }
-          // the slot is free once these MMAs have read the page: each commit arrives
-          // on its empty barrier when every MMA issued so far has completed, and the
-          // barrier counts the 8 arrivals a consumer page release gives
-#pragma unroll
-          for (int c = 0; c < kConsumerWarps; ++c) umma_commit(&empty[rp.slot]);
+          // the slot is free once these MMAs have read the page: the barrier counts
+          // the 8 arrivals a consumer page release gives; 7 now, and the last from a
+          // commit, when every MMA issued so far has completed
+          mbar_arrive_cnt(&empty[rp.slot], (uint32_t)kConsumerWarps - 1u);
+          umma_commit(&empty[rp.slot]);
           ++tc_q;
         }
         umma_commit(&misc->tc_accf[buf]);  // the unit's accumulator is complete
@@ -1263,17 +1281,27 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
         const uint32_t n = tc_n + k, buf = n & 1u;
         const bool ok =
             __all_sync(0xFFFFFFFFu, wait_mbar(p, &misc->tc_accf[buf], (n >> 1) & 1u, E_WAIT_FULL, ii, true));
+        const long long te = prec ? (long long)globaltimer_ns() : 0;
         tc_fence_after();
-        uint32_t r[16];
-        tmem_ld16(tmem + ((uint32_t)(32 * qd) << 16) + buf * 16u, r);
-        tmem_ld_wait();
+        float v[NBT];
+#pragma unroll
+        for (int b = 0; b < NBT; ++b) v[b] = 0.f;
+        const uint32_t ta = tmem + ((uint32_t)(32 * qd) << 16) + buf * (uint32_t)(kTcAcc * 16);
+        for (int a = 0; a < na; a += 2) {  // two accumulators per load
+          uint32_t r[32];
+          tmem_ld32(ta + 16u * (uint32_t)a, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int b = 0; b < NBT; ++b)
+            v[b] += (__uint_as_float(r[b]) + __uint_as_float(r[8 + b])) +
+                    (__uint_as_float(r[16 + b]) + __uint_as_float(r[24 + b]));
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&misc->tc_acce[buf]);
         if (!ok) continue;
-        float v[NBT];
 #pragma unroll
-        for (int b = 0; b < NBT; ++b) v[b] = (__uint_as_float(r[b]) + __uint_as_float(r[8 + b])) * rinv[b];
+        for (int b = 0; b < NBT; ++b) v[b] *= rinv[b];
         const int u = (int)(I.u0 + k);
         if constexpr (OPK == OP_GU_TC) {
           const int row = 32 * qd + lane, f = 64 * u + (row >> 1);  // even rows gate, odd rows up
@@ -1294,8 +1322,15 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
             }
           }
         }
+        if (prec) c_epi += (long long)globaltimer_ns() - te;
       }
     }
+  }
+  if (prec && lane == 0 && (c_pages || c_epi)) {  // summed over the warps, like the matvec's
+    unsigned long long* pr = reinterpret_cast<unsigned long long*>(prec);
+    atomicAdd(pr + 7, (unsigned long long)c_wait);
+    atomicAdd(pr + 8, (unsigned long long)c_pages);
+    atomicAdd(pr + 15, (unsigned long long)c_epi);
   }
   tc_n += I.n_units;
   // this warp's share is written: bump the hint counter (every warp, as the matvec does)
@@ -1859,11 +1894,11 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
   uint32_t page_base = 0;
   const int half = D.d / 2;
   // tensor-core units: the 8-lane kernel of the Llama-3.2-1B shape family holds two
-  // 16-column fp32 accumulators in tensor memory for the whole launch
+  // accumulator buffers (kTcCols fp32 columns) in tensor memory for the whole launch
   constexpr bool kTC = NBT == 8 && SPEC == 1;
   uint32_t tc_n = 0, tc_q = 0;
   if constexpr (kTC) {
-    if (ct < 32) tmem_alloc(&misc->tmem_base, 32);
+    if (ct < 32) tmem_alloc(&misc->tmem_base, kTcCols);
     tc_fence_before();
     cbar();
     tc_fence_after();
@@ -2044,7 +2079,7 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
     tc_fence_before();
     cbar();
     tc_fence_after();
-    if (ct < 32) tmem_dealloc(misc->tmem_base, 32);
+    if (ct < 32) tmem_dealloc(misc->tmem_base, kTcCols);
   }
 }
 

@@ -224,6 +224,8 @@ def main(argv=None):
     ap.add_argument("--from-json", default=None, help="render a saved JSON summary (no GPU)")
     ap.add_argument("--ring-pages", type=int, default=0)
     ap.add_argument("--dyn-percent", type=int, default=0, help="claimed share of the streaming phases (0: none)")
+    ap.add_argument("--tensor-core-units", type=int, default=0,
+                    help="8-lane matvecs on tcgen05 (mk_options.tensor_core_units; 0 measured default)")
     ap.add_argument("--max-seq-extra", type=int, default=181,
                     help="max_seq = prompt + this (181: bench.py's default sizing, which sets the "
                          "attention slices per kv head)")
@@ -237,7 +239,8 @@ def main(argv=None):
     nb, P = wl["batch"], max(wl["prompt_lens"])
     cfg = configs.model_config(args.workload, max_seq=P + max(8, args.max_seq_extra))
     w = synth.make_weights(cfg, device="cuda")
-    mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages, dyn_percent=args.dyn_percent)
+    mk = Megakernel(cfg, w, profile=1, ring_pages=args.ring_pages, dyn_percent=args.dyn_percent,
+                    tensor_core_units=args.tensor_core_units)
     prompts = [synth.prompt_tokens(cfg, b, wl["prompt_lens"][b]).tolist() for b in range(nb)]
     ids = torch.tensor([mk.prefill(b, prompts[b]) for b in range(nb)], dtype=torch.int32, device="cuda")
     pos = [len(p) for p in prompts]

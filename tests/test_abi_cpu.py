@@ -102,6 +102,43 @@ def test_create_rejects_missing_weights_before_touching_the_gpu():
     assert mk.STATUS[st] == "MK_ERR_INVALID_ARG"
 
 
+def _fake_weights(cfg):
+    """Non-null, 16-byte aligned placeholders: enough for mk_create's host checks,
+    never dereferenced before the device checks."""
+    L = cfg["n_layers"]
+    arrs = [(ctypes.c_void_p * L)(*([4096] * L)) for _ in range(9)]
+    w = mk.MkWeights(embed=4096, lm_head=None if cfg["tied"] else 4096, final_norm=4096,
+                     **{n: ctypes.cast(a, mk._PP) for n, a in zip(mk.Megakernel._LAYER, arrs)})
+    return w, arrs
+
+
+@pytest.mark.parametrize("field,value", [("tensor_core_units", 5), ("tensor_core_units", -1), ("region_cut", 2),
+                                         ("dyn_percent", 91), ("ring_pages", -1)])
+def test_create_rejects_out_of_range_options_before_touching_the_gpu(field, value):
+    cfg = configs.model_config("tiny")
+    c = mk.config_struct(cfg)
+    w, _keep = _fake_weights(cfg)
+    h = ctypes.c_void_p()
+    o = mk.MkOptions(**{field: value})
+    assert mk.STATUS[mk.lib().mk_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(o), ctypes.byref(h))] \
+        == "MK_ERR_INVALID_ARG"
+
+
+def test_create_accepts_the_options_range_up_to_the_device_checks():
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("placeholder weight pointers: the accepted case would reach the device")
+    cfg = configs.model_config("tiny")
+    c = mk.config_struct(cfg)
+    w, _keep = _fake_weights(cfg)
+    for kw in ({}, {"tensor_core_units": 4}, {"region_cut": 1}, {"dyn_percent": 90}):
+        h = ctypes.c_void_p()
+        o = mk.MkOptions(**kw)
+        st = mk.STATUS[mk.lib().mk_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(o), ctypes.byref(h))]
+        assert st == "MK_ERR_CUDA", (kw, st)  # past every host check: no device here
+
+
 def test_noalloc_head_rejects_bad_arguments_on_the_host():
     f = mk.lib().mk_greedy_head_noalloc
     ids = ctypes.c_void_p(16)

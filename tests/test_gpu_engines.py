@@ -29,7 +29,7 @@ def test_engine_rejects_bad_requests_on_the_host():
 @pytest.mark.gpu
 @pytest.mark.parametrize("engine", ["cuda_cores", "tcgen05"])
 @pytest.mark.parametrize("nb", [1, 3, 8])
-@pytest.mark.parametrize("rows,K", [(1024, 2048), (4096, 2048), (768, 4096)])
+@pytest.mark.parametrize("rows,K", [(1024, 2048), (4096, 2048), (768, 4096), (1024, 64)])
 def test_engine_matches_float64(engine, nb, rows, K):
     import torch
 

@@ -78,6 +78,13 @@ def test_tiny_ragged_vocab_and_ffn():
     _teacher_forced_case("tiny", vocab=4099, ffn=1000)
 
 
+@pytest.mark.parametrize("kvh", [2, 1])
+def test_tiny_head_dim_128_short_context(kvh):
+    # 128-dim heads over a one-page context: each SM takes one query head of a KV
+    # group (two threads per output dim pair of a run of positions in P.V)
+    _teacher_forced_case("tiny", head_dim=128, n_kv_heads=kvh)
+
+
 def test_tiny_batch_of_three_lanes():
     cfg = configs.model_config("tiny", max_batch=3, max_seq=64)
     w = H.gpu_weights(cfg)
