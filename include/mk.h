@@ -133,9 +133,8 @@ typedef struct {
                                 tcgen05 tensor cores (128-row blocks, accumulators in tensor
                                 memory) where the shape allows it (the Llama-3.2-1B-shaped
                                 kernel): 0 (default) the choice measured faster -- the LM head
-                                on tcgen05, gate/up on CUDA cores --, 1 none (CUDA cores
-                                everywhere), 2 the LM head, 3 gate/up, 4 both; other values:
-                                MK_ERR_INVALID_ARG */
+                                and gate/up on tcgen05 --, 1 none (CUDA cores everywhere), 2 the
+                                LM head, 3 gate/up, 4 both; other values: MK_ERR_INVALID_ARG */
 } mk_options;
 
 /* Create a handle: validates the config, lowers it into per-SM instruction

@@ -161,10 +161,10 @@ bool tc_units(const Dims& D) {
 
 // Tensor-core units of the 8-lane kernel by default (mk_options.tensor_core_units 0):
 // the engine each op measured faster on with 8 lanes (bit 0 LM head, bit 1 gate/up).
-// Llama-3.2-1B shape, batch 8, one box: CUDA cores 1505.9 us/step, LM head on tcgen05
-// 1467.9, gate/up on tcgen05 1714.2, both 1669.7 -- the LM head's long stream gains,
-// gate/up (one 32-page block per SM, 20 SMs without one) loses.
-constexpr int kTcDefault = 1;
+// Llama-3.2-1B shape, batch 8, one box: CUDA cores 1504.3 us/step, LM head on tcgen05
+// 1441.3, gate/up 1463.7, both 1387.6 (eight accumulators per unit, and the gate/up
+// blocks kept out of the scheduler's cumulative balance).
+constexpr int kTcDefault = 3;
 
 std::string dims_from_config(const mk_config* c, int n_sm, Dims* D, int tc_sel = 0) {
   if (!(c->rms_eps >= 0.f) || !std::isfinite(c->rms_eps)) return "rms_eps must be finite and >= 0";

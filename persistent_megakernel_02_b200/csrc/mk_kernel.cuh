@@ -1200,16 +1200,16 @@ __device__ __forceinline__ void mv_units(const KParams& p, const Instr& I, uint3
 // 1/rms and run the epilogue: for
 // gate/up, whose block rows alternate gate and up rows of the same ffn index, the
 // two values meet by one shuffle and the even lane writes silu(g) * u; for the LM
-// head, logits and the running argmax.  tc_n / tc_q count the units and pages of
-// every tensor-core instruction so far in this launch (tc_n gives the accumulator
-// barriers' parities).  Measured faster than the CUDA cores with 8 lanes, where the CUDA-core
+// head, logits and the running argmax.  tc_n counts the units of every
+// tensor-core instruction so far in this launch (the accumulator barriers'
+// parities).  Measured faster than the CUDA cores with 8 lanes, where the CUDA-core
 // matvec reads 32 bytes of activations from shared memory per 16 bytes of weights.
 constexpr int kTcAcc = 8;                      // 16-column accumulators per buffer
 constexpr uint32_t kTcCols = 2 * kTcAcc * 16;  // tensor-memory columns: two buffers
 template <int OPK>
 static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I, uint32_t page_base, uint8_t* ring,
                                                 const float* act, uint64_t* full, uint64_t* empty, Misc* misc,
-                                                uint32_t ii, uint32_t& tc_n, uint32_t& tc_q) {
+                                                uint32_t ii, uint32_t& tc_n) {
   constexpr int NBT = 8;
   static_assert(OPK == OP_GU_TC || OPK == OP_LM_TC, "tensor-core op");
   const Dims& D = p.D;
@@ -1269,7 +1269,6 @@ static __device__ __noinline__ void mv_units_tc(const KParams& p, const Instr& I
           // commit, when every MMA issued so far has completed
           mbar_arrive_cnt(&empty[rp.slot], (uint32_t)kConsumerWarps - 1u);
           umma_commit(&empty[rp.slot]);
-          ++tc_q;
         }
         umma_commit(&misc->tc_accf[buf]);  // the unit's accumulator is complete
       }
@@ -1896,7 +1895,7 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
   // tensor-core units: the 8-lane kernel of the Llama-3.2-1B shape family holds two
   // accumulator buffers (kTcCols fp32 columns) in tensor memory for the whole launch
   constexpr bool kTC = NBT == 8 && SPEC == 1;
-  uint32_t tc_n = 0, tc_q = 0;
+  uint32_t tc_n = 0;
   if constexpr (kTC) {
     if (ct < 32) tmem_alloc(&misc->tmem_base, kTcCols);
     tc_fence_before();
@@ -2032,7 +2031,7 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
           stage<NBT, ST_ONE, true, true>(p, act, misc, lay + p.off_x1, D.H, D.H,
                                          static_cast<const uint16_t*>(I.ptr[3]), ii);
           if (rec) rec[11] = (long long)globaltimer_ns();
-          mv_units_tc<OP_GU_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n, tc_q);
+          mv_units_tc<OP_GU_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n);
           used = I.n_units * (uint32_t)D.nkt;
         }
         break;
@@ -2041,7 +2040,7 @@ static __device__ __noinline__ void consumer(const KParams& p, uint8_t* ring, fl
           stage<NBT, ST_ACC, true, true>(p, act, misc, reinterpret_cast<const float*>(acc_of(p, misc, D.L - 1)),
                                          D.H, D.H, static_cast<const uint16_t*>(I.ptr[3]), ii);
           if (rec) rec[11] = (long long)globaltimer_ns();
-          mv_units_tc<OP_LM_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n, tc_q);
+          mv_units_tc<OP_LM_TC>(p, I, page_base, ring, act, full, empty, misc, ii, tc_n);
           used = I.n_units * (uint32_t)D.nkt;
         }
         break;

@@ -192,7 +192,13 @@ Tape lower(const Dims& D, int n_sm, int nb, int dyn_percent, int region) {
     const int n_dyn = pool >= 0 ? (int)((int64_t)n * dyn_percent / 100) : 0;
     const int n_st = n - n_dyn;
     const int64_t ub = unit_bytes(D, op, t.S);
+    // Gate/up tensor-core blocks are 32 pages each and fewer than the SMs: counted
+    // in the cumulative load they would hand the SMs without one extra units of
+    // every later phase, and those SMs would lead the latency-bound phases.  They
+    // take the least-loaded SMs without changing the balance of the rest.
+    const std::vector<int64_t> saved = op == OP_GU_TC ? load : std::vector<int64_t>();
     auto st = as.run(n_st, ub, lo, hi);
+    if (op == OP_GU_TC) load = saved;
     // each SM's expected share of the pool counts toward its load
     if (n_dyn > 0)
       for (int s = lo; s < hi; ++s) load[s] += ub * n_dyn / n_part;
