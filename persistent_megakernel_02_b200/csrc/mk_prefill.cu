@@ -332,8 +332,10 @@ __device__ __forceinline__ float kv_elem(uint4 w, int e) {
   return (e & 1) ? kv_hi<F16>(u) : kv_lo<F16>(u);
 }
 
-// Causal GQA attention of a chunk's queries over the cache.  CTA = (block of
-// 64 / rep tokens, kv head g): its 64 query rows are the rep query heads of g for
+// Causal GQA attention of a chunk's queries over the cache.  CTA = (kv head g,
+// block of 64 / rep tokens, the last block first: blocks read more pages the later
+// their tokens, so the longest go out first and the short ones fill the tail).  Its
+// 64 query rows are the rep query heads of g for
 // each token (row r: head g * rep + r / QB, token t0 + r % QB).  The KV pages of
 // positions 0 .. the block's last position are read in order; per page the
 // scores of every (row, position) pair, the running max / sum / output of an
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kAttnThreads)
   float* Vs = kT + DH * PL;             // [PL][DH]
   float* Ps = Vs + PL * DH;             // [64][PSTR]
   const int QB = kAttnRows / rep;
-  const int g = blockIdx.y, t0 = blockIdx.x * QB;
+  const int g = blockIdx.x, t0 = (gridDim.y - 1 - blockIdx.y) * QB;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   for (int e = tid; e < kAttnRows * DH; e += kAttnThreads) {
     const int r = e / DH, dd = e % DH, t = t0 + r % QB;
@@ -369,13 +371,14 @@ __global__ void __launch_bounds__(kAttnThreads)
     rv[i] = t < T;
     qpos[i] = pos0 + t;
   }
-  float m[4], l[4], o[4][DPT];
+  float m[4], l[4];
+  float2 o[4][DPT / 2];  // output dims in pairs (FFMA2)
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     m[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
-    for (int e = 0; e < DPT; ++e) o[i][e] = 0.f;
+    for (int e = 0; e < DPT / 2; ++e) o[i][e] = make_float2(0.f, 0.f);
   }
   const int last_pos = pos0 + min(T, t0 + QB) - 1;
   const int npages = last_pos / PL + 1;
@@ -397,28 +400,37 @@ __global__ void __launch_bounds__(kAttnThreads)
       for (int j = 0; j < 8; ++j) Vs[pos * DH + c * 8 + j] = kv_elem<KV16F>(w, j);
     }
     __syncthreads();
-    float s[4][KPT];
+    // scores: packed FP32 FMA (FFMA2) over pairs of keys; each element rounds as fmaf
+    float2 s2[4][KPT / 2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < KPT; ++j) s[i][j] = 0.f;
+      for (int j = 0; j < KPT / 2; ++j) s2[i][j] = make_float2(0.f, 0.f);
 #pragma unroll 8
     for (int dd = 0; dd < DH; ++dd) {
       const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kAttnRows + 4 * ty);
-      float kk[KPT];
+      float2 kk[KPT / 2];
       if constexpr (KPT == 4) {
         const float4 k4 = *reinterpret_cast<const float4*>(kT + dd * PL + 4 * tx);
-        kk[0] = k4.x; kk[1] = k4.y; kk[2] = k4.z; kk[3] = k4.w;
+        kk[0] = make_float2(k4.x, k4.y);
+        kk[1] = make_float2(k4.z, k4.w);
       } else {
-        const float2 k2 = *reinterpret_cast<const float2*>(kT + dd * PL + 2 * tx);
-        kk[0] = k2.x; kk[1] = k2.y;
+        kk[0] = *reinterpret_cast<const float2*>(kT + dd * PL + 2 * tx);
       }
       const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < KPT; ++j) s[i][j] = fmaf(qa[i], kk[j], s[i][j]);
+        for (int j = 0; j < KPT / 2; ++j) s2[i][j] = __ffma2_rn(make_float2(qa[i], qa[i]), kk[j], s2[i][j]);
     }
+    float s[4][KPT];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < KPT / 2; ++j) {
+        s[i][2 * j] = s2[i][j].x;
+        s[i][2 * j + 1] = s2[i][j].y;
+      }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       float mx = -INFINITY;
@@ -444,24 +456,36 @@ __global__ void __launch_bounds__(kAttnThreads)
       l[i] = l[i] * corr + ps;
       m[i] = mn;
 #pragma unroll
-      for (int e = 0; e < DPT; ++e) o[i][e] *= corr;
+      for (int e = 0; e < DPT / 2; ++e) {
+        o[i][e].x *= corr;
+        o[i][e].y *= corr;
+      }
     }
     __syncthreads();
-#pragma unroll 4
-    for (int k = 0; k < PL; ++k) {
-      float p[4];
+    // P.V, four keys per step: each row's four probabilities in one 16-byte load
+    static_assert(PL % 4 == 0 && PSTR % 4 == 0, "float4 rows of probabilities");
+#pragma unroll 2
+    for (int k0 = 0; k0 < PL; k0 += 4) {
+      float4 p4[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) p[i] = Ps[(4 * ty + i) * PSTR + k];
-      float v[DPT];
+      for (int i = 0; i < 4; ++i) p4[i] = *reinterpret_cast<const float4*>(Ps + (4 * ty + i) * PSTR + k0);
 #pragma unroll
-      for (int e = 0; e < DPT; e += 4) {
-        const float4 v4 = *reinterpret_cast<const float4*>(Vs + k * DH + tx * DPT + e);
-        v[e] = v4.x; v[e + 1] = v4.y; v[e + 2] = v4.z; v[e + 3] = v4.w;
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = k0 + kk;
+        float2 v[DPT / 2];
+#pragma unroll
+        for (int e = 0; e < DPT / 2; e += 2) {
+          const float4 v4 = *reinterpret_cast<const float4*>(Vs + k * DH + tx * DPT + 2 * e);
+          v[e] = make_float2(v4.x, v4.y);
+          v[e + 1] = make_float2(v4.z, v4.w);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float pk = kk == 0 ? p4[i].x : kk == 1 ? p4[i].y : kk == 2 ? p4[i].z : p4[i].w;
+#pragma unroll
+          for (int e = 0; e < DPT / 2; ++e) o[i][e] = __ffma2_rn(make_float2(pk, pk), v[e], o[i][e]);
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < DPT; ++e) o[i][e] = fmaf(p[i], v[e], o[i][e]);
     }
   }
 #pragma unroll
@@ -472,7 +496,10 @@ __global__ void __launch_bounds__(kAttnThreads)
     const size_t base = (size_t)t * qdim + (size_t)(g * rep + r / QB) * DH + tx * DPT;
     uint16_t h[DPT], lo[DPT];
 #pragma unroll
-    for (int e = 0; e < DPT; ++e) split_bf16(o[i][e] * inv, h[e], lo[e]);
+    for (int e = 0; e < DPT / 2; ++e) {
+      split_bf16(o[i][e].x * inv, h[2 * e], lo[2 * e]);
+      split_bf16(o[i][e].y * inv, h[2 * e + 1], lo[2 * e + 1]);
+    }
 #pragma unroll
     for (int e = 0; e < DPT; e += 4) {
       *reinterpret_cast<uint2*>(Ohi + base + e) = *reinterpret_cast<const uint2*>(h + e);
@@ -635,7 +662,7 @@ mk_status prefill_run(PrefillPlan* p, const PrefillCtx& c, const int* tokens_dev
       pf_gemm<EPI_QKV><<<dim3(mt, q.nq + 2 * q.nk), kGThreads, kGSmem, st>>>(nhi, nlo, p->wq[l], p->wk[l],
                                                                              p->wv[l], q);
       if (l == D.L - 1) break;  // only the last layer's K and V are read later
-      const dim3 ag((T + kAttnRows / D.rep - 1) / (kAttnRows / D.rep), D.Hkv);
+      const dim3 ag(D.Hkv, (T + kAttnRows / D.rep - 1) / (kAttnRows / D.rep));
       if (D.d == 64) {
         if (D.kv_fp16)
           pf_attn<64, true><<<ag, kAttnThreads, attn_smem<64>(), st>>>(p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages,

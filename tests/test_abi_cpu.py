@@ -226,6 +226,18 @@ def test_plan_check_rejects_an_unknown_region():
     assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 0, 5, ctypes.byref(rep)) == 1
 
 
+def test_gate_up_blocks_stay_out_of_the_cumulative_balance():
+    """The 128 gate/up tensor-core blocks (32 pages each, fewer than the SMs) must not
+    tilt the other phases: the SMs that hold one carry its 32 pages on top of an even
+    share of everything else, so the step's per-SM bytes spread by at least a block."""
+    cfg = configs.model_config("llama1b_bs8")
+    page = 16384
+    cuda_cores = mk.plan_check(cfg, 148, 8, tensor_core_units=1)
+    gu = mk.plan_check(cfg, 148, 8, tensor_core_units=3)
+    assert cuda_cores["bytes_max_sm"] - cuda_cores["bytes_min_sm"] <= 2 * page
+    assert gu["bytes_max_sm"] - gu["bytes_min_sm"] >= 32 * page
+
+
 @pytest.mark.parametrize("units", [2, 3, 4])
 @pytest.mark.parametrize("region", [0, 1, 2])
 def test_tensor_core_unit_tapes_cover_their_blocks(units, region):
