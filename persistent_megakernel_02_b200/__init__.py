@@ -320,21 +320,29 @@ class Megakernel:
 
     def decode_step_host(self, tokens, positions, want_logits=False, stream=None):
         """Step over host buffers; returns (ids list, logits numpy [nb, V] or None)."""
-        import numpy as np
-
         nb = len(positions)
         if len(tokens) != nb or not 1 <= nb <= 8:
             raise MkError(1, "mk_decode_step_host: one token and one position per lane, 1..8 lanes")
-        if self._host_io is None:  # argument buffers reused by every call
-            self._host_io = tuple((ctypes.c_int32 * 8)() for _ in range(3))
-        tk, ps, ids = self._host_io
-        for i in range(nb):
-            tk[i] = tokens[i]
-            ps[i] = positions[i]
-        lg = np.empty((nb, self.cfg["vocab"]), dtype=np.float32) if want_logits else None
-        _check(lib().mk_decode_step_host(
-            self._h, nb, tk, ps, None if lg is None else lg.ctypes.data_as(ctypes.c_void_p), ids,
-            _stream_handle(stream)), "mk_decode_step_host")
+        io = self._host_io
+        if io is None:  # argument buffers reused by every call
+            io = self._host_io = tuple((ctypes.c_int32 * 8)() for _ in range(3))
+        tk, ps, ids = io
+        try:
+            tk[:nb] = tokens
+            ps[:nb] = positions
+        except TypeError:  # e.g. tensors: element by element
+            for i in range(nb):
+                tk[i] = int(tokens[i])
+                ps[i] = int(positions[i])
+        lg = None
+        if want_logits:
+            import numpy as np
+
+            lg = np.empty((nb, self.cfg["vocab"]), dtype=np.float32)
+        st = lib().mk_decode_step_host(self._h, nb, tk, ps, None if lg is None else lg.ctypes.data_as(ctypes.c_void_p),
+                                       ids, None if stream is None else _stream_handle(stream))
+        if st:
+            raise MkError(st, "mk_decode_step_host")
         return ids[:nb], lg
 
     def prefill(self, seq, tokens, start_pos=0, logits_last=None, want_id=True, stream=None):
