@@ -123,6 +123,33 @@ def test_tiny_long_context_split_attention(lens):
             H.compare_ids(ids[t, b], w_steps[t])
 
 
+@pytest.mark.parametrize("lens", [[600], [700, 300]])
+def test_tiny_head_dim_128_merges_many_slices(lens):
+    """128-dim heads over contexts of 19-22 KV pages: a (lane, kv head) runs as 9 or more
+    slices, and the last one merges them through shared-memory weights; a lane with 10
+    pages (5 slices) merges by the per-thread walk in the same step."""
+    nb = len(lens)
+    cfg = configs.model_config("tiny", max_batch=nb, max_seq=max(lens) + 8, head_dim=128)
+    w = H.gpu_weights(cfg)
+    prompts = [synth.prompt_tokens(cfg, b, n).numpy() for b, n in enumerate(lens)]
+    teacher = [synth.teacher_tokens(cfg, b, 6).numpy() for b in range(nb)]
+    mk = _mk(cfg, w)
+    pre, lg, ids = H.run_teacher_forced(mk, cfg, prompts, teacher, 6)
+    mk.close()
+    orc = H.oracle_for(cfg, w)
+    worst = (0.0, 0.0)
+    checked = 0
+    for b in range(nb):
+        w_pre, w_steps = H.oracle_teacher_forced(orc, prompts[b], teacher[b], 6)
+        e = H.compare_logits(pre[b], w_pre, f"lane {b} prefill")
+        worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+        for t in range(6):
+            e = H.compare_logits(lg[t, b], w_steps[t], f"lane {b} step {t}")
+            worst = (max(worst[0], e[0]), max(worst[1], e[1]))
+            checked += H.compare_ids(ids[t, b], w_steps[t])
+    H.record(f"tiny[head_dim=128] contexts {lens} x{nb} lanes", worst, 6, checked)
+
+
 def test_tiny_free_run_greedy_chained_on_device():
     wlc = configs.WORKLOADS["tiny"]
     cfg = configs.model_config("tiny")
