@@ -53,7 +53,12 @@ constexpr int kGSmem = 1024 + kGStages * kGStageBytes + 256;
 constexpr uint32_t kGIdesc = idesc_bf16(kGM, kGN);
 constexpr uint32_t kGTmemCols = kGN;
 constexpr int kAttnThreads = 256;
-constexpr int kAttnRows = 64;                 // query rows (tokens x query heads of one kv head) per CTA
+// query rows (tokens x query heads of one kv head) per CTA: 64, or 128 with 64-dim heads when
+// the chunk gives every SM three such CTAs (8 rows per thread: a larger register tile and
+// half the K/V page loads per query; 8192-token prompt in 2048-token chunks 158.7 -> 146.0
+// ms, while 512-1408-token prompts, too short to fill the SMs with 128-row CTAs, lost 1-3 %)
+constexpr int kAttnRowsMin = 64;
+constexpr int kAttnRowsWide = 128;
 
 // error word of the handle: [0] code, [4] abort flag (the decode kernel's layout)
 constexpr uint32_t kErrPrefillWait = 7;
@@ -342,7 +347,7 @@ __device__ __forceinline__ float kv_elem(uint4 w, int e) {
 // online softmax per row, and the key mask pos_key <= pos_query.  Thread (ty, tx)
 // owns rows 4 ty .. 4 ty + 3 and keys tx * KPT .. (scores) or output dims
 // tx * DPT .. (P V).  Output: o / l as bf16 high and low parts [T][qdim].
-template <int DH, bool KV16F>
+template <int DH, bool KV16F, int ROWS>
 __global__ void __launch_bounds__(kAttnThreads)
     pf_attn(const float* __restrict__ Q, int T, int qdim, const uint16_t* __restrict__ kv, const int* __restrict__ pt,
             int layer, int n_phys_pages, int Hkv, int rep, int pos0, uint16_t* __restrict__ Ohi,
@@ -351,30 +356,31 @@ __global__ void __launch_bounds__(kAttnThreads)
   constexpr int KPT = PL / 16;          // keys per thread
   constexpr int DPT = DH / 16;          // output dims per thread
   constexpr int PSTR = PL + 4;          // padded row of the probabilities
+  constexpr int RPT = ROWS / 16;        // query rows per thread
   extern __shared__ float sm[];
-  float* qT = sm;                       // [DH][64]
-  float* kT = qT + DH * kAttnRows;      // [DH][PL]
+  float* qT = sm;                       // [DH][ROWS]
+  float* kT = qT + DH * ROWS;           // [DH][PL]
   float* Vs = kT + DH * PL;             // [PL][DH]
-  float* Ps = Vs + PL * DH;             // [64][PSTR]
-  const int QB = kAttnRows / rep;
+  float* Ps = Vs + PL * DH;             // [ROWS][PSTR]
+  const int QB = ROWS / rep;
   const int g = blockIdx.x, t0 = (gridDim.y - 1 - blockIdx.y) * QB;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  for (int e = tid; e < kAttnRows * DH; e += kAttnThreads) {
+  for (int e = tid; e < ROWS * DH; e += kAttnThreads) {
     const int r = e / DH, dd = e % DH, t = t0 + r % QB;
-    qT[dd * kAttnRows + r] = t < T ? Q[(size_t)t * qdim + (size_t)(g * rep + r / QB) * DH + dd] : 0.f;
+    qT[dd * ROWS + r] = t < T ? Q[(size_t)t * qdim + (size_t)(g * rep + r / QB) * DH + dd] : 0.f;
   }
-  int qpos[4];
-  bool rv[4];
+  int qpos[RPT];
+  bool rv[RPT];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int r = 4 * ty + i, t = t0 + r % QB;
+  for (int i = 0; i < RPT; ++i) {
+    const int r = RPT * ty + i, t = t0 + r % QB;
     rv[i] = t < T;
     qpos[i] = pos0 + t;
   }
-  float m[4], l[4];
-  float2 o[4][DPT / 2];  // output dims in pairs (FFMA2)
+  float m[RPT], l[RPT];
+  float2 o[RPT][DPT / 2];  // output dims in pairs (FFMA2)
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < RPT; ++i) {
     m[i] = -INFINITY;
     l[i] = 0.f;
 #pragma unroll
@@ -401,14 +407,19 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
     __syncthreads();
     // scores: packed FP32 FMA (FFMA2) over pairs of keys; each element rounds as fmaf
-    float2 s2[4][KPT / 2];
+    float2 s2[RPT][KPT / 2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
       for (int j = 0; j < KPT / 2; ++j) s2[i][j] = make_float2(0.f, 0.f);
 #pragma unroll 8
     for (int dd = 0; dd < DH; ++dd) {
-      const float4 qv = *reinterpret_cast<const float4*>(qT + dd * kAttnRows + 4 * ty);
+      float qa[RPT];
+#pragma unroll
+      for (int i = 0; i < RPT; i += 4) {
+        const float4 qv = *reinterpret_cast<const float4*>(qT + dd * ROWS + RPT * ty + i);
+        qa[i] = qv.x; qa[i + 1] = qv.y; qa[i + 2] = qv.z; qa[i + 3] = qv.w;
+      }
       float2 kk[KPT / 2];
       if constexpr (KPT == 4) {
         const float4 k4 = *reinterpret_cast<const float4*>(kT + dd * PL + 4 * tx);
@@ -417,22 +428,21 @@ __global__ void __launch_bounds__(kAttnThreads)
       } else {
         kk[0] = *reinterpret_cast<const float2*>(kT + dd * PL + 2 * tx);
       }
-      const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < RPT; ++i)
 #pragma unroll
         for (int j = 0; j < KPT / 2; ++j) s2[i][j] = __ffma2_rn(make_float2(qa[i], qa[i]), kk[j], s2[i][j]);
     }
-    float s[4][KPT];
+    float s[RPT][KPT];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < RPT; ++i)
 #pragma unroll
       for (int j = 0; j < KPT / 2; ++j) {
         s[i][2 * j] = s2[i][j].x;
         s[i][2 * j + 1] = s2[i][j].y;
       }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < RPT; ++i) {
       float mx = -INFINITY;
 #pragma unroll
       for (int j = 0; j < KPT; ++j) {
@@ -448,7 +458,7 @@ __global__ void __launch_bounds__(kAttnThreads)
 #pragma unroll
       for (int j = 0; j < KPT; ++j) {
         const float p = mn == -INFINITY ? 0.f : __expf(s[i][j] - mn);
-        Ps[(4 * ty + i) * PSTR + tx * KPT + j] = p;
+        Ps[(RPT * ty + i) * PSTR + tx * KPT + j] = p;
         ps += p;
       }
 #pragma unroll
@@ -466,9 +476,9 @@ __global__ void __launch_bounds__(kAttnThreads)
     static_assert(PL % 4 == 0 && PSTR % 4 == 0, "float4 rows of probabilities");
 #pragma unroll 2
     for (int k0 = 0; k0 < PL; k0 += 4) {
-      float4 p4[4];
+      float4 p4[RPT];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) p4[i] = *reinterpret_cast<const float4*>(Ps + (4 * ty + i) * PSTR + k0);
+      for (int i = 0; i < RPT; ++i) p4[i] = *reinterpret_cast<const float4*>(Ps + (RPT * ty + i) * PSTR + k0);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const int k = k0 + kk;
@@ -480,7 +490,7 @@ __global__ void __launch_bounds__(kAttnThreads)
           v[e + 1] = make_float2(v4.z, v4.w);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < RPT; ++i) {
           const float pk = kk == 0 ? p4[i].x : kk == 1 ? p4[i].y : kk == 2 ? p4[i].z : p4[i].w;
 #pragma unroll
           for (int e = 0; e < DPT / 2; ++e) o[i][e] = __ffma2_rn(make_float2(pk, pk), v[e], o[i][e]);
@@ -489,9 +499,9 @@ __global__ void __launch_bounds__(kAttnThreads)
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < RPT; ++i) {
     if (!rv[i]) continue;
-    const int r = 4 * ty + i, t = t0 + r % QB;
+    const int r = RPT * ty + i, t = t0 + r % QB;
     const float inv = 1.0f / l[i];
     const size_t base = (size_t)t * qdim + (size_t)(g * rep + r / QB) * DH + tx * DPT;
     uint16_t h[DPT], lo[DPT];
@@ -508,9 +518,9 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 }
 
-template <int DH>
+template <int DH, int ROWS>
 constexpr int attn_smem() {
-  return (DH * kAttnRows + DH * (16384 / (4 * DH)) * 2 + kAttnRows * (16384 / (4 * DH) + 4)) * 4;
+  return (DH * ROWS + DH * (16384 / (4 * DH)) * 2 + ROWS * (16384 / (4 * DH) + 4)) * 4;
 }
 
 using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -537,6 +547,7 @@ bool encode(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uin
 struct PrefillPlan {
   Dims D{};
   int chunk = 0;
+  int n_sm = 148;  // SMs of the device (the attention's tile choice)
   const uint16_t* embed = nullptr;
   std::vector<const uint16_t*> attn_norm, mlp_norm;
   std::vector<CUtensorMap> wq, wk, wv, wo, wg, wu, wd;
@@ -548,7 +559,7 @@ struct PrefillPlan {
 
 bool prefill_supported(const Dims& D) {
   return D.H % kGN == 0 && D.qdim % kGN == 0 && D.kvdim % kGN == 0 && D.F % (kGN / 2) == 0 &&
-         (D.d == 64 || D.d == 128) && kAttnRows % D.rep == 0;
+         (D.d == 64 || D.d == 128) && kAttnRowsMin % D.rep == 0;
 }
 
 void prefill_destroy(PrefillPlan* p) {
@@ -560,6 +571,10 @@ void prefill_destroy(PrefillPlan* p) {
 mk_status prefill_create(const Dims& D, const mk_weights* w, int chunk, PrefillPlan** out) {
   *out = nullptr;
   if (!prefill_supported(D) || chunk < 1) return MK_ERR_UNSUPPORTED;
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
+    return MK_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lock(g_pf_mutex);
     if (!g_pf_encode) {
@@ -572,6 +587,7 @@ mk_status prefill_create(const Dims& D, const mk_weights* w, int chunk, PrefillP
     }
   }
   PrefillPlan* p = new PrefillPlan();
+  p->n_sm = n_sm;
   p->D = D;
   p->chunk = chunk;
   p->embed = static_cast<const uint16_t*>(w->embed);
@@ -607,14 +623,18 @@ mk_status prefill_create(const Dims& D, const mk_weights* w, int chunk, PrefillP
     ok &= cudaFuncSetAttribute(pf_gemm<EPI_RESID>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pf_gemm<EPI_SWIGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGSmem) ==
           cudaSuccess;
-    ok &= cudaFuncSetAttribute(pf_attn<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<64>()) ==
-          cudaSuccess;
-    ok &= cudaFuncSetAttribute(pf_attn<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<64>()) ==
-          cudaSuccess;
-    ok &= cudaFuncSetAttribute(pf_attn<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<128>()) ==
-          cudaSuccess;
-    ok &= cudaFuncSetAttribute(pf_attn<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem<128>()) ==
-          cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<64, false, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<64, kAttnRowsMin>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<64, true, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<64, kAttnRowsMin>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<64, false, kAttnRowsWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<64, kAttnRowsWide>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<64, true, kAttnRowsWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<64, kAttnRowsWide>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<128, false, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<128, kAttnRowsMin>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn<128, true, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               attn_smem<128, kAttnRowsMin>()) == cudaSuccess;
   }
   if (!ok) {
     prefill_destroy(p);
@@ -662,24 +682,27 @@ mk_status prefill_run(PrefillPlan* p, const PrefillCtx& c, const int* tokens_dev
       pf_gemm<EPI_QKV><<<dim3(mt, q.nq + 2 * q.nk), kGThreads, kGSmem, st>>>(nhi, nlo, p->wq[l], p->wk[l],
                                                                              p->wv[l], q);
       if (l == D.L - 1) break;  // only the last layer's K and V are read later
-      const dim3 ag(D.Hkv, (T + kAttnRows / D.rep - 1) / (kAttnRows / D.rep));
+      // 128-row CTAs where the chunk gives every SM three of them (64-dim heads)
+      const bool wide = D.d == 64 && (long long)((T + kAttnRowsWide / D.rep - 1) / (kAttnRowsWide / D.rep)) * D.Hkv >=
+                                         3LL * p->n_sm;
+      const int qb = (wide ? kAttnRowsWide : kAttnRowsMin) / D.rep;  // tokens per CTA
+      const dim3 ag(D.Hkv, (T + qb - 1) / qb);
+#define MK_PF_ATTN(DH_, F16_, ROWS_)                                                                      \
+  pf_attn<DH_, F16_, ROWS_><<<ag, kAttnThreads, attn_smem<DH_, ROWS_>(), st>>>(                           \
+      p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages, D.Hkv, D.rep, pos, p->Ohi, p->Olo)
       if (D.d == 64) {
-        if (D.kv_fp16)
-          pf_attn<64, true><<<ag, kAttnThreads, attn_smem<64>(), st>>>(p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages,
-                                                                      D.Hkv, D.rep, pos, p->Ohi, p->Olo);
-        else
-          pf_attn<64, false><<<ag, kAttnThreads, attn_smem<64>(), st>>>(p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages,
-                                                                       D.Hkv, D.rep, pos, p->Ohi, p->Olo);
+        if (wide) {
+          if (D.kv_fp16) MK_PF_ATTN(64, true, kAttnRowsWide);
+          else MK_PF_ATTN(64, false, kAttnRowsWide);
+        } else {
+          if (D.kv_fp16) MK_PF_ATTN(64, true, kAttnRowsMin);
+          else MK_PF_ATTN(64, false, kAttnRowsMin);
+        }
       } else {
-        if (D.kv_fp16)
-          pf_attn<128, true><<<ag, kAttnThreads, attn_smem<128>(), st>>>(p->Q, T, D.qdim, c.kv, pt, l,
-                                                                        D.n_phys_pages, D.Hkv, D.rep, pos, p->Ohi,
-                                                                        p->Olo);
-        else
-          pf_attn<128, false><<<ag, kAttnThreads, attn_smem<128>(), st>>>(p->Q, T, D.qdim, c.kv, pt, l,
-                                                                         D.n_phys_pages, D.Hkv, D.rep, pos, p->Ohi,
-                                                                         p->Olo);
+        if (D.kv_fp16) MK_PF_ATTN(128, true, kAttnRowsMin);
+        else MK_PF_ATTN(128, false, kAttnRowsMin);
       }
+#undef MK_PF_ATTN
       GemmArgs r = g;
       r.K = D.qdim;
       r.X = p->X;
