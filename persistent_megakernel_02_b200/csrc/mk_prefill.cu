@@ -518,6 +518,216 @@ __global__ void __launch_bounds__(kAttnThreads)
   }
 }
 
+// Causal GQA attention of a chunk's queries on the tensor cores (64-dim heads, bf16
+// cache).  CTA = (kv head g, block of 128 / rep tokens, the last block first): its 128
+// query rows are the rep query heads of g for each token (row r: head g * rep + r / QB,
+// token t0 + r % QB), one row per tensor-memory lane.  Per KV page (64 positions):
+//   - all threads stage K as the B operand of S (64 key rows of 64 dims, 128-byte
+//     swizzle) and V transposed as the B operand of P.V (64 dim rows of 64 keys);
+//   - thread 0 issues S = Q_hi K^T + Q_lo K^T (M = 128, N = 64, K = 64: 8 MMAs) into
+//     tensor-memory columns 0..63 and commits;
+//   - warps 0-3, one query row per thread, read S back, apply the scale and the causal
+//     mask, update the row's online softmax (max m, sum l), rescale the row's output
+//     (kept in registers) and write P as bf16 high and low parts (the A operand);
+//   - thread 0 issues P.V = P_hi V + P_lo V into columns 64..127 and commits, and warps
+//     0-3 add it to their rows' outputs.
+// Q and P are split into bf16 high and low parts, so the products keep fp32-level
+// accuracy; K and V are the cache's bf16 values.  Output: o / l as bf16 high and low
+// parts [T][qdim].  Every wait is bounded (pf_wait); tensor memory is freed on every
+// exit path.
+constexpr int kTcAttnRows = 128;
+constexpr int kTcAttnThreads = 256;
+constexpr int kTcAttnCols = 128;  // S in columns 0..63, P.V in 64..127
+constexpr uint32_t kTcAttnIdesc = idesc_bf16(128, 64);
+constexpr int kTcAttnSmem = 1024 + 2 * 16384 + 8192 + 8192 + 2 * 16384 + 64;
+
+// byte offset of element (row, col) in a tile of 128-byte rows (64 bf16), 128-byte swizzle
+__device__ __forceinline__ uint32_t sw128_off(int row, int col) {
+  return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2);
+}
+
+__global__ void __launch_bounds__(kTcAttnThreads, 1)
+    pf_attn_tc(const float* __restrict__ Q, int T, int qdim, const uint16_t* __restrict__ kv,
+               const int* __restrict__ pt, int layer, int n_phys_pages, int Hkv, int rep, int pos0,
+               uint16_t* __restrict__ Ohi, uint16_t* __restrict__ Olo, uint32_t* err, unsigned long long limit_ns) {
+  constexpr int DH = 64, PL = 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* qhi = smem;                // [128][64] bf16, swizzled
+  uint8_t* qlo = qhi + 16384;
+  uint8_t* kt = qlo + 16384;          // [64 keys][64 dims]
+  uint8_t* vt = kt + 8192;            // [64 dims][64 keys]
+  uint8_t* phi = vt + 8192;           // [128][64 keys]
+  uint8_t* plo = phi + 16384;
+  uint64_t* sdone = reinterpret_cast<uint64_t*>(plo + 16384);
+  uint64_t* pvdone = sdone + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(pvdone + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int QB = kTcAttnRows / rep;
+  const int g = blockIdx.x, t0 = (gridDim.y - 1 - blockIdx.y) * QB;
+
+  if (tid == 0) {
+    mbar_init(sdone, 1);
+    mbar_init(pvdone, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, kTcAttnCols);
+  // queries, scaled by 1/sqrt(d), as bf16 high and low parts (the A operand of S)
+  const float scale = 1.0f / sqrtf((float)DH);
+  for (int e = tid; e < kTcAttnRows * (DH / 8); e += kTcAttnThreads) {
+    const int r = e / (DH / 8), c = e % (DH / 8), t = t0 + r % QB;
+    uint16_t h8[8], l8[8];
+    if (t < T) {
+      const float* src = Q + (size_t)t * qdim + (size_t)(g * rep + r / QB) * DH + c * 8;
+      const float4 a = *reinterpret_cast<const float4*>(src), b = *reinterpret_cast<const float4*>(src + 4);
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) split_bf16(v[j] * scale, h8[j], l8[j]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) h8[j] = l8[j] = 0;
+    }
+    *reinterpret_cast<uint4*>(qhi + sw128_off(r, c * 8)) = *reinterpret_cast<const uint4*>(h8);
+    *reinterpret_cast<uint4*>(qlo + sw128_off(r, c * 8)) = *reinterpret_cast<const uint4*>(l8);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  // this thread's query row (warps 0-3: tensor-memory lane = row)
+  const int row = tid;                 // meaningful for tid < 128
+  const int qt = t0 + row % QB;
+  const bool rv = tid < kTcAttnRows && qt < T;
+  const int qpos = pos0 + qt;
+  float m = -INFINITY, l = 0.f, o[DH];
+#pragma unroll
+  for (int d = 0; d < DH; ++d) o[d] = 0.f;
+  const int last_pos = pos0 + min(T, t0 + QB) - 1;
+  const int npages = last_pos / PL + 1;
+  const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  bool ok = true;
+  for (int pg = 0; pg < npages; ++pg) {
+    // K as is (key rows), V transposed (dim rows), both swizzled
+    const uint16_t* kp = kv + (((size_t)layer * n_phys_pages + pt[pg]) * Hkv + g) * (size_t)(2 * PL * DH);
+    const uint16_t* vp = kp + PL * DH;
+    for (int e = tid; e < PL * (DH / 8); e += kTcAttnThreads) {
+      const int r = e / (DH / 8), c = e % (DH / 8);
+      const uint4 w = ldnc16(kp + (size_t)r * DH + c * 8);
+      *reinterpret_cast<uint4*>(kt + sw128_off(r, c * 8)) = w;
+      const uint4 v = ldnc16(vp + (size_t)r * DH + c * 8);
+      const uint16_t* v16 = reinterpret_cast<const uint16_t*>(&v);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) *reinterpret_cast<uint16_t*>(vt + sw128_off(c * 8 + j, r)) = v16[j];
+    }
+    fence_proxy_async_smem();  // the tensor cores read the tiles through the async proxy
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0 && ok) {
+      const uint32_t a0 = smem_u32(qhi), a1 = smem_u32(qlo), b = smem_u32(kt);
+#pragma unroll
+      for (int j = 0; j < DH / 16; ++j) {
+        umma_f16(tmem, sw128_desc(a0 + 32 * j), sw128_desc(b + 32 * j), kTcAttnIdesc, j ? 1u : 0u);
+        umma_f16(tmem, sw128_desc(a1 + 32 * j), sw128_desc(b + 32 * j), kTcAttnIdesc, 1u);
+      }
+      umma_commit(sdone);
+    }
+    if (warp < 4) {
+      ok = __all_sync(0xFFFFFFFFu, ok && pf_wait(sdone, pg & 1, err, limit_ns, 11));
+      tc_fence_after();
+      float sv[PL];
+      if (ok) {
+#pragma unroll
+        for (int c0 = 0; c0 < PL; c0 += 32) {
+          uint32_t r32[32];
+          tmem_ld32(tl + (uint32_t)c0, r32);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sv[c0 + j] = __uint_as_float(r32[j]);
+        }
+      }
+      // online softmax of this row over the page's positions (key pos <= query pos)
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < PL; ++c) {
+        const int kpos = pg * PL + c;
+        sv[c] = (rv && kpos <= qpos) ? sv[c] : -INFINITY;
+        mx = fmaxf(mx, sv[c]);
+      }
+      const float mn = fmaxf(m, mx);
+      const float corr = mn == -INFINITY ? 1.f : __expf(m - mn);
+      float ps = 0.f;
+#pragma unroll
+      for (int c0 = 0; c0 < PL; c0 += 8) {
+        uint16_t h8[8], l8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float pv = mn == -INFINITY ? 0.f : __expf(sv[c0 + j] - mn);
+          ps += pv;
+          split_bf16(pv, h8[j], l8[j]);
+        }
+        *reinterpret_cast<uint4*>(phi + sw128_off(row, c0)) = *reinterpret_cast<const uint4*>(h8);
+        *reinterpret_cast<uint4*>(plo + sw128_off(row, c0)) = *reinterpret_cast<const uint4*>(l8);
+      }
+      l = l * corr + ps;
+      m = mn;
+#pragma unroll
+      for (int d = 0; d < DH; ++d) o[d] *= corr;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 0-3: every row's P is written
+      tc_fence_after();
+      if (tid == 0 && ok) {
+        const uint32_t a0 = smem_u32(phi), a1 = smem_u32(plo), b = smem_u32(vt);
+#pragma unroll
+        for (int j = 0; j < PL / 16; ++j) {
+          umma_f16(tmem + 64u, sw128_desc(a0 + 32 * j), sw128_desc(b + 32 * j), kTcAttnIdesc, j ? 1u : 0u);
+          umma_f16(tmem + 64u, sw128_desc(a1 + 32 * j), sw128_desc(b + 32 * j), kTcAttnIdesc, 1u);
+        }
+        umma_commit(pvdone);
+      }
+      ok = __all_sync(0xFFFFFFFFu, ok && pf_wait(pvdone, pg & 1, err, limit_ns, 12));
+      tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          uint32_t r32[32];
+          tmem_ld32(tl + 64u + (uint32_t)c0, r32);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) o[c0 + j] += __uint_as_float(r32[j]);
+        }
+      }
+    }
+    // the tiles are free once P.V has read them (warps 0-3 saw it complete)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    ok = __syncthreads_and(ok ? 1 : 0) != 0;
+    if (!ok) break;
+  }
+  if (rv && ok) {
+    const int t = qt, h = g * rep + row / QB;
+    const float inv = 1.0f / l;
+    uint16_t* dh = Ohi + (size_t)t * qdim + (size_t)h * DH;
+    uint16_t* dl = Olo + (size_t)t * qdim + (size_t)h * DH;
+#pragma unroll
+    for (int d0 = 0; d0 < DH; d0 += 8) {
+      uint16_t h8[8], l8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) split_bf16(o[d0 + j] * inv, h8[j], l8[j]);
+      *reinterpret_cast<uint4*>(dh + d0) = *reinterpret_cast<const uint4*>(h8);
+      *reinterpret_cast<uint4*>(dl + d0) = *reinterpret_cast<const uint4*>(l8);
+    }
+  }
+  // every MMA issued has completed (each was waited for) before tensor memory is freed
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTcAttnCols);
+}
+
 template <int DH, int ROWS>
 constexpr int attn_smem() {
   return (DH * ROWS + DH * (16384 / (4 * DH)) * 2 + ROWS * (16384 / (4 * DH) + 4)) * 4;
@@ -631,6 +841,7 @@ mk_status prefill_create(const Dims& D, const mk_weights* w, int chunk, PrefillP
                                attn_smem<64, kAttnRowsWide>()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pf_attn<64, true, kAttnRowsWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                attn_smem<64, kAttnRowsWide>()) == cudaSuccess;
+    ok &= cudaFuncSetAttribute(pf_attn_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, kTcAttnSmem) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pf_attn<128, false, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                attn_smem<128, kAttnRowsMin>()) == cudaSuccess;
     ok &= cudaFuncSetAttribute(pf_attn<128, true, kAttnRowsMin>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -690,7 +901,11 @@ mk_status prefill_run(PrefillPlan* p, const PrefillCtx& c, const int* tokens_dev
 #define MK_PF_ATTN(DH_, F16_, ROWS_)                                                                      \
   pf_attn<DH_, F16_, ROWS_><<<ag, kAttnThreads, attn_smem<DH_, ROWS_>(), st>>>(                           \
       p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages, D.Hkv, D.rep, pos, p->Ohi, p->Olo)
-      if (D.d == 64) {
+      if (D.d == 64 && !D.kv_fp16 && kTcAttnRows % D.rep == 0) {  // tensor cores
+        const int qbt = kTcAttnRows / D.rep;
+        pf_attn_tc<<<dim3(D.Hkv, (T + qbt - 1) / qbt), kTcAttnThreads, kTcAttnSmem, st>>>(
+            p->Q, T, D.qdim, c.kv, pt, l, D.n_phys_pages, D.Hkv, D.rep, pos, p->Ohi, p->Olo, g.err, g.limit_ns);
+      } else if (D.d == 64) {
         if (wide) {
           if (D.kv_fp16) MK_PF_ATTN(64, true, kAttnRowsWide);
           else MK_PF_ATTN(64, false, kAttnRowsWide);
