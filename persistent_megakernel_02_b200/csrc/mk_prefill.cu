@@ -522,21 +522,23 @@ __global__ void __launch_bounds__(kAttnThreads)
 // cache).  CTA = (kv head g, block of 128 / rep tokens, the last block first): its 128
 // query rows are the rep query heads of g for each token (row r: head g * rep + r / QB,
 // token t0 + r % QB), one row per tensor-memory lane.  Per KV page (64 positions):
-//   - all threads stage K as the B operand of S (64 key rows of 64 dims, 128-byte
-//     swizzle) and V transposed as the B operand of P.V (64 dim rows of 64 keys);
+//   - the 128 threads (one per query row) stage K as the B operand of S (64 key rows
+//     of 64 dims, 128-byte swizzle) and V transposed as the B operand of P.V (64 dim
+//     rows of 64 keys);
 //   - thread 0 issues S = Q_hi K^T + Q_lo K^T (M = 128, N = 64, K = 64: 8 MMAs) into
 //     tensor-memory columns 0..63 and commits;
-//   - warps 0-3, one query row per thread, read S back, apply the scale and the causal
-//     mask, update the row's online softmax (max m, sum l), rescale the row's output
-//     (kept in registers) and write P as bf16 high and low parts (the A operand);
-//   - thread 0 issues P.V = P_hi V + P_lo V into columns 64..127 and commits, and warps
-//     0-3 add it to their rows' outputs.
+//   - each thread reads its row of S back, applies the causal mask, updates the row's
+//     online softmax (max m, sum l), rescales the row's output (kept in registers) and
+//     writes P as bf16 high and low parts (the A operand);
+//   - thread 0 issues P.V = P_hi V + P_lo V into columns 64..127 and commits, and every
+//     thread adds it to its row's output.
+// Two CTAs share an SM (one's loads overlap the other's MMAs and softmax).
 // Q and P are split into bf16 high and low parts, so the products keep fp32-level
 // accuracy; K and V are the cache's bf16 values.  Output: o / l as bf16 high and low
 // parts [T][qdim].  Every wait is bounded (pf_wait); tensor memory is freed on every
 // exit path.
 constexpr int kTcAttnRows = 128;
-constexpr int kTcAttnThreads = 256;
+constexpr int kTcAttnThreads = 128;  // one thread per query row; two CTAs per SM
 constexpr int kTcAttnCols = 128;  // S in columns 0..63, P.V in 64..127
 constexpr uint32_t kTcAttnIdesc = idesc_bf16(128, 64);
 constexpr int kTcAttnSmem = 1024 + 2 * 16384 + 8192 + 8192 + 2 * 16384 + 64;
@@ -546,7 +548,7 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int col) {
   return (uint32_t)((row >> 3) * 1024 + (row & 7) * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2);
 }
 
-__global__ void __launch_bounds__(kTcAttnThreads, 1)
+__global__ void __launch_bounds__(kTcAttnThreads, 2)
     pf_attn_tc(const float* __restrict__ Q, int T, int qdim, const uint16_t* __restrict__ kv,
                const int* __restrict__ pt, int layer, int n_phys_pages, int Hkv, int rep, int pos0,
                uint16_t* __restrict__ Ohi, uint16_t* __restrict__ Olo, uint32_t* err, unsigned long long limit_ns) {
@@ -676,7 +678,7 @@ __global__ void __launch_bounds__(kTcAttnThreads, 1)
       for (int d = 0; d < DH; ++d) o[d] *= corr;
       fence_proxy_async_smem();
       tc_fence_before();
-      asm volatile("bar.sync 1, 128;" ::: "memory");  // warps 0-3: every row's P is written
+      asm volatile("bar.sync 1, 128;" ::: "memory");  // every row's P is written
       tc_fence_after();
       if (tid == 0 && ok) {
         const uint32_t a0 = smem_u32(phi), a1 = smem_u32(plo), b = smem_u32(vt);
