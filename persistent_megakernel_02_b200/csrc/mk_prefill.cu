@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(kTcAttnThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tslot;
 
-  // this thread's query row (warps 0-3: tensor-memory lane = row)
+  // this thread's query row (tensor-memory lane = row = thread)
   const int row = tid;                 // meaningful for tid < 128
   const int qt = t0 + row % QB;
   const bool rv = tid < kTcAttnRows && qt < T;
@@ -635,7 +635,7 @@ __global__ void __launch_bounds__(kTcAttnThreads, 2)
       }
       umma_commit(sdone);
     }
-    if (warp < 4) {
+    if (warp < 4) {  // every warp (128 threads): one query row per thread
       ok = __all_sync(0xFFFFFFFFu, ok && pf_wait(sdone, pg & 1, err, limit_ns, 11));
       tc_fence_after();
       float sv[PL];
@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(kTcAttnThreads, 2)
         }
       }
     }
-    // the tiles are free once P.V has read them (warps 0-3 saw it complete)
+    // the tiles are free once P.V has read them (every thread saw it complete)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
