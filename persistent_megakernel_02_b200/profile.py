@@ -179,10 +179,15 @@ def markdown(s: dict, bench_us: float | None = None) -> str:
             out.append(f"| attn | {ph.get('attn', 0):.2f} | {d['wait_us_mean']:.2f} | - | - | - | "
                        f"{d['work_us_mean']:.2f} (work) | - | - | - | - | - |")
             continue
+        # tensor-core units record no per-page dot products (the MMAs run asynchronously)
+        # and their pages' slot waits are not timed by the producer
+        tc = op.endswith("_tc")
+        core = "-" if tc else f"{d['c_core_us_per_page']:.2f}"
+        slot = "-" if tc else f"{d['p_wait_us_per_page']:.2f}"
         out.append(f"| {op} | {ph.get(op, 0):.2f} | {d['wait_us_mean']:.2f} | {d['stage_us_mean']:.2f} | "
                    f"{d['w_entry_us_mean']:.2f} | {d['w_first_us_mean']:.2f} | {d['units_us_mean']:.2f} | "
-                   f"{d['c_core_us_per_page']:.2f} | {d['c_epi_us_per_page']:.2f} | "
-                   f"{d['c_wait_us_per_page']:.2f} | {d['p_wait_us_per_page']:.2f} | "
+                   f"{core} | {d['c_epi_us_per_page']:.2f} | "
+                   f"{d['c_wait_us_per_page']:.2f} | {slot} | "
                    f"{d['pages_per_instr_mean']:.2f} |")
     out.append("")
     out.append("| layer | op | first start | last start | last end |")
