@@ -226,6 +226,18 @@ def test_plan_check_rejects_an_unknown_region():
     assert mk.lib().mk_plan_check(ctypes.byref(c), 148, 1, 0, 0, 0, 5, ctypes.byref(rep)) == 1
 
 
+def test_default_tensor_core_units_are_gate_up_and_lm_head():
+    """The measured default (tensor_core_units 0) runs gate/up and the LM head as
+    tensor-core units with 5-8 lanes, and nothing with 1-4 lanes: its tapes equal the
+    explicit selections."""
+    cfg = configs.model_config("llama1b_bs8")
+    keys = ("n_instr_total", "bytes_min_sm", "bytes_max_sm")
+    pick = lambda nb, u: tuple(mk.plan_check(cfg, 148, nb, tensor_core_units=u)[k] for k in keys)
+    assert pick(8, 0) == pick(8, 4) != pick(8, 1)
+    assert pick(5, 0) == pick(5, 4)
+    assert pick(4, 0) == pick(4, 1)
+
+
 def test_gate_up_blocks_stay_out_of_the_cumulative_balance():
     """The 128 gate/up tensor-core blocks (32 pages each, fewer than the SMs) must not
     tilt the other phases: the SMs that hold one carry its 32 pages on top of an even
